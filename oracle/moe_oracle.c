@@ -1,0 +1,226 @@
+/*
+ * moe_oracle.c -- plain, slow CPU reference of one top-k MoE SwiGLU layer forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or call this
+ * file; only the tests, the smoke check and the benchmark's CPU-baseline leg do.  It
+ * shares no code with the CUDA library (no headers, helpers or tables).
+ *
+ * Precision: the inputs are bf16 bit patterns, widened exactly to double; every sum,
+ * exp and product below is in double, with no intermediate rounding.
+ *
+ * Sources (page title, section, equation):
+ *   "MoE" (llm.rainlin.net), section 2 "Router":   r = x W_r^T;  p_t = Softmax(r_t);
+ *        I_t = TopK(p_t, K);  alpha_{t,e} = p_{t,e} / sum_{j in I_t} p_{t,j}.
+ *   "MoE", section 3:  E_e(x) = W_down (SiLU(W_gate x) (.) W_up x), gate_up weights
+ *        stored as one [2f, D] matrix whose first f rows are the gate and last f the up
+ *        projection (the expert loop splits F.linear's output in two halves).
+ *   "MoE", section 4:  y_t = sum_{e in I_t} alpha_{t,e} E_e(x_t)
+ *                            + sigma(w_s^T x_t) E_s(x_t)   (shared expert, optional).
+ *   "1.6 混合专家（MoE）" (llm.satori-ai.cn), section 2 worked example: the selected
+ *        scores are renormalised among the selected experts only (0.90, 0.60 -> 0.60,
+ *        0.40); the unselected experts never enter the forward pass.
+ *
+ * Readings where the pages are silent: the router logits are not rounded (fp32 or
+ * better); top-K ties go to the lower expert index and the selected indices are listed
+ * by descending probability; the renormalisation has no epsilon; the shared-expert gate
+ * has no bias.  An optional per-expert logit bias b (added to r before the softmax)
+ * expresses the synthetic routing regimes.
+ *
+ * Build: gcc -O2 -ffp-contract=off -fopenmp -shared -fPIC moe_oracle.c -lm
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+static double bf16_to_double(uint16_t bits) {
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static double dot_bf16(const uint16_t* a, const uint16_t* b, int n) {
+    double s = 0.0;
+    for (int i = 0; i < n; ++i) s += bf16_to_double(a[i]) * bf16_to_double(b[i]);
+    return s;
+}
+
+static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
+
+static double silu(double z) { return z * sigmoid(z); }
+
+/*
+ * Router ("MoE", section 2).  For each token t:
+ *   r_t[e]  = x_t . W_r[e]  (+ bias[e])
+ *   p_t     = softmax(r_t)                       (max-subtracted, double)
+ *   I_t     = the K largest p_t[e]; ties -> lower e; listed by descending p
+ *   alpha   = p_t[I_t] / sum p_t[I_t]
+ *   gap[t]  = p_(K) - p_(K+1)  (K-th minus (K+1)-th largest probability; +inf if K == E)
+ *   sgate[t]= sigma(w_s . x_t)                   (shared-expert scalar gate, section 4)
+ * Outputs idx [T*K], alpha [T*K]; probs [T*E], gap [T], sgate [T] are optional (NULL).
+ * Returns 0, or -1 on bad arguments.
+ */
+int oracle_route(const uint16_t* x, const uint16_t* w_r, const double* bias,
+                 const uint16_t* w_sg, int T, int D, int E, int K,
+                 int32_t* idx, double* alpha, double* probs, double* gap, double* sgate) {
+    if (T < 0 || D <= 0 || E <= 0 || K <= 0 || K > E) return -1;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int t = 0; t < T; ++t) {
+        double* p = (double*)malloc(sizeof(double) * (size_t)E);
+        char* taken = (char*)calloc((size_t)E, 1);
+        if (!p || !taken) { bad = 1; free(p); free(taken); continue; }
+        const uint16_t* xt = x + (size_t)t * D;
+        double m = -INFINITY;
+        for (int e = 0; e < E; ++e) {
+            p[e] = dot_bf16(xt, w_r + (size_t)e * D, D) + (bias ? bias[e] : 0.0);
+            if (p[e] > m) m = p[e];
+        }
+        double z = 0.0;
+        for (int e = 0; e < E; ++e) { p[e] = exp(p[e] - m); z += p[e]; }
+        for (int e = 0; e < E; ++e) p[e] /= z;
+        if (probs) memcpy(probs + (size_t)t * E, p, sizeof(double) * (size_t)E);
+
+        /* TopK by repeated selection of the largest remaining probability. */
+        double sel_sum = 0.0;
+        for (int k = 0; k < K; ++k) {
+            int best = -1;
+            for (int e = 0; e < E; ++e)
+                if (!taken[e] && (best < 0 || p[e] > p[best])) best = e;
+            taken[best] = 1;
+            idx[(size_t)t * K + k] = best;
+            sel_sum += p[best];
+        }
+        for (int k = 0; k < K; ++k)
+            alpha[(size_t)t * K + k] = p[idx[(size_t)t * K + k]] / sel_sum;
+        if (gap) {
+            double next = -INFINITY;
+            for (int e = 0; e < E; ++e)
+                if (!taken[e] && p[e] > next) next = p[e];
+            gap[t] = (K == E) ? INFINITY : p[idx[(size_t)t * K + K - 1]] - next;
+        }
+        if (sgate) sgate[t] = w_sg ? sigmoid(dot_bf16(xt, w_sg, D)) : 0.0;
+        free(p);
+        free(taken);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * One SwiGLU expert applied to one token ("MoE", section 3), accumulated with a weight:
+ *   acc += a * W_down (SiLU(W_gate x) (.) W_up x)
+ * w_gu is the expert's [2f, D] gate_up matrix (gate rows first), w_d its [D, f] down
+ * matrix.  h is caller scratch of f doubles.
+ */
+static void expert_accumulate(const uint16_t* xt, const uint16_t* w_gu, const uint16_t* w_d,
+                              int D, int f, double a, double* h, double* acc) {
+    for (int n = 0; n < f; ++n) {
+        double g = dot_bf16(xt, w_gu + (size_t)n * D, D);
+        double u = dot_bf16(xt, w_gu + (size_t)(f + n) * D, D);
+        h[n] = silu(g) * u;
+    }
+    for (int d = 0; d < D; ++d) {
+        const uint16_t* row = w_d + (size_t)d * f;
+        double s = 0.0;
+        for (int n = 0; n < f; ++n) s += bf16_to_double(row[n]) * h[n];
+        acc[d] += a * s;
+    }
+}
+
+/*
+ * Sparse layer output ("MoE", section 4) for the listed tokens:
+ *   y[i] = sum_k alpha[t,k] E_{idx[t,k]}(x_t)  (+ sgate[t] E_s(x_t) when w_s_gu != NULL)
+ * with t = tokens[i] (or t = i when tokens == NULL).  Expert e's weights are
+ * w_gu + e*2f*D and w_d + e*D*f, so callers may pass a compacted weight set with idx
+ * renumbered into it.  Output y is [ntok, D] double.
+ */
+int oracle_experts(const uint16_t* x, const int32_t* idx, const double* alpha,
+                   const uint16_t* w_gu, const uint16_t* w_d,
+                   const uint16_t* w_s_gu, const uint16_t* w_s_d, const double* sgate,
+                   int D, int E, int K, int f, int f_s,
+                   const int32_t* tokens, int ntok, double* y) {
+    if (D <= 0 || E <= 0 || K <= 0 || f <= 0 || ntok < 0) return -1;
+    if (w_s_gu && (!w_s_d || !sgate || f_s <= 0)) return -1;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < ntok; ++i) {
+        int t = tokens ? tokens[i] : i;
+        int hn = (w_s_gu && f_s > f) ? f_s : f;
+        double* h = (double*)malloc(sizeof(double) * (size_t)hn);
+        if (!h) { bad = 1; continue; }
+        double* acc = y + (size_t)i * D;
+        for (int d = 0; d < D; ++d) acc[d] = 0.0;
+        const uint16_t* xt = x + (size_t)t * D;
+        for (int k = 0; k < K; ++k) {
+            int e = idx[(size_t)t * K + k];
+            if (e < 0 || e >= E) { bad = 1; continue; }
+            expert_accumulate(xt, w_gu + (size_t)e * 2 * f * D, w_d + (size_t)e * D * f,
+                              D, f, alpha[(size_t)t * K + k], h, acc);
+        }
+        if (w_s_gu) expert_accumulate(xt, w_s_gu, w_s_d, D, f_s, sgate[t], h, acc);
+        free(h);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * Dense-masked layer output, the brute-force form of the same sum: every one of the E
+ * experts is evaluated on every token and weighted by dense_alpha[t,e] (zero for the
+ * experts outside I_t).  Unselected experts contribute exactly nothing, so this equals
+ * oracle_experts when dense_alpha scatters the sparse alpha ("1.6 混合专家（MoE）",
+ * section 2: the weighting acts on each expert's output vector).  y is [T, D] double.
+ */
+int oracle_dense_masked(const uint16_t* x, const double* dense_alpha,
+                        const uint16_t* w_gu, const uint16_t* w_d,
+                        const uint16_t* w_s_gu, const uint16_t* w_s_d, const double* sgate,
+                        int T, int D, int E, int f, int f_s, double* y) {
+    if (T < 0 || D <= 0 || E <= 0 || f <= 0) return -1;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int t = 0; t < T; ++t) {
+        int hn = (w_s_gu && f_s > f) ? f_s : f;
+        double* h = (double*)malloc(sizeof(double) * (size_t)hn);
+        if (!h) { bad = 1; continue; }
+        double* acc = y + (size_t)t * D;
+        for (int d = 0; d < D; ++d) acc[d] = 0.0;
+        const uint16_t* xt = x + (size_t)t * D;
+        for (int e = 0; e < E; ++e)
+            expert_accumulate(xt, w_gu + (size_t)e * 2 * f * D, w_d + (size_t)e * D * f,
+                              D, f, dense_alpha[(size_t)t * E + e], h, acc);
+        if (w_s_gu) expert_accumulate(xt, w_s_gu, w_s_d, D, f_s, sgate[t], h, acc);
+        free(h);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * Token permutation: group the T*K (token, slot) pairs by expert ("MoE", section 3.2:
+ * each routed expert gathers the tokens routed to it; "1.6 混合专家（MoE）", section 2:
+ * tokens are first grouped by their routes).  Plain definition: walk the experts in
+ * order, and for each expert walk the tokens in ascending order and their slots.
+ *   counts[e]          rows of expert e
+ *   offsets[e]         first row of expert e (offsets[E] = T*K)
+ *   sorted_token[row]  token of that row
+ *   sorted_slot[row]   t*K + k of that row
+ *   slot_to_row[t*K+k] row of that pair (the inverse map)
+ */
+int oracle_permute(const int32_t* idx, int T, int E, int K, int32_t* counts, int32_t* offsets,
+                   int32_t* sorted_token, int32_t* sorted_slot, int32_t* slot_to_row) {
+    if (T < 0 || E <= 0 || K <= 0) return -1;
+    int32_t row = 0;
+    for (int e = 0; e < E; ++e) {
+        offsets[e] = row;
+        for (int t = 0; t < T; ++t)
+            for (int k = 0; k < K; ++k)
+                if (idx[(size_t)t * K + k] == e) {
+                    sorted_token[row] = t;
+                    sorted_slot[row] = t * K + k;
+                    slot_to_row[(size_t)t * K + k] = row;
+                    ++row;
+                }
+        counts[e] = row - offsets[e];
+    }
+    offsets[E] = row;
+    return row == T * K ? 0 : -1;
+}
