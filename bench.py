@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Throughput of one top-k MoE SwiGLU layer forward on B200 GPUs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one whole layer call (router, permutation, gather, grouped gate_up + SwiGLU,
+grouped down + weighted combine, bf16 output) over one batch of synthetic tokens already
+resident in HBM.  L2 is flushed (512 MiB write) before every timed step, outside the timed
+interval; each step is timed with CUDA events recorded by the library on its own stream,
+and the per-kernel intervals come from the same events.  With N > 1 (torchrun, one
+process per GPU) every rank runs an independent replica of the batch (no exchange): the
+reported value is all ranks' tokens over the slowest rank's time.
+
+``--impl reference`` times the CPU oracle (fp64, OpenMP) on this host instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/s on 1 B200 and % of roofline (HBM GB/s or bf16 TC util)"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 512 << 20
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+
+
+# ---------------------------------------------------------------- accounting
+
+
+def describe(cfg) -> str:
+    s = f"{cfg.name}: T={cfg.T} D={cfg.D} E={cfg.E} K={cfg.K} f={cfg.f}"
+    if cfg.f_s:
+        s += f" f_s={cfg.f_s}"
+    return s + f" routing={cfg.routing}"
+
+
+def layer_flops(cfg) -> float:
+    """2*3*D*f per routed (token, expert) row, 2*3*D*f_s per token for the shared expert,
+    plus the router's 2*D*E per token."""
+    return 6.0 * cfg.D * cfg.f * cfg.T * cfg.K + 6.0 * cfg.D * cfg.f_s * cfg.T + \
+        2.0 * cfg.T * cfg.D * cfg.E
+
+
+def layer_bytes(cfg, U: int) -> float:
+    """bf16 weights of the U experts hit (+ shared, + router), x in, y out."""
+    return 2.0 * 3 * cfg.D * cfg.f * U + 2.0 * 3 * cfg.D * cfg.f_s + 2.0 * cfg.E * cfg.D + \
+        4.0 * cfg.T * cfg.D
+
+
+def gate_up_bytes(cfg, U: int) -> float:
+    """Algorithmic bytes of one grouped gate_up launch: gate+up weights of the U experts
+    hit, the T*K gathered token rows read, the T*K x f SwiGLU rows written."""
+    rows = cfg.T * cfg.K
+    return 2.0 * 2 * cfg.D * cfg.f * U + 2.0 * rows * cfg.D + 2.0 * rows * cfg.f
+
+
+def gate_up_flops(cfg) -> float:
+    return 4.0 * cfg.D * cfg.f * cfg.T * cfg.K
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("grouped_gemm.cu", "ptx.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "top_routing_grouped_03_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """dram read+write bytes per launch from the committed ncu summary of this kernel and
+    workload, or None when absent or taken on a different kernel source."""
+    path = os.path.join(PROFILE_DIR, f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path, encoding="utf-8") as fh:
+        for line in fh:
+            if line.startswith("- ") and ":" in line:
+                k, v = line[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha256") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = [l.strip().split(", ") for l in self.tmp.read().splitlines() if l.strip()]
+        self.tmp.close()
+        os.unlink(self.tmp.name)
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+
+def oracle_step(inp, tokens):
+    import numpy as np
+
+    import oracle
+    r = oracle.route(inp.x, inp.w_router, inp.cfg.K, inp.logit_bias, inp.w_shared_gate)
+    toks = np.asarray(tokens, np.int32)
+    oracle.experts(inp.x, r["idx"], r["alpha"], inp.w_gate_up, inp.w_down, toks,
+                   inp.w_shared_gate_up, inp.w_shared_down, r["shared_gate"])
+    return len(toks)
+
+
+def cpu_baseline(inp, budget_s=10.0):
+    """The oracle as it stands on this host's cores: the whole batch (router over every
+    token, expert sum for every token), repeated until ~budget_s of work."""
+    import oracle
+    oracle.build()
+    T = inp.cfg.T
+    n, t0 = 0, time.perf_counter()
+    reps = 0
+    while True:
+        n += oracle_step(inp, range(T))
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": UNIT, "cores": int(os.environ.get("OMP_NUM_THREADS", "1")),
+            "kind": "oracle",
+            "sample": f"the full {T}-token batch (router + expert sum, fp64) x {reps}, {dt:.1f} s"}
+
+
+def run_reference(args, cfg, world, rank):
+    if rank != 0:
+        return 0
+    import workloads
+    inp = workloads.make_inputs(cfg)
+    import oracle
+    oracle.build()
+    t1 = time.perf_counter()
+    oracle_step(inp, [0])
+    per_tok = max(time.perf_counter() - t1, 1e-3)
+    budget = 90.0  # seconds for the whole warmup + timed run
+    ntok = int(max(1, min(cfg.T, budget / (args.steps + args.warmup) / per_tok)))
+    toks = list(range(ntok))
+    for _ in range(args.warmup):
+        oracle_step(inp, toks)
+    t0 = time.perf_counter()
+    n = 0
+    for _ in range(args.steps):
+        n += oracle_step(inp, toks)
+    dt = time.perf_counter() - t0
+    value = n / dt
+    cores = int(os.environ.get("OMP_NUM_THREADS", "1"))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": describe(cfg), "tokens_per_step": ntok},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{ntok} token(s) per step: router over all {cfg.T} tokens "
+                                   f"+ expert sum of the sampled tokens, fp64"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default="decode")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--deterministic", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    os.environ.setdefault("OMP_NUM_THREADS", str(os.cpu_count() or 1))
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    import workloads
+    cfg = workloads.CONFIGS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, cfg, world, rank)
+
+    import torch
+    import torch.distributed as dist
+
+    import top_routing_grouped_03_b200 as moe
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    big = cfg.T * cfg.D * cfg.E > (1 << 31)
+    inp = workloads.make_inputs(cfg, device=dev if big else "cpu").to(dev)
+    layer = moe.MoELayer.from_inputs(inp, deterministic=args.deterministic)
+    T, K, E = cfg.T, cfg.K, cfg.E
+    out = torch.empty((T, cfg.D), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((T, K), dtype=torch.int32, device=dev)
+    tw = torch.empty((T, K), dtype=torch.float32, device=dev)
+    counts = torch.empty((E,), dtype=torch.int32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def events():
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(moe.NUM_STEP_EVENTS)]
+        for e in evs:
+            e.record(stream)  # creates the handle; the library re-records it
+        return evs
+
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        layer(inp.x, out=out, topk_idx=idx, topk_w=tw, counts=counts)
+    torch.cuda.synchronize()
+    if layer.device_status() != 0:
+        raise RuntimeError("device status after warm-up is not ok")
+
+    step_evs = [events() for _ in range(args.steps)]
+    arrs = [moe.event_array(e) for e in step_evs]
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}")
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = moe.launch_count()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        layer(inp.x, out=out, topk_idx=idx, topk_w=tw, counts=counts, step_events=arrs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = moe.launch_count() - n0
+    clocks = sampler.stop()
+    if layer.device_status() != 0:
+        raise RuntimeError("device status after the timed steps is not ok")
+
+    names = moe.STEP_EVENT_NAMES
+    per_kernel = {n: 0.0 for n in names[1:-1]}
+    total_ms = 0.0
+    for evs in step_evs:
+        total_ms += evs[0].elapsed_time(evs[-1])
+        for j, n in enumerate(names[1:-1], start=1):
+            per_kernel[n] += evs[j].elapsed_time(evs[j + 1])
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * T * args.steps / (total_ms / 1e3)
+
+    # ---- end to end through the public API: pinned host x in, pinned host y out
+    x_host = inp.x.cpu().pin_memory()
+    y_host = torch.empty((T, cfg.D), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(inp.x)
+    for i in range(args.warmup):
+        layer.forward_host(x_host, y_host, x_dev, out)
+    e_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e_a[i].record(stream)
+        layer.forward_host(x_host, y_host, x_dev, out)
+        e_b[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in zip(e_a, e_b))
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+        dist.destroy_process_group()
+    e2e = {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+           "d2h_bytes_per_step": y_host.numel() * y_host.element_size()}
+
+    if rank != 0:
+        return 0
+
+    cnt = counts.cpu()
+    U = int((cnt > 0).sum())
+    peaks, peak_src = load_peaks()
+    gu_ms = per_kernel["gate_up"] / args.steps
+    gu_bytes = gate_up_bytes(cfg, U)
+    achieved_gbs = gu_bytes / (gu_ms / 1e3) / 1e9
+    traffic = ncu_traffic("grouped_gemm_gate_up", cfg.name)
+    F, B = layer_flops(cfg), layer_bytes(cfg, U)
+    t_roof = max(F / (peaks["bf16_tflops"] * 1e12), B / (peaks["hbm_gbs"] * 1e9))
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": describe(cfg), "global_batch": world * T, "tokens_per_gpu": T,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "flushed before every timed step (512 MiB write); expert weights read per "
+                  "step exceed L2",
+            "routing_U": U, "max_rows_per_expert": int(cnt.max()),
+            "deterministic_combine": bool(args.deterministic),
+        },
+        "roofline": {
+            "bound": "hbm", "kernel": "grouped_gemm gate_up + SwiGLU",
+            "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
+            "algorithmic_bytes_per_launch": gu_bytes, "avg_launch_ms": gu_ms,
+            "peak_source": f"{peak_src} (hbm_gbs)",
+        },
+        "layer_roofline": {
+            "flops": F, "bytes": B, "t_roof_ms": 1e3 * t_roof,
+            "frac": 1e3 * t_roof / ms_per_step,
+            "achieved_tflops": F / (ms_per_step / 1e3) / 1e12,
+            "achieved_gbs": B / (ms_per_step / 1e3) / 1e9,
+        },
+        "kernel_ms": {n: v / args.steps for n, v in per_kernel.items()},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        cpu_inp = inp.to("cpu")
+        line["cpu_baseline"] = cpu_baseline(cpu_inp)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,222 @@
+/*
+ * moe_api.h -- C ABI of libmoe_b200.so: the forward pass of one top-k Mixture-of-Experts
+ * SwiGLU FFN layer on one NVIDIA B200 (sm_100a).
+ *
+ * The layer (page "MoE", llm.rainlin.net, sections 2-4):
+ *   r_t      = x_t W_r^T (+ b)                         router logits, fp32 accumulate
+ *   p_t      = Softmax(r_t)                            fp32
+ *   I_t      = TopK(p_t, K)
+ *   alpha_te = p_te / sum_{j in I_t} p_tj              renormalised routing weights
+ *   E_e(x)   = W_down^e (SiLU(W_gate^e x) (.) W_up^e x)
+ *   y_t      = sum_{e in I_t} alpha_te E_e(x_t) + sigma(w_s^T x_t) E_s(x_t)
+ * The shared expert term is optional.  The residual add h + y of the decoder layer is
+ * not part of this library.
+ *
+ * Conventions that hold for every entry point:
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise.  The caller
+ *     allocates and owns every buffer, including the workspace; the library never
+ *     allocates, frees or synchronises.  All work is enqueued on `stream` (a
+ *     cudaStream_t passed as void*; NULL is the legacy default stream) and returns
+ *     before it completes.
+ *   - bf16 tensors are raw bf16 bit patterns (moe_bf16), row-major and contiguous.
+ *     Matrix base pointers must be 16-byte aligned (MOE_ERR_ALIGN otherwise).
+ *   - Arguments are checked on the host before anything is launched; a negative
+ *     status means nothing was enqueued.  MOE_ERR_CUDA means a launch failed.
+ *   - Device-side problems (an inconsistent routing table, a wait that ran out of its
+ *     time budget) are recorded in a status word inside the workspace; read it with
+ *     moe_read_device_status().
+ *   - Supported shapes: 1 <= E <= 512, 1 <= K <= min(E, 16), D and f multiples of 128,
+ *     128 <= D <= 8192, 128 <= f <= 8192, f_s = 0 or a multiple of 128 up to 8192,
+ *     T >= 0 and T*K < 2^31.  Others return MOE_ERR_UNSUPPORTED.
+ *   - Calls that share a workspace must not overlap on the GPU (same stream, or
+ *     ordered by events).
+ */
+#ifndef MOE_API_H
+#define MOE_API_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef uint16_t moe_bf16; /* bf16 bit pattern */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_ARG = -1,         /* null pointer, negative size, inconsistent arguments */
+    MOE_ERR_UNSUPPORTED = -2, /* shape outside the supported set */
+    MOE_ERR_ALIGN = -3,       /* a matrix pointer is not 16-byte aligned */
+    MOE_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed */
+    MOE_ERR_TIMEOUT = -5,     /* device status only: a device wait ran out of its budget */
+    MOE_ERR_WORKSPACE = -6,   /* workspace pointer null or smaller than required */
+    MOE_ERR_DEVICE = -7       /* device status only: inconsistent routing table seen */
+} moe_status;
+
+/* Flags of moe_layer_params.flags. */
+#define MOE_FLAG_DETERMINISTIC 1u /* combine by a fixed-order gather instead of fp32 atomics */
+
+/* Human-readable name of a status code (static string). */
+MOE_API const char* moe_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+MOE_API int moe_version(void);
+
+/*
+ * Bytes of device workspace that moe_layer_forward needs for this shape (it also covers
+ * moe_route and moe_grouped_swiglu with the same or smaller sizes).  f_s = 0 when there
+ * is no shared expert.  Returns 0 for unsupported shapes.  The workspace must be 256-byte
+ * aligned; its contents need no initialisation.
+ */
+MOE_API size_t moe_workspace_size(int T, int D, int E, int K, int f, int f_s);
+
+/*
+ * Router: logits, fp32 softmax, TopK and renormalisation ("MoE", section 2, router
+ * equations; "1.6 混合专家（MoE）", section 2, renormalisation worked example).
+ *   x            [T, D] bf16 tokens
+ *   w_router     [E, D] bf16 router weight W_r (no bias)
+ *   logit_bias   [E] fp32 added to the logits before the softmax, or NULL
+ *   w_shared_gate[D] bf16 shared-expert gate vector w_s, or NULL
+ * Outputs (device, caller-owned):
+ *   topk_idx     [T, K] int32 selected experts, by descending probability; ties go to
+ *                the lower expert index
+ *   topk_w       [T, K] fp32 renormalised weights alpha (sum to 1 per token)
+ *   expert_counts[E] int32 rows routed to each expert (overwritten, not accumulated)
+ *   shared_gate  [T] fp32 sigma(w_s . x_t); required iff w_shared_gate != NULL
+ * The logits are accumulated in fp32 and never rounded to bf16.  Since the softmax is
+ * monotone and its denominator cancels in the renormalisation, the selection is made on
+ * the logits and alpha_k = exp(r_k - r_max) / sum_{j in I} exp(r_j - r_max).
+ * workspace: at least moe_workspace_size(T, D, E, K, 128, 0) bytes.
+ */
+MOE_API int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* logit_bias,
+              const moe_bf16* w_shared_gate, int T, int D, int E, int K,
+              int32_t* topk_idx, float* topk_w, int32_t* expert_counts, float* shared_gate,
+              void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Permutation: group the T*K (token, slot) pairs by expert ("MoE", section 3.2: each
+ * routed expert gathers the tokens routed to it).  Row order inside a group is by
+ * ascending token (stable).
+ *   topk_idx [T, K] int32, topk_w [T, K] fp32 (NULL: sorted_w not written),
+ *   expert_counts [E] int32 (as written by moe_route)
+ * Outputs:
+ *   expert_offsets [E+1] int32: rows of expert e are [offsets[e], offsets[e+1]);
+ *                  offsets[E] = T*K
+ *   sorted_token   [T*K] int32 token of each row
+ *   sorted_w       [T*K] fp32 routing weight of each row (ignored if topk_w is NULL)
+ *   slot_to_row    [T*K] int32 row of pair t*K+k (the inverse map)
+ * Counts that disagree with topk_idx set MOE_ERR_DEVICE in the device status word of
+ * `workspace` when it is not NULL.
+ */
+MOE_API int moe_permute(const int32_t* topk_idx, const float* topk_w, const int32_t* expert_counts,
+                int T, int E, int K, int32_t* expert_offsets, int32_t* sorted_token,
+                float* sorted_w, int32_t* slot_to_row, void* workspace, void* stream);
+
+/*
+ * Grouped SwiGLU experts ("MoE", section 3 expert equation and section 3.2 expert loop):
+ * for every group e and every row r in [offsets[e], offsets[e+1]) with token
+ * t = sorted_token[r]:
+ *   h_r = SiLU(W_gate^e x_t) (.) (W_up^e x_t)            bf16, fp32 accumulate
+ *   v_r = W_down^e h_r                                    fp32 accumulate
+ * and then, with w_r = sorted_w[r] (1 when sorted_w is NULL):
+ *   out_acc[t, :] += w_r * v_r     (fp32 atomics; out_acc is NOT cleared), and/or
+ *   y_sorted[r, :] = bf16(w_r * v_r)
+ * At least one of out_acc / y_sorted must be non-NULL.
+ *   x            [T, D] bf16
+ *   sorted_token [rows] int32, or NULL for the identity (row r is token r, rows <= T)
+ *   expert_offsets [E+1] int32 on the device; offsets[E] = rows
+ *   w_gate_up    [E, 2f, D] bf16: rows [0,f) gate, [f,2f) up of each expert
+ *   w_down       [E, D, f] bf16
+ * `rows` is the number of sorted rows (T*K for routed experts; T for a dense expert
+ * given as E = 1, identity tokens and offsets {0, T}).
+ * workspace: at least moe_workspace_size(T, D, E, K, f, 0) bytes with K = rows / T
+ * rounded up (holds the gathered token rows and h).
+ */
+MOE_API int moe_grouped_swiglu(const moe_bf16* x, const int32_t* sorted_token,
+                       const int32_t* expert_offsets, const float* sorted_w,
+                       const moe_bf16* w_gate_up, const moe_bf16* w_down,
+                       int T, int rows, int D, int E, int f,
+                       moe_bf16* y_sorted, float* out_acc,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Combine back to token order ("MoE", section 4 aggregation; the expert loop's weighted
+ * index_add):
+ *   out[t, :] = bf16( acc[t, :] + sum_k w_tk * y_sorted[slot_to_row[t*K+k], :]
+ *                     + shared_gate[t] * shared_out[t, :] )
+ * Every term is optional: out_acc (fp32 [T, D]) NULL -> acc = 0; y_sorted (bf16 [T*K, D])
+ * NULL -> no routed sum; topk_w NULL -> w = 1 (y_sorted already weighted); shared_out
+ * (bf16 [T, D]) NULL -> no shared term.  The k-sum runs in slot order (deterministic).
+ */
+MOE_API int moe_combine(const float* out_acc, const moe_bf16* y_sorted, const int32_t* slot_to_row,
+                const float* topk_w, const moe_bf16* shared_out, const float* shared_gate,
+                int T, int D, int K, moe_bf16* out, void* stream);
+
+/* Every input of one layer call. */
+typedef struct moe_layer_params {
+    const moe_bf16* x;                /* [T, D] */
+    const moe_bf16* w_router;         /* [E, D] */
+    const float* logit_bias;          /* [E] or NULL */
+    const moe_bf16* w_gate_up;        /* [E, 2f, D] */
+    const moe_bf16* w_down;           /* [E, D, f] */
+    const moe_bf16* w_shared_gate;    /* [D] or NULL (no shared expert) */
+    const moe_bf16* w_shared_gate_up; /* [2 f_s, D] or NULL */
+    const moe_bf16* w_shared_down;    /* [D, f_s] or NULL */
+    int T, D, E, K, f, f_s;           /* f_s = 0: no shared expert */
+    unsigned flags;                   /* MOE_FLAG_* */
+    int32_t* topk_idx_out;            /* optional [T, K] copy of the routing, or NULL */
+    float* topk_w_out;                /* optional [T, K], or NULL */
+    int32_t* expert_counts_out;       /* optional [E], or NULL */
+    void* const* step_events;         /* optional: MOE_NUM_STEP_EVENTS cudaEvent_t handles */
+} moe_layer_params;
+
+/*
+ * Step boundaries at which moe_layer_forward records p->step_events[i] on its stream when
+ * step_events is not NULL (events created by the caller; used to time each kernel of the
+ * layer).  Steps absent from a call (no shared expert) get a zero-length interval.
+ */
+enum {
+    MOE_EV_START = 0,    /* before the workspace clears */
+    MOE_EV_ROUTER,       /* router kernel */
+    MOE_EV_PERMUTE,      /* permutation kernel */
+    MOE_EV_GATHER,       /* gather of token rows into expert order */
+    MOE_EV_GATE_UP,      /* grouped gate_up GEMM + SwiGLU */
+    MOE_EV_DOWN,         /* grouped down GEMM + weighted scatter */
+    MOE_EV_SHARED,       /* shared expert (gate_up and down) */
+    MOE_EV_COMBINE,      /* combine / bf16 output */
+    MOE_EV_END,
+    MOE_NUM_STEP_EVENTS
+};
+
+/*
+ * The whole layer: route, permute, grouped SwiGLU (routed experts and, when present, the
+ * shared expert scaled by sigma(w_s . x)), combine to out [T, D] bf16.  No host
+ * synchronisation; every step reads its sizes from the device, so the call can be
+ * captured in a CUDA graph.  workspace: at least moe_workspace_size(T, D, E, K, f, f_s)
+ * bytes, 256-byte aligned.
+ */
+MOE_API int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
+                      size_t ws_bytes, void* stream);
+
+/* Kernels this library has launched in this process so far (all devices, all calls). */
+MOE_API unsigned long long moe_launch_count(void);
+
+/*
+ * Synchronously reads (and clears) the device status word of a workspace after the
+ * work on `stream` completes: MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE.  This call
+ * synchronises `stream`; it is a diagnostic, not part of the layer.
+ */
+MOE_API int moe_read_device_status(void* workspace, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_API_H */

@@ -1,0 +1,264 @@
+"""top_routing_grouped_03_b200 -- one top-k MoE SwiGLU FFN layer forward on a B200.
+
+A thin ctypes binding over ``libmoe_b200.so`` (C ABI in ``include/moe_api.h``).  Every
+step of the layer runs in the library's sm_100a kernels; this module only allocates
+tensors with PyTorch, passes their device pointers and the current CUDA stream, and turns
+status codes into exceptions.  There is no fallback: without the built library (or on a
+machine without a CUDA device) the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe_api.h")
+
+MOE_FLAG_DETERMINISTIC = 1
+
+_lib = None
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+
+
+class LayerParams(ctypes.Structure):
+    _fields_ = [
+        ("x", ctypes.c_void_p), ("w_router", ctypes.c_void_p), ("logit_bias", ctypes.c_void_p),
+        ("w_gate_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
+        ("w_shared_gate", ctypes.c_void_p), ("w_shared_gate_up", ctypes.c_void_p),
+        ("w_shared_down", ctypes.c_void_p),
+        ("T", ctypes.c_int), ("D", ctypes.c_int), ("E", ctypes.c_int), ("K", ctypes.c_int),
+        ("f", ctypes.c_int), ("f_s", ctypes.c_int), ("flags", ctypes.c_uint),
+        ("topk_idx_out", ctypes.c_void_p), ("topk_w_out", ctypes.c_void_p),
+        ("expert_counts_out", ctypes.c_void_p), ("step_events", ctypes.c_void_p),
+    ]
+
+
+# Step boundaries recorded by moe_layer_forward when step_events is given.
+STEP_EVENT_NAMES = ("start", "router", "permute", "gather", "gate_up", "down", "shared",
+                    "combine", "end")
+NUM_STEP_EVENTS = len(STEP_EVENT_NAMES)
+
+
+def lib() -> ctypes.CDLL:
+    """Load the C library (built in-tree by ``build.build()`` / ``__graft_entry__.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m top_routing_grouped_03_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.moe_status_string.argtypes = [I]
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_version.argtypes = []
+        L.moe_version.restype = I
+        L.moe_workspace_size.argtypes = [I, I, I, I, I, I]
+        L.moe_workspace_size.restype = Z
+        L.moe_route.argtypes = [P, P, P, P, I, I, I, I, P, P, P, P, P, Z, P]
+        L.moe_route.restype = I
+        L.moe_permute.argtypes = [P, P, P, I, I, I, P, P, P, P, P, P]
+        L.moe_permute.restype = I
+        L.moe_grouped_swiglu.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P, P, Z, P]
+        L.moe_grouped_swiglu.restype = I
+        L.moe_combine.argtypes = [P, P, P, P, P, P, I, I, I, P, P]
+        L.moe_combine.restype = I
+        L.moe_layer_forward.argtypes = [ctypes.POINTER(LayerParams), P, P, Z, P]
+        L.moe_layer_forward.restype = I
+        L.moe_read_device_status.argtypes = [P, P]
+        L.moe_read_device_status.restype = I
+        L.moe_launch_count.argtypes = []
+        L.moe_launch_count.restype = ctypes.c_ulonglong
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().moe_status_string(int(code)).decode()
+
+
+def version() -> int:
+    return lib().moe_version()
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise MoEError(rc, what)
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def workspace_size(T: int, D: int, E: int, K: int, f: int, f_s: int = 0) -> int:
+    return int(lib().moe_workspace_size(T, D, E, K, f, f_s))
+
+
+def alloc_workspace(T, D, E, K, f, f_s=0, device=None) -> torch.Tensor:
+    n = workspace_size(T, D, E, K, f, f_s)
+    if n == 0:
+        raise MoEError(-2, "moe_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def route(x, w_router, K, logit_bias=None, w_shared_gate=None, workspace=None, stream=None):
+    """Router step.  Returns (topk_idx [T,K] int32, topk_w [T,K] f32, expert_counts [E]
+    int32, shared_gate [T] f32 or None)."""
+    T, D = x.shape
+    E = w_router.shape[0]
+    dev = x.device
+    ws = workspace if workspace is not None else alloc_workspace(T, D, E, K, 128, 0, dev)
+    idx = torch.empty((T, K), dtype=torch.int32, device=dev)
+    w = torch.empty((T, K), dtype=torch.float32, device=dev)
+    counts = torch.empty((E,), dtype=torch.int32, device=dev)
+    sg = torch.empty((T,), dtype=torch.float32, device=dev) if w_shared_gate is not None else None
+    rc = lib().moe_route(_p(x), _p(w_router), _p(logit_bias), _p(w_shared_gate), T, D, E, K,
+                         _p(idx), _p(w), _p(counts), _p(sg), _p(ws), ws.numel(), _stream(stream))
+    _check(rc, "moe_route")
+    return idx, w, counts, sg
+
+
+def permute(topk_idx, topk_w, expert_counts, E, workspace=None, stream=None):
+    """Permutation step.  Returns dict(offsets [E+1], sorted_token, sorted_w, slot_to_row)."""
+    T, K = topk_idx.shape
+    dev = topk_idx.device
+    off = torch.empty((E + 1,), dtype=torch.int32, device=dev)
+    st = torch.empty((T * K,), dtype=torch.int32, device=dev)
+    sw = torch.empty((T * K,), dtype=torch.float32, device=dev) if topk_w is not None else None
+    s2r = torch.empty((T * K,), dtype=torch.int32, device=dev)
+    rc = lib().moe_permute(_p(topk_idx), _p(topk_w), _p(expert_counts), T, E, K, _p(off),
+                           _p(st), _p(sw), _p(s2r), _p(workspace), _stream(stream))
+    _check(rc, "moe_permute")
+    return dict(offsets=off, sorted_token=st, sorted_w=sw, slot_to_row=s2r)
+
+
+def grouped_swiglu(x, sorted_token, offsets, sorted_w, w_gate_up, w_down, rows,
+                   out_acc=None, y_sorted=None, workspace=None, stream=None):
+    """Grouped SwiGLU experts over the sorted rows; writes out_acc (+=) and/or y_sorted."""
+    T, D = x.shape
+    E, twof, _ = w_gate_up.shape
+    f = twof // 2
+    if workspace is None:
+        Kr = max(1, -(-rows // max(T, 1)))
+        workspace = alloc_workspace(max(T, 1), D, E, min(Kr, E, 16), f, 0, x.device)
+    rc = lib().moe_grouped_swiglu(_p(x), _p(sorted_token), _p(offsets), _p(sorted_w),
+                                  _p(w_gate_up), _p(w_down), T, rows, D, E, f, _p(y_sorted),
+                                  _p(out_acc), _p(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "moe_grouped_swiglu")
+
+
+def combine(T, D, K, out=None, out_acc=None, y_sorted=None, slot_to_row=None, topk_w=None,
+            shared_out=None, shared_gate=None, device=None, stream=None):
+    dev = device or "cuda"
+    out = out if out is not None else torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+    rc = lib().moe_combine(_p(out_acc), _p(y_sorted), _p(slot_to_row), _p(topk_w),
+                           _p(shared_out), _p(shared_gate), T, D, K, _p(out), _stream(stream))
+    _check(rc, "moe_combine")
+    return out
+
+
+def launch_count() -> int:
+    """Kernels launched by the library in this process so far."""
+    return int(lib().moe_launch_count())
+
+
+def event_array(events):
+    """ctypes array of raw cudaEvent_t handles of recorded ``torch.cuda.Event`` objects."""
+    assert len(events) == NUM_STEP_EVENTS
+    arr = (ctypes.c_void_p * NUM_STEP_EVENTS)()
+    for i, e in enumerate(events):
+        if not e.cuda_event:
+            raise ValueError("record each event once before passing it (creates the handle)")
+        arr[i] = e.cuda_event
+    return arr
+
+
+def read_device_status(workspace, stream=None) -> int:
+    return int(lib().moe_read_device_status(_p(workspace), _stream(stream)))
+
+
+class MoELayer:
+    """One MoE layer with resident weights and a reusable workspace.
+
+    ``layer(x)`` runs moe_layer_forward on the current stream and returns y [T, D] bf16.
+    """
+
+    def __init__(self, w_router, w_gate_up, w_down, K, logit_bias=None, w_shared_gate=None,
+                 w_shared_gate_up=None, w_shared_down=None, deterministic=False):
+        self.w_router, self.w_gate_up, self.w_down = w_router, w_gate_up, w_down
+        self.logit_bias = logit_bias
+        self.w_shared_gate, self.w_shared_gate_up = w_shared_gate, w_shared_gate_up
+        self.w_shared_down = w_shared_down
+        self.E, self.D = w_router.shape
+        self.f = w_gate_up.shape[1] // 2
+        self.f_s = 0 if w_shared_gate_up is None else w_shared_gate_up.shape[0] // 2
+        self.K = K
+        self.flags = MOE_FLAG_DETERMINISTIC if deterministic else 0
+        self._ws = None
+        self._ws_T = -1
+
+    @classmethod
+    def from_inputs(cls, inp, deterministic=False):
+        return cls(inp.w_router, inp.w_gate_up, inp.w_down, inp.cfg.K, inp.logit_bias,
+                   inp.w_shared_gate, inp.w_shared_gate_up, inp.w_shared_down, deterministic)
+
+    def workspace(self, T: int) -> torch.Tensor:
+        if self._ws is None or self._ws_T < T:
+            self._ws = alloc_workspace(T, self.D, self.E, self.K, self.f, self.f_s,
+                                       self.w_router.device)
+            self._ws_T = T
+        return self._ws
+
+    def params(self, x, topk_idx=None, topk_w=None, counts=None, events=None) -> LayerParams:
+        T = x.shape[0]
+        ev = None if events is None else ctypes.cast(events, ctypes.c_void_p)
+        return LayerParams(_p(x), _p(self.w_router), _p(self.logit_bias), _p(self.w_gate_up),
+                           _p(self.w_down), _p(self.w_shared_gate), _p(self.w_shared_gate_up),
+                           _p(self.w_shared_down), T, self.D, self.E, self.K, self.f, self.f_s,
+                           self.flags, _p(topk_idx), _p(topk_w), _p(counts), ev)
+
+    def __call__(self, x, out=None, topk_idx=None, topk_w=None, counts=None, stream=None,
+                 step_events=None):
+        """y = layer(x) on the device.  ``step_events``: an ``event_array(...)`` to time
+        each kernel of the call."""
+        T = x.shape[0]
+        if x.shape[1] != self.D:
+            raise MoEError(-1, "moe_layer_forward (x has the wrong width)")
+        out = out if out is not None else torch.empty((T, self.D), dtype=torch.bfloat16,
+                                                      device=x.device)
+        ws = self.workspace(T)
+        prm = self.params(x, topk_idx, topk_w, counts, step_events)
+        rc = lib().moe_layer_forward(ctypes.byref(prm), _p(out), _p(ws), ws.numel(),
+                                     _stream(stream))
+        _check(rc, "moe_layer_forward")
+        return out
+
+    def forward_host(self, x_host, y_host, x_dev, y_dev, stream=None):
+        """End to end from host memory: copy x (pinned host) in, run the layer, copy y
+        out to pinned host memory; everything enqueued on one stream."""
+        x_dev.copy_(x_host, non_blocking=True)
+        self(x_dev, out=y_dev, stream=stream)
+        y_host.copy_(y_dev, non_blocking=True)
+        return y_host
+
+    def device_status(self, stream=None) -> int:
+        return read_device_status(self._ws, stream) if self._ws is not None else 0

@@ -1,0 +1,106 @@
+// common.cuh -- types and small helpers shared by the kernels of libmoe_b200.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/moe_api.h"
+
+namespace moe {
+
+using bf16 = __nv_bfloat16;
+
+// Records the first device-side error in the status word (later errors are dropped).
+__device__ __forceinline__ void set_status(int* status, int code) {
+    if (status != nullptr) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t packed) {
+    return __uint_as_float(packed << 16);
+}
+
+__device__ __forceinline__ float bf16_hi(uint32_t packed) {
+    return __uint_as_float(packed & 0xFFFF0000u);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Host-side count of kernel launches issued by the library (read by moe_launch_count).
+void count_launches(unsigned n);
+
+// ---------------------------------------------------------------- kernel launchers
+// (defined in the .cu files, called by the C entry points in moe_api.cu)
+
+struct RouterLaunch {
+    const bf16* x;
+    const bf16* w_router;
+    const float* logit_bias;
+    const bf16* w_shared_gate;
+    int T, D, E, K;
+    float* logits;        // [T, E+1] workspace
+    unsigned* counters;   // [ceil(T/8)] workspace, zeroed before the launch
+    int32_t* topk_idx;
+    float* topk_w;
+    int32_t* counts;      // zeroed before the launch
+    float* shared_gate;
+    int* status;
+};
+cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s);
+
+struct PermuteLaunch {
+    const int32_t* topk_idx;
+    const float* topk_w;
+    const int32_t* counts;
+    int T, E, K;
+    int32_t* offsets;
+    int32_t* sorted_token;
+    float* sorted_w;
+    int32_t* slot_to_row;
+    int32_t* dense_offsets;  // optional [2] = {0, T} for a dense (shared) expert group
+    int* status;
+};
+cudaError_t launch_permute(const PermuteLaunch& a, cudaStream_t s);
+
+struct GatherLaunch {
+    const bf16* x;
+    const int32_t* sorted_token;
+    int rows, D;
+    bf16* x_sorted;
+};
+cudaError_t launch_gather(const GatherLaunch& a, int num_sms, cudaStream_t s);
+
+struct GroupedGemmLaunch {
+    bool gate_up;               // true: SiLU(gate)*up epilogue -> h; false: down epilogue
+    const void* w;              // weights: gate_up [E, 2f, D] or down [E, D, f]
+    const void* act;            // activations in row order: x_sorted [rows, D] or h [rows, f]
+    const int32_t* offsets;     // [E+1]
+    const int32_t* sorted_token;  // down only; NULL = identity
+    const float* sorted_w;      // down only; NULL = 1
+    int rows, E, D, f;
+    bf16* h_out;                // gate_up: [rows, f]
+    float* acc_out;             // down: [T, D] scatter-add target or NULL
+    bf16* y_out;                // down: [rows, D] or NULL
+    int* status;
+};
+cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s);
+
+struct CombineLaunch {
+    const float* out_acc;
+    const bf16* y_sorted;
+    const int32_t* slot_to_row;
+    const float* topk_w;
+    const bf16* shared_out;
+    const float* shared_gate;
+    int T, D, K;
+    bf16* out;
+};
+cudaError_t launch_combine(const CombineLaunch& a, int num_sms, cudaStream_t s);
+
+}  // namespace moe

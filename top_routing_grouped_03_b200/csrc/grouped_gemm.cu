@@ -1,0 +1,409 @@
+// grouped_gemm.cu -- grouped SwiGLU expert GEMMs on tcgen05 tensor cores.
+//
+// "MoE" (llm.rainlin.net), section 3: E_e(x) = W_down (SiLU(W_gate x) (.) W_up x), the
+// gate_up weight of an expert is one [2f, D] matrix (gate rows, then up rows); section
+// 3.2: the routed output is scaled by the routing weight and index-added back to its
+// token.  "MoE 到底省了什么" (clxhxhhr.top), section 3: with few rows per expert the
+// layer is bound by reading the expert weights, with many rows it is bound by compute.
+//
+// Both projections run through one persistent, warp-specialised kernel template:
+//   * operand A = 128 weight rows x 64 K (TMA, 128-byte swizzle) -- the MMA's M side,
+//     so an expert with only a couple of rows still fills the 128-lane tensor-core tile
+//     ("swap-AB": weights on M, tokens on N);
+//   * operand B = BN rows of activations in expert order x 64 K (TMA);
+//   * D = fp32 accumulator in tensor memory, 128 lanes (features) x BN columns (rows);
+//     the gate_up kernel keeps the gate block in columns [0, BN) and the up block in
+//     [BN, 2BN) so one thread holds gate and up of the same feature;
+//   * two accumulator buffers so the epilogue of one tile overlaps the MMAs of the next.
+// Warp 0 issues TMA loads into a STAGES-deep ring, warp 1 issues tcgen05.mma (one
+// thread) and owns the TMEM allocation, warps 2-5 drain TMEM (tcgen05.ld) and run the
+// epilogue: h = SiLU(g) * u -> bf16 for gate_up; w * v -> fp32 red.add into the token's
+// output row (and/or bf16 y_sorted) for down.
+// The work list (group, feature block, row block) is derived on the device from the
+// group offsets, so no host synchronisation is needed.  Every wait is bounded.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kBM = 128;          // weight rows per tile (MMA M)
+constexpr int kBK = 64;           // K per stage: one 128-byte swizzle row of bf16
+constexpr int kThreads = 192;     // 6 warps
+constexpr int kEpiThreads = 128;  // warps 2..5
+constexpr int kMaxGroups = 1024;
+
+__host__ __device__ constexpr int pow2_at_least(int v) {
+    int p = 32;
+    while (p < v) p <<= 1;
+    return p;
+}
+
+template <int BN, bool GATE_UP>
+struct Cfg {
+    static constexpr int kNumA = GATE_UP ? 2 : 1;
+    static constexpr int kABytes = kBM * kBK * 2;
+    static constexpr int kBBytes = BN * kBK * 2;
+    static constexpr int kStageBytes = kNumA * kABytes + kBBytes;
+    static constexpr int kStages0 = (200 * 1024) / kStageBytes;
+    static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
+    static constexpr int kAccCols = GATE_UP ? 2 * BN : BN;
+    static constexpr int kTmemCols = pow2_at_least(2 * kAccCols);
+    static_assert(kTmemCols <= 512, "accumulators exceed tensor memory");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128");
+    static_assert(kStageBytes % 1024 == 0, "stage buffers must keep 1024-byte alignment");
+};
+
+struct Params {
+    const int32_t* offsets;
+    const int32_t* sorted_token;
+    const float* sorted_w;
+    int G;             // groups
+    int nf;            // feature blocks (of 128 weight rows) per group
+    int nk;            // K steps of 64
+    int w_group_rows;  // weight rows per group in the 2-D weight view (2f or D)
+    int up_rows;       // gate_up: offset of the up rows inside a group (f)
+    int out_cols;      // gate_up: f (h row length); down: D (output row length)
+    bf16* h_out;
+    float* acc_out;
+    bf16* y_out;
+    int* status;
+};
+
+struct Tile {
+    int g, i, row0, row_end;
+};
+
+__device__ __forceinline__ Tile decode_tile(int tile, const int* g_tile, const int* g_off, int G,
+                                            int BN) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (g_tile[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    Tile t;
+    t.g = lo;
+    const int n = g_off[lo + 1] - g_off[lo];
+    const int nb = (n + BN - 1) / BN;
+    const int local = tile - g_tile[lo];
+    t.i = local / nb;
+    const int j = local - t.i * nb;
+    t.row0 = g_off[lo] + j * BN;
+    t.row_end = g_off[lo + 1];
+    return t;
+}
+
+template <int BN, bool GATE_UP>
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
+                    const __grid_constant__ CUtensorMap map_act, Params p) {
+    using C = Cfg<BN, GATE_UP>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+    uint64_t* empty = full + C::kStages;
+    uint64_t* tfull = empty + C::kStages;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* total_slot = reinterpret_cast<int*>(tmem_slot + 2);
+    int* g_off = reinterpret_cast<int*>(tmem_slot + 4);
+    int* g_tile = g_off + (p.G + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], kEpiThreads);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&map_w);
+        tma_prefetch_desc(&map_act);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    for (int i = threadIdx.x; i <= p.G; i += kThreads) g_off[i] = p.offsets[i];
+    __syncthreads();
+    if (warp == 2) {
+        // tile prefix over groups: lane l owns a contiguous run of groups
+        const int per = (p.G + 31) / 32;
+        const int gb = min(lane * per, p.G), ge = min(gb + per, p.G);
+        int local = 0;
+        for (int g = gb; g < ge; ++g) local += ((g_off[g + 1] - g_off[g] + BN - 1) / BN) * p.nf;
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - local;
+        for (int g = gb; g < ge; ++g) {
+            g_tile[g] = run;
+            run += ((g_off[g + 1] - g_off[g] + BN - 1) / BN) * p.nf;
+        }
+        if (lane == 31) {
+            g_tile[p.G] = incl;
+            *total_slot = incl;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = *total_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            const uint64_t pol_w = policy_evict_first();  // weights stream through once
+            const uint64_t pol_a = policy_evict_last();   // activations are re-read
+            int stage = 0;
+            uint32_t phase = 0, filled = 0, fill_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const Tile t = decode_tile(tile, g_tile, g_off, p.G, BN);
+                const int wr0 = t.g * p.w_group_rows + t.i * kBM;
+                for (int kk = 0; kk < p.nk; ++kk) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, kWaitBudgetNs, abort_flag)) {
+                        set_status(p.status, MOE_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+                    uint8_t* st = smem + stage * C::kStageBytes;
+                    tma_load_2d(st, &map_w, &full[stage], kk * kBK, wr0, pol_w);
+                    if (GATE_UP)
+                        tma_load_2d(st + C::kABytes, &map_w, &full[stage], kk * kBK,
+                                    wr0 + p.up_rows, pol_w);
+                    tma_load_2d(st + C::kNumA * C::kABytes, &map_act, &full[stage], kk * kBK,
+                                t.row0, pol_a);
+                    filled |= 1u << stage;
+                    fill_phase = (fill_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok) {  // let the copies already in flight land before the CTA exits
+                for (int s = 0; s < C::kStages; ++s)
+                    if (filled & (1u << s))
+                        mbar_wait(&full[s], (fill_phase >> s) & 1u, kDrainBudgetNs, nullptr);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
+            int stage = 0;
+            uint32_t phase = 0, abuf = 0, aphase = 0;
+            bool ok = true, issued = false;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                if (!mbar_wait(&tempty[abuf], aphase ^ 1u, kWaitBudgetNs, abort_flag)) {
+                    set_status(p.status, MOE_ERR_TIMEOUT);
+                    *abort_flag = 1;
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + abuf * C::kAccCols;
+                for (int kk = 0; kk < p.nk; ++kk) {
+                    if (!mbar_wait(&full[stage], phase, kWaitBudgetNs, abort_flag)) {
+                        set_status(p.status, MOE_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
+                    const uint32_t a1 = a0 + C::kABytes;
+                    const uint32_t b0 = a0 + C::kNumA * C::kABytes;
+#pragma unroll
+                    for (int s = 0; s < kBK / 16; ++s) {
+                        const uint32_t acc = (kk | s) != 0 ? 1u : 0u;
+                        const uint64_t bd = sdesc_k_sw128(b0 + s * 32);
+                        umma_bf16(d0, sdesc_k_sw128(a0 + s * 32), bd, idesc, acc);
+                        if (GATE_UP) umma_bf16(d0 + BN, sdesc_k_sw128(a1 + s * 32), bd, idesc, acc);
+                    }
+                    issued = true;
+                    umma_commit(&empty[stage]);
+                    if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                umma_commit(&tfull[abuf]);
+                abuf ^= 1u;
+                if (abuf == 0) aphase ^= 1u;
+            }
+            if (!ok && issued) {  // the MMAs still read shared memory: wait for them
+                umma_commit(drain);
+                mbar_wait(drain, 0, kDrainBudgetNs, nullptr);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- epilogue
+        const int q = warp & 3;  // tensor-memory lane quarter this warp may read
+        const int feat_in_tile = q * 32 + lane;
+        uint32_t abuf = 0, aphase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const Tile t = decode_tile(tile, g_tile, g_off, p.G, BN);
+            if (!mbar_wait(&tfull[abuf], aphase, kWaitBudgetNs, abort_flag)) {
+                set_status(p.status, MOE_ERR_TIMEOUT);
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   abuf * C::kAccCols;
+            const int feat = t.i * kBM + feat_in_tile;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                uint32_t gv[16];
+                uint32_t uv[16];
+                tmem_ld16(tbase + c0, gv);
+                if (GATE_UP) tmem_ld16(tbase + BN + c0, uv);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const int row = t.row0 + c0 + c;
+                    if (row >= t.row_end) break;
+                    const float g = __uint_as_float(gv[c]);
+                    if (GATE_UP) {
+                        const float u = __uint_as_float(uv[c]);
+                        const float h = g / (1.f + __expf(-g)) * u;
+                        p.h_out[static_cast<size_t>(row) * p.out_cols + feat] = __float2bfloat16_rn(h);
+                    } else {
+                        const float w = p.sorted_w ? __ldg(p.sorted_w + row) : 1.f;
+                        const float v = w * g;
+                        if (p.acc_out) {
+                            const int tok = p.sorted_token ? __ldg(p.sorted_token + row) : row;
+                            red_add_f32(p.acc_out + static_cast<size_t>(tok) * p.out_cols + feat, v);
+                        }
+                        if (p.y_out)
+                            p.y_out[static_cast<size_t>(row) * p.out_cols + feat] = __float2bfloat16_rn(v);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[abuf]);
+            abuf ^= 1u;
+            if (abuf == 0) aphase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+cudaError_t get_encoder() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode ? cudaSuccess : cudaErrorNotSupported;
+}
+
+// 2-D bf16 view [rows, cols] (cols contiguous), box [box_rows, 64], 128-byte swizzle.
+cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, int box_rows) {
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int BN, bool GATE_UP>
+cudaError_t launch_tpl(const CUtensorMap& mw, const CUtensorMap& ma, const Params& p, int grid,
+                       cudaStream_t s) {
+    using C = Cfg<BN, GATE_UP>;
+    const size_t smem = 1024 + static_cast<size_t>(C::kStages) * C::kStageBytes +
+                        (2 * C::kStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int);
+    auto kfn = grouped_gemm_kernel<BN, GATE_UP>;
+    cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    kfn<<<grid, kThreads, smem, s>>>(mw, ma, p);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int pick_block_rows(int rows, int groups) {
+    const int avg = rows / (groups > 0 ? groups : 1);
+    if (avg <= 16) return 16;
+    if (avg <= 32) return 32;
+    if (avg <= 64) return 64;
+    return 128;
+}
+
+cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s) {
+    if (a.rows == 0 || a.E == 0) return cudaSuccess;
+    if (a.E > kMaxGroups) return cudaErrorInvalidValue;
+    cudaError_t err = get_encoder();
+    if (err != cudaSuccess) return err;
+    const int BN = pick_block_rows(a.rows, a.E);
+    const int K = a.gate_up ? a.D : a.f;
+    const uint64_t w_group_rows = a.gate_up ? 2ull * a.f : static_cast<uint64_t>(a.D);
+    CUtensorMap mw, ma;
+    if ((err = make_map(&mw, a.w, w_group_rows * a.E, K, kBM)) != cudaSuccess) return err;
+    if ((err = make_map(&ma, a.act, a.rows, K, BN)) != cudaSuccess) return err;
+    Params p{};
+    p.offsets = a.offsets;
+    p.sorted_token = a.sorted_token;
+    p.sorted_w = a.sorted_w;
+    p.G = a.E;
+    p.nf = (a.gate_up ? a.f : a.D) / kBM;
+    p.nk = K / kBK;
+    p.w_group_rows = static_cast<int>(w_group_rows);
+    p.up_rows = a.f;
+    p.out_cols = a.gate_up ? a.f : a.D;
+    p.h_out = a.h_out;
+    p.acc_out = a.acc_out;
+    p.y_out = a.y_out;
+    p.status = a.status;
+    const long long max_tiles = (static_cast<long long>(ceil_div(a.rows, BN)) + a.E) * p.nf;
+    const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
+    switch (BN) {
+        case 16: return a.gate_up ? launch_tpl<16, true>(mw, ma, p, grid, s) : launch_tpl<16, false>(mw, ma, p, grid, s);
+        case 32: return a.gate_up ? launch_tpl<32, true>(mw, ma, p, grid, s) : launch_tpl<32, false>(mw, ma, p, grid, s);
+        case 64: return a.gate_up ? launch_tpl<64, true>(mw, ma, p, grid, s) : launch_tpl<64, false>(mw, ma, p, grid, s);
+        default: return a.gate_up ? launch_tpl<128, true>(mw, ma, p, grid, s) : launch_tpl<128, false>(mw, ma, p, grid, s);
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,392 @@
+// moe_api.cu -- the extern "C" entry points of libmoe_b200.so: argument checks on the
+// host, workspace layout, and the launch sequence of the layer.  See include/moe_api.h.
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+
+namespace moe {
+
+std::atomic<unsigned long long> g_launches{0};
+void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxDevices = 64;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms_current() {
+    static int cache[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+// Workspace of the whole layer.  The status word is always at offset 0.
+struct Layout {
+    size_t status, counters, counts, logits, offsets, dense_offsets, topk_idx, topk_w, sgate,
+        sorted_token, sorted_w, slot_to_row, x_sorted, h, h_s, out_acc, y_sorted, total;
+    size_t zero_end;  // [0, zero_end) is cleared at the start of a layer call
+};
+
+Layout layout(long long T, long long D, long long E, long long K, long long f, long long fs) {
+    Layout L{};
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t r = o;
+        o = align_up(o + bytes);
+        return r;
+    };
+    L.status = take(kAlign);
+    L.counters = take(sizeof(unsigned) * static_cast<size_t>((T + 7) / 8));
+    L.counts = take(sizeof(int32_t) * E);
+    L.zero_end = o;
+    L.logits = take(sizeof(float) * T * (E + 1));
+    L.offsets = take(sizeof(int32_t) * (E + 1));
+    L.dense_offsets = take(sizeof(int32_t) * 2);
+    L.topk_idx = take(sizeof(int32_t) * T * K);
+    L.topk_w = take(sizeof(float) * T * K);
+    L.sgate = take(sizeof(float) * T);
+    L.sorted_token = take(sizeof(int32_t) * T * K);
+    L.sorted_w = take(sizeof(float) * T * K);
+    L.slot_to_row = take(sizeof(int32_t) * T * K);
+    L.x_sorted = take(2 * T * K * D);
+    L.h = take(2 * T * K * f);
+    L.h_s = take(2 * T * fs);
+    L.out_acc = take(sizeof(float) * T * D);
+    L.y_sorted = take(2 * T * K * D);
+    L.total = o;
+    return L;
+}
+
+int check_shape(int T, int D, int E, int K, int f, int fs) {
+    if (T < 0 || D <= 0 || E <= 0 || K <= 0 || f <= 0 || fs < 0) return MOE_ERR_ARG;
+    if (E > 512 || K > 16 || K > E) return MOE_ERR_UNSUPPORTED;
+    if (D % 128 || D > 8192 || f % 128 || f > 8192 || fs % 128 || fs > 8192)
+        return MOE_ERR_UNSUPPORTED;
+    if (static_cast<long long>(T) * K >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+template <class P>
+P* at(void* ws, size_t off) {
+    return reinterpret_cast<P*>(static_cast<uint8_t*>(ws) + off);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(int status) {
+    switch (status) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+        case MOE_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case MOE_ERR_CUDA: return "CUDA launch failed";
+        case MOE_ERR_TIMEOUT: return "device wait timed out";
+        case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+        case MOE_ERR_DEVICE: return "inconsistent routing table on the device";
+        default: return "unknown status";
+    }
+}
+
+int moe_version(void) { return 100; }
+
+unsigned long long moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+size_t moe_workspace_size(int T, int D, int E, int K, int f, int f_s) {
+    if (check_shape(T, D, E, K, f, f_s) != MOE_OK) return 0;
+    return layout(T, D, E, K, f, f_s).total;
+}
+
+int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* logit_bias,
+              const moe_bf16* w_shared_gate, int T, int D, int E, int K, int32_t* topk_idx,
+              float* topk_w, int32_t* expert_counts, float* shared_gate, void* workspace,
+              size_t ws_bytes, void* stream) {
+    int rc = check_shape(T, D, E, K, 128, 0);
+    if (rc) return rc;
+    if (!w_router || !expert_counts) return MOE_ERR_ARG;
+    if (T > 0 && (!x || !topk_idx || !topk_w || (w_shared_gate && !shared_gate))) return MOE_ERR_ARG;
+    if (!aligned16(x) || !aligned16(w_router) || (w_shared_gate && !aligned16(w_shared_gate)))
+        return MOE_ERR_ALIGN;
+    const Layout L = layout(T, D, E, K, 128, 0);
+    if (!workspace) return MOE_ERR_WORKSPACE;
+    if (ws_bytes < L.logits + sizeof(float) * static_cast<size_t>(T) * (E + 1)) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = as_stream(stream);
+    if (cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * E, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (T == 0) return MOE_OK;
+    if (cudaMemsetAsync(workspace, 0, L.counts, s) != cudaSuccess) return MOE_ERR_CUDA;
+    RouterLaunch a{};
+    a.x = reinterpret_cast<const bf16*>(x);
+    a.w_router = reinterpret_cast<const bf16*>(w_router);
+    a.logit_bias = logit_bias;
+    a.w_shared_gate = reinterpret_cast<const bf16*>(w_shared_gate);
+    a.T = T; a.D = D; a.E = E; a.K = K;
+    a.logits = at<float>(workspace, L.logits);
+    a.counters = at<unsigned>(workspace, L.counters);
+    a.topk_idx = topk_idx;
+    a.topk_w = topk_w;
+    a.counts = expert_counts;
+    a.shared_gate = shared_gate;
+    a.status = at<int>(workspace, L.status);
+    return launch_router(a, num_sms_current(), s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_permute(const int32_t* topk_idx, const float* topk_w, const int32_t* expert_counts, int T,
+                int E, int K, int32_t* expert_offsets, int32_t* sorted_token, float* sorted_w,
+                int32_t* slot_to_row, void* workspace, void* stream) {
+    int rc = check_shape(T, 128, E, K, 128, 0);
+    if (rc) return rc;
+    if (!expert_counts || !expert_offsets) return MOE_ERR_ARG;
+    if (T > 0 && (!topk_idx || !sorted_token || !slot_to_row || (topk_w && !sorted_w)))
+        return MOE_ERR_ARG;
+    PermuteLaunch a{};
+    a.topk_idx = topk_idx;
+    a.topk_w = topk_w;
+    a.counts = expert_counts;
+    a.T = T; a.E = E; a.K = K;
+    a.offsets = expert_offsets;
+    a.sorted_token = sorted_token;
+    a.sorted_w = sorted_w;
+    a.slot_to_row = slot_to_row;
+    a.status = workspace ? at<int>(workspace, 0) : nullptr;
+    return launch_permute(a, as_stream(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_grouped_swiglu(const moe_bf16* x, const int32_t* sorted_token,
+                       const int32_t* expert_offsets, const float* sorted_w,
+                       const moe_bf16* w_gate_up, const moe_bf16* w_down, int T, int rows, int D,
+                       int E, int f, moe_bf16* y_sorted, float* out_acc, void* workspace,
+                       size_t ws_bytes, void* stream) {
+    int rc = check_shape(T, D, E, 1, f, 0);
+    if (rc) return rc;
+    if (rows < 0 || (T == 0 && rows > 0)) return MOE_ERR_ARG;
+    if (!sorted_token && rows > T) return MOE_ERR_ARG;
+    if (!x || !expert_offsets || !w_gate_up || !w_down || (!y_sorted && !out_acc)) return MOE_ERR_ARG;
+    if (!aligned16(x) || !aligned16(w_gate_up) || !aligned16(w_down) ||
+        (y_sorted && !aligned16(y_sorted)))
+        return MOE_ERR_ALIGN;
+    if (!workspace) return MOE_ERR_WORKSPACE;
+    const size_t xs_off = kAlign;
+    const size_t h_off = align_up(xs_off + 2ull * rows * D);
+    const size_t need = align_up(h_off + 2ull * rows * f);
+    if (ws_bytes < need) return MOE_ERR_WORKSPACE;
+    if (rows == 0) return MOE_OK;
+    cudaStream_t s = as_stream(stream);
+    const int sms = num_sms_current();
+    int* status = at<int>(workspace, 0);
+    const bf16* act = reinterpret_cast<const bf16*>(x);
+    if (sorted_token) {
+        GatherLaunch g{reinterpret_cast<const bf16*>(x), sorted_token, rows, D,
+                       at<bf16>(workspace, xs_off)};
+        if (launch_gather(g, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+        act = at<bf16>(workspace, xs_off);
+    }
+    GroupedGemmLaunch up{};
+    up.gate_up = true;
+    up.w = w_gate_up;
+    up.act = act;
+    up.offsets = expert_offsets;
+    up.rows = rows; up.E = E; up.D = D; up.f = f;
+    up.h_out = at<bf16>(workspace, h_off);
+    up.status = status;
+    if (launch_grouped_gemm(up, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    GroupedGemmLaunch dn{};
+    dn.gate_up = false;
+    dn.w = w_down;
+    dn.act = at<bf16>(workspace, h_off);
+    dn.offsets = expert_offsets;
+    dn.sorted_token = sorted_token;
+    dn.sorted_w = sorted_w;
+    dn.rows = rows; dn.E = E; dn.D = D; dn.f = f;
+    dn.acc_out = out_acc;
+    dn.y_out = reinterpret_cast<bf16*>(y_sorted);
+    dn.status = status;
+    return launch_grouped_gemm(dn, sms, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_combine(const float* out_acc, const moe_bf16* y_sorted, const int32_t* slot_to_row,
+                const float* topk_w, const moe_bf16* shared_out, const float* shared_gate, int T,
+                int D, int K, moe_bf16* out, void* stream) {
+    if (T < 0 || D <= 0 || D % 8 || K < 0) return MOE_ERR_ARG;
+    if (!out || (y_sorted && (!slot_to_row || K <= 0)) || (shared_out && !shared_gate))
+        return MOE_ERR_ARG;
+    if (!aligned16(out) || (out_acc && !aligned16(out_acc)) || (y_sorted && !aligned16(y_sorted)) ||
+        (shared_out && !aligned16(shared_out)))
+        return MOE_ERR_ALIGN;
+    CombineLaunch a{};
+    a.out_acc = out_acc;
+    a.y_sorted = reinterpret_cast<const bf16*>(y_sorted);
+    a.slot_to_row = slot_to_row;
+    a.topk_w = topk_w;
+    a.shared_out = reinterpret_cast<const bf16*>(shared_out);
+    a.shared_gate = shared_gate;
+    a.T = T; a.D = D; a.K = K;
+    a.out = reinterpret_cast<bf16*>(out);
+    return launch_combine(a, num_sms_current(), as_stream(stream)) == cudaSuccess ? MOE_OK
+                                                                                   : MOE_ERR_CUDA;
+}
+
+int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace, size_t ws_bytes,
+                      void* stream) {
+    if (!p) return MOE_ERR_ARG;
+    const int T = p->T, D = p->D, E = p->E, K = p->K, f = p->f, fs = p->f_s;
+    int rc = check_shape(T, D, E, K, f, fs);
+    if (rc) return rc;
+    const bool shared = fs > 0;
+    if (!p->x || !p->w_router || !p->w_gate_up || !p->w_down || !out) return MOE_ERR_ARG;
+    if (shared && (!p->w_shared_gate || !p->w_shared_gate_up || !p->w_shared_down)) return MOE_ERR_ARG;
+    if (!shared && (p->w_shared_gate || p->w_shared_gate_up || p->w_shared_down)) return MOE_ERR_ARG;
+    if (!aligned16(p->x) || !aligned16(p->w_router) || !aligned16(p->w_gate_up) ||
+        !aligned16(p->w_down) || !aligned16(out) ||
+        (shared && (!aligned16(p->w_shared_gate) || !aligned16(p->w_shared_gate_up) ||
+                    !aligned16(p->w_shared_down))))
+        return MOE_ERR_ALIGN;
+    if (!workspace) return MOE_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return MOE_ERR_ALIGN;
+    const Layout L = layout(T, D, E, K, f, fs);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    if (T == 0) return MOE_OK;
+
+    cudaStream_t s = as_stream(stream);
+    const int sms = num_sms_current();
+    const bool det = (p->flags & MOE_FLAG_DETERMINISTIC) != 0;
+    auto mark = [&](int i) {
+        return p->step_events == nullptr ||
+               cudaEventRecord(reinterpret_cast<cudaEvent_t>(p->step_events[i]), s) == cudaSuccess;
+    };
+    int* status = at<int>(workspace, L.status);
+    int32_t* counts = p->expert_counts_out ? p->expert_counts_out : at<int32_t>(workspace, L.counts);
+    int32_t* idx = p->topk_idx_out ? p->topk_idx_out : at<int32_t>(workspace, L.topk_idx);
+    float* tw = p->topk_w_out ? p->topk_w_out : at<float>(workspace, L.topk_w);
+    float* sgate = at<float>(workspace, L.sgate);
+    float* out_acc = at<float>(workspace, L.out_acc);
+
+    if (!mark(MOE_EV_START)) return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, L.zero_end, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (p->expert_counts_out && cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if ((!det || shared) &&
+        cudaMemsetAsync(out_acc, 0, sizeof(float) * static_cast<size_t>(T) * D, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+
+    RouterLaunch r{};
+    r.x = reinterpret_cast<const bf16*>(p->x);
+    r.w_router = reinterpret_cast<const bf16*>(p->w_router);
+    r.logit_bias = p->logit_bias;
+    r.w_shared_gate = shared ? reinterpret_cast<const bf16*>(p->w_shared_gate) : nullptr;
+    r.T = T; r.D = D; r.E = E; r.K = K;
+    r.logits = at<float>(workspace, L.logits);
+    r.counters = at<unsigned>(workspace, L.counters);
+    r.topk_idx = idx;
+    r.topk_w = tw;
+    r.counts = counts;
+    r.shared_gate = sgate;
+    r.status = status;
+    if (!mark(MOE_EV_ROUTER) || launch_router(r, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+    PermuteLaunch pm{};
+    pm.topk_idx = idx;
+    pm.topk_w = tw;
+    pm.counts = counts;
+    pm.T = T; pm.E = E; pm.K = K;
+    pm.offsets = at<int32_t>(workspace, L.offsets);
+    pm.sorted_token = at<int32_t>(workspace, L.sorted_token);
+    pm.sorted_w = at<float>(workspace, L.sorted_w);
+    pm.slot_to_row = at<int32_t>(workspace, L.slot_to_row);
+    pm.dense_offsets = at<int32_t>(workspace, L.dense_offsets);
+    pm.status = status;
+    if (!mark(MOE_EV_PERMUTE) || launch_permute(pm, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+    const int rows = T * K;
+    GatherLaunch g{reinterpret_cast<const bf16*>(p->x), pm.sorted_token, rows, D,
+                   at<bf16>(workspace, L.x_sorted)};
+    if (!mark(MOE_EV_GATHER) || launch_gather(g, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+    GroupedGemmLaunch up{};
+    up.gate_up = true;
+    up.w = p->w_gate_up;
+    up.act = g.x_sorted;
+    up.offsets = pm.offsets;
+    up.rows = rows; up.E = E; up.D = D; up.f = f;
+    up.h_out = at<bf16>(workspace, L.h);
+    up.status = status;
+    if (!mark(MOE_EV_GATE_UP) || launch_grouped_gemm(up, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+    GroupedGemmLaunch dn{};
+    dn.gate_up = false;
+    dn.w = p->w_down;
+    dn.act = up.h_out;
+    dn.offsets = pm.offsets;
+    dn.sorted_token = pm.sorted_token;
+    dn.sorted_w = det ? nullptr : pm.sorted_w;
+    dn.rows = rows; dn.E = E; dn.D = D; dn.f = f;
+    dn.acc_out = det ? nullptr : out_acc;
+    dn.y_out = det ? at<bf16>(workspace, L.y_sorted) : nullptr;
+    dn.status = status;
+    if (!mark(MOE_EV_DOWN) || launch_grouped_gemm(dn, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+    if (!mark(MOE_EV_SHARED)) return MOE_ERR_CUDA;
+    if (shared) {
+        GroupedGemmLaunch su{};
+        su.gate_up = true;
+        su.w = p->w_shared_gate_up;
+        su.act = p->x;
+        su.offsets = pm.dense_offsets;
+        su.rows = T; su.E = 1; su.D = D; su.f = fs;
+        su.h_out = at<bf16>(workspace, L.h_s);
+        su.status = status;
+        if (launch_grouped_gemm(su, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+        GroupedGemmLaunch sd{};
+        sd.gate_up = false;
+        sd.w = p->w_shared_down;
+        sd.act = su.h_out;
+        sd.offsets = pm.dense_offsets;
+        sd.sorted_token = nullptr;
+        sd.sorted_w = sgate;
+        sd.rows = T; sd.E = 1; sd.D = D; sd.f = fs;
+        sd.acc_out = out_acc;
+        sd.status = status;
+        if (launch_grouped_gemm(sd, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+
+    CombineLaunch c{};
+    c.out_acc = (!det || shared) ? out_acc : nullptr;
+    c.y_sorted = det ? at<bf16>(workspace, L.y_sorted) : nullptr;
+    c.slot_to_row = pm.slot_to_row;
+    c.topk_w = det ? tw : nullptr;
+    c.T = T; c.D = D; c.K = K;
+    c.out = reinterpret_cast<bf16*>(out);
+    if (!mark(MOE_EV_COMBINE) || launch_combine(c, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    return mark(MOE_EV_END) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_read_device_status(void* workspace, void* stream) {
+    if (!workspace) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = as_stream(stream);
+    int h = 0;
+    if (cudaMemcpyAsync(&h, workspace, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
+    return h;
+}
+
+}  // extern "C"

@@ -1,0 +1,124 @@
+// permute.cu -- group the (token, slot) pairs by expert, build the inverse map, and
+// gather the token rows into expert order.
+//
+// "MoE" (llm.rainlin.net), section 3.2: each routed expert gathers the tokens routed to
+// it (the expert loop's torch.where over the expert mask, then hidden_states[token_idx]).
+// "1.6 混合专家（MoE）", section 2: tokens are first grouped by route, computed per
+// expert, then merged back in their original order.
+//
+// permute_kernel: one CTA per expert e.
+//   offsets[e] = sum_{e' < e} counts[e']            (block reduction over <= 512 counts)
+//   a block-wide ballot scan walks the T*K routing entries in order and writes the
+//   entries equal to e to rows offsets[e] + rank  -> ascending token order (stable).
+// gather_kernel: x_sorted[r] = x[sorted_token[r]], 16-byte vectors, grid-stride.
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kPermThreads = 512;
+
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteLaunch a) {
+    __shared__ int warp_tot[kPermThreads / 32];
+    __shared__ int warp_pre[kPermThreads / 32];
+    __shared__ int s_off;
+    __shared__ int s_block_hits;
+    const int e = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int total = a.T * a.K;
+
+    int v = 0;
+    for (int i = tid; i < e; i += kPermThreads) v += a.counts[i];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if (lane == 0) warp_tot[warp] = v;
+    __syncthreads();
+    if (tid == 0) {
+        int s = 0;
+        for (int w = 0; w < kPermThreads / 32; ++w) s += warp_tot[w];
+        s_off = s;
+    }
+    __syncthreads();
+    const int off = s_off;
+    const int n_e = a.counts[e];
+    if (tid == 0) {
+        a.offsets[e] = off;
+        if (e == a.E - 1) {
+            a.offsets[a.E] = off + n_e;
+            if (off + n_e != total) set_status(a.status, MOE_ERR_DEVICE);
+        }
+        if (e == 0 && a.dense_offsets) {
+            a.dense_offsets[0] = 0;
+            a.dense_offsets[1] = a.T;
+        }
+    }
+    if (n_e == 0) return;
+
+    const unsigned lt_mask = (1u << lane) - 1u;
+    int base = 0;
+    for (int j0 = 0; j0 < total; j0 += kPermThreads) {
+        const int j = j0 + tid;
+        const bool hit = (j < total) && (__ldg(a.topk_idx + j) == e);
+        const unsigned b = __ballot_sync(0xffffffffu, hit);
+        if (lane == 0) warp_tot[warp] = __popc(b);
+        __syncthreads();
+        if (warp == 0) {
+            const int c = (lane < kPermThreads / 32) ? warp_tot[lane] : 0;
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            if (lane < kPermThreads / 32) warp_pre[lane] = incl - c;
+            if (lane == kPermThreads / 32 - 1) s_block_hits = incl;
+        }
+        __syncthreads();
+        if (hit) {
+            const int r = base + warp_pre[warp] + __popc(b & lt_mask);
+            if (r < n_e) {
+                const int row = off + r;
+                a.sorted_token[row] = j / a.K;
+                if (a.topk_w) a.sorted_w[row] = __ldg(a.topk_w + j);
+                a.slot_to_row[j] = row;
+            }
+        }
+        base += s_block_hits;
+        __syncthreads();
+    }
+    if (tid == 0 && base != n_e) set_status(a.status, MOE_ERR_DEVICE);
+}
+
+__global__ void __launch_bounds__(256) gather_kernel(GatherLaunch a) {
+    const int vec = a.D / 8;
+    const long long n = static_cast<long long>(a.rows) * vec;
+    const uint4* src = reinterpret_cast<const uint4*>(a.x);
+    uint4* dst = reinterpret_cast<uint4*>(a.x_sorted);
+    for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n; i += 256ll * gridDim.x) {
+        const int r = static_cast<int>(i / vec);
+        const int c = static_cast<int>(i - static_cast<long long>(r) * vec);
+        const int t = __ldg(a.sorted_token + r);
+        dst[i] = __ldg(src + static_cast<size_t>(t) * vec + c);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const PermuteLaunch& a, cudaStream_t s) {
+    permute_kernel<<<a.E, kPermThreads, 0, s>>>(a);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const GatherLaunch& a, int num_sms, cudaStream_t s) {
+    if (a.rows == 0) return cudaSuccess;
+    const long long n = static_cast<long long>(a.rows) * (a.D / 8);
+    const int blocks = static_cast<int>(std::min<long long>((n + 255) / 256, 8ll * num_sms));
+    gather_kernel<<<blocks, 256, 0, s>>>(a);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

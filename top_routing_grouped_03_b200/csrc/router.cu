@@ -1,0 +1,167 @@
+// router.cu -- router logits, fp32 softmax/TopK/renormalisation and per-expert counts.
+//
+// "MoE" (llm.rainlin.net), section 2: r = x W_r^T, p = Softmax(r) in fp32,
+// I = TopK(p, K), alpha = p_I / sum p_I; plus the shared-expert scalar gate
+// sigma(w_s^T x) of section 4.
+//
+// One kernel.  CTA (tb, eb) computes the fp32 logits of 8 tokens against a slab of
+// experts (the shared gate vector rides along as expert index E) and writes them to a
+// workspace.  The CTA that finishes a token block last (atomic ticket, no waiting) then
+// runs the selection for those 8 tokens, one warp per token, in registers:
+//   * TopK on the logits: the softmax is strictly increasing, so the K largest
+//     probabilities are the K largest logits; ties go to the lower expert index.
+//   * alpha_k = exp(r_k - r_max) / sum_{j in I} exp(r_j - r_max): the full softmax
+//     denominator cancels in the renormalisation, so only the K selected terms are
+//     exponentiated.
+//   * expert_counts[e] += 1 per selected expert (global atomics, for the permutation).
+#include <cfloat>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kTokensPerCta = 8;
+constexpr int kRouterThreads = 256;
+constexpr int kMaxExpertsPerLane = 16;  // E <= 512
+
+__global__ void __launch_bounds__(kRouterThreads)
+router_kernel(RouterLaunch a, int experts_per_cta) {
+    extern __shared__ __align__(16) uint4 xs[];  // [8][D] bf16 tokens of this block
+    __shared__ int s_last;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int D = a.D, E = a.E;
+    const int t0 = blockIdx.x * kTokensPerCta;
+    const int nt = min(kTokensPerCta, a.T - t0);
+    const int rows_total = E + (a.w_shared_gate ? 1 : 0);
+
+    // ---- stage the 8 token rows (zeros past T)
+    const int vec_per_row = D / 8;
+    const uint4* xsrc = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0) * D);
+    for (int i = tid; i < kTokensPerCta * vec_per_row; i += kRouterThreads) {
+        const int r = i / vec_per_row;
+        xs[i] = (r < nt) ? __ldg(xsrc + i) : make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+
+    // ---- logits of this CTA's expert slab: one warp per expert row
+    const int e_begin = blockIdx.y * experts_per_cta;
+    const int e_end = min(e_begin + experts_per_cta, rows_total);
+    for (int e = e_begin + warp; e < e_end; e += kRouterThreads / 32) {
+        const bf16* wrow = (e < E) ? a.w_router + static_cast<size_t>(e) * D : a.w_shared_gate;
+        const uint4* wv = reinterpret_cast<const uint4*>(wrow);
+        float acc[kTokensPerCta];
+#pragma unroll
+        for (int t = 0; t < kTokensPerCta; ++t) acc[t] = 0.f;
+        for (int c = lane; c < vec_per_row; c += 32) {
+            const uint4 w = __ldg(wv + c);
+            const float w0 = bf16_lo(w.x), w1 = bf16_hi(w.x), w2 = bf16_lo(w.y), w3 = bf16_hi(w.y);
+            const float w4 = bf16_lo(w.z), w5 = bf16_hi(w.z), w6 = bf16_lo(w.w), w7 = bf16_hi(w.w);
+#pragma unroll
+            for (int t = 0; t < kTokensPerCta; ++t) {
+                const uint4 xv = xs[t * vec_per_row + c];
+                float s = acc[t];
+                s = fmaf(w0, bf16_lo(xv.x), s);
+                s = fmaf(w1, bf16_hi(xv.x), s);
+                s = fmaf(w2, bf16_lo(xv.y), s);
+                s = fmaf(w3, bf16_hi(xv.y), s);
+                s = fmaf(w4, bf16_lo(xv.z), s);
+                s = fmaf(w5, bf16_hi(xv.z), s);
+                s = fmaf(w6, bf16_lo(xv.w), s);
+                s = fmaf(w7, bf16_hi(xv.w), s);
+                acc[t] = s;
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < kTokensPerCta; ++t) {
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+        }
+        if (lane == 0) {
+            const float b = (e < E && a.logit_bias) ? a.logit_bias[e] : 0.f;
+            for (int t = 0; t < nt; ++t)
+                a.logits[static_cast<size_t>(t0 + t) * (E + 1) + e] = acc[t] + b;
+        }
+    }
+
+    // ---- ticket: the last CTA of this token block does the selection
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(&a.counters[blockIdx.x], 1u);
+        s_last = (prev == gridDim.y - 1) ? 1 : 0;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+
+    for (int t = warp; t < nt; t += kRouterThreads / 32) {
+        const int token = t0 + t;
+        const float* lg = a.logits + static_cast<size_t>(token) * (E + 1);
+        float v[kMaxExpertsPerLane];
+#pragma unroll
+        for (int j = 0; j < kMaxExpertsPerLane; ++j) {
+            const int e = j * 32 + lane;
+            v[j] = (e < E) ? __ldcg(lg + e) : -FLT_MAX;
+        }
+        float my_v = -FLT_MAX;
+        int my_i = 0;
+        for (int k = 0; k < a.K; ++k) {
+            float bv = -FLT_MAX;
+            int bi = 0x7fffffff;
+#pragma unroll
+            for (int j = 0; j < kMaxExpertsPerLane; ++j) {
+                const int e = j * 32 + lane;
+                if (e < E && v[j] > bv) { bv = v[j]; bi = e; }  // strict: lowest e per lane
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+                if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+            }
+            if (lane == k) { my_v = bv; my_i = bi; }
+            // retire the winner (owner lane only); -inf never wins against finite logits
+#pragma unroll
+            for (int j = 0; j < kMaxExpertsPerLane; ++j)
+                if (j * 32 + lane == bi) v[j] = -INFINITY;
+        }
+        const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
+        float ex = (lane < a.K) ? expf(my_v - vmax) : 0.f;
+        float sum = ex;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if (lane < a.K) {
+            a.topk_idx[static_cast<size_t>(token) * a.K + lane] = my_i;
+            a.topk_w[static_cast<size_t>(token) * a.K + lane] = ex / sum;
+            atomicAdd(&a.counts[my_i], 1);
+        }
+        if (a.w_shared_gate && lane == 0) {
+            const float g = __ldcg(lg + E);
+            a.shared_gate[token] = 1.f / (1.f + expf(-g));
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s) {
+    if (a.T == 0) return cudaSuccess;
+    const int n_tb = ceil_div(a.T, kTokensPerCta);
+    const int rows_total = a.E + (a.w_shared_gate ? 1 : 0);
+    const int warps = kRouterThreads / 32;
+    // split the experts so that the grid covers about two waves of the GPU
+    int n_eb = ceil_div(2 * num_sms, n_tb);
+    n_eb = max(1, min(n_eb, ceil_div(rows_total, warps)));
+    int per_cta = ceil_div(ceil_div(rows_total, n_eb), warps) * warps;
+    n_eb = ceil_div(rows_total, per_cta);
+    const size_t smem = static_cast<size_t>(kTokensPerCta) * a.D * sizeof(bf16);
+    cudaError_t err = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    router_kernel<<<dim3(n_tb, n_eb), kRouterThreads, smem, s>>>(a, per_cta);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace moe
