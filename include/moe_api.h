@@ -127,7 +127,7 @@ MOE_API int moe_permute(const int32_t* topk_idx, const float* topk_w, const int3
  *   v_r = W_down^e h_r                                    fp32 accumulate
  * and then, with w_r = sorted_w[r] (1 when sorted_w is NULL):
  *   out_acc[t, :] += w_r * v_r     (fp32 atomics; out_acc is NOT cleared), and/or
- *   y_sorted[r, :] = bf16(w_r * v_r)
+ *   y_sorted[r, :] = w_r * v_r     (fp32 [rows, D], one row per (token, expert) pair)
  * At least one of out_acc / y_sorted must be non-NULL.
  *   x            [T, D] bf16
  *   sorted_token [rows] int32, or NULL for the identity (row r is token r, rows <= T)
@@ -143,7 +143,7 @@ MOE_API int moe_grouped_swiglu(const moe_bf16* x, const int32_t* sorted_token,
                        const int32_t* expert_offsets, const float* sorted_w,
                        const moe_bf16* w_gate_up, const moe_bf16* w_down,
                        int T, int rows, int D, int E, int f,
-                       moe_bf16* y_sorted, float* out_acc,
+                       float* y_sorted, float* out_acc,
                        void* workspace, size_t ws_bytes, void* stream);
 
 /*
@@ -151,11 +151,11 @@ MOE_API int moe_grouped_swiglu(const moe_bf16* x, const int32_t* sorted_token,
  * index_add):
  *   out[t, :] = bf16( acc[t, :] + sum_k w_tk * y_sorted[slot_to_row[t*K+k], :]
  *                     + shared_gate[t] * shared_out[t, :] )
- * Every term is optional: out_acc (fp32 [T, D]) NULL -> acc = 0; y_sorted (bf16 [T*K, D])
+ * Every term is optional: out_acc (fp32 [T, D]) NULL -> acc = 0; y_sorted (fp32 [T*K, D])
  * NULL -> no routed sum; topk_w NULL -> w = 1 (y_sorted already weighted); shared_out
  * (bf16 [T, D]) NULL -> no shared term.  The k-sum runs in slot order (deterministic).
  */
-MOE_API int moe_combine(const float* out_acc, const moe_bf16* y_sorted, const int32_t* slot_to_row,
+MOE_API int moe_combine(const float* out_acc, const float* y_sorted, const int32_t* slot_to_row,
                 const float* topk_w, const moe_bf16* shared_out, const float* shared_gate,
                 int T, int D, int K, moe_bf16* out, void* stream);
 

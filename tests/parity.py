@@ -6,8 +6,12 @@ Acceptance rules for one layer call:
     be a valid top-K up to that gap (every chosen expert has p >= p_(K) - NEAR_TIE);
   * routing weights: |alpha_gpu - alpha_oracle| <= W_TOL for every matched expert (on
     tokens whose set differs, the oracle renormalises over the CUDA path's set);
-  * output: max |y_gpu - y_oracle| <= Y_TOL * RMS(y_oracle), where tokens whose CUDA
-    selection differs are compared with the oracle output for that selection.
+  * output: |y_gpu - y_oracle| <= Y_TOL * RMS(y_oracle) + half_ulp_bf16(y) elementwise,
+    where tokens whose CUDA selection differs are compared with the oracle output for that
+    selection.  The half-ulp term is the rounding of the exact value to the bf16 output
+    format itself: no bf16 number is closer than that to a value midway between two bf16
+    neighbours, so without it the bound could not be met by elements beyond ~5 x RMS.
+    Intermediate fp32 results (out_acc, y_sorted) are checked against the plain bound.
 """
 from __future__ import annotations
 
@@ -26,6 +30,21 @@ class RouteReport:
     near_tie: int
     differing_sets: np.ndarray  # token ids whose CUDA set differs (all near ties)
     max_w_err: float
+
+
+def half_ulp_bf16(v: np.ndarray) -> np.ndarray:
+    """Half the spacing of bf16 numbers (8 significant bits) at |v|."""
+    a = np.abs(np.asarray(v, np.float64))
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, np.exp2(e - 8), 0.0)
+
+
+def output_error(y_gpu_bf16: np.ndarray, y_ref: np.ndarray):
+    """(max |dy|, RMS(y_ref), worst fraction of the allowed bound) for a bf16 output."""
+    rms = float(np.sqrt(np.mean(y_ref ** 2)))
+    d = np.abs(y_gpu_bf16 - y_ref)
+    allow = Y_TOL * rms + half_ulp_bf16(np.maximum(np.abs(y_ref), np.abs(y_gpu_bf16)))
+    return float(d.max()) if d.size else 0.0, rms, float((d / allow).max()) if d.size else 0.0
 
 
 def check_route(orc, gpu_idx, gpu_w, gpu_counts=None, E=None) -> RouteReport:
@@ -95,9 +114,9 @@ def check_layer(orc_mod, inp, y_gpu, gpu_idx, gpu_w, tokens=None, orc=None):
         alpha[t] = p / p.sum()
     y_ref = oracle_outputs(orc_mod, inp, idx, alpha, toks, orc["shared_gate"])
     y = y_gpu[torch.as_tensor(toks, device=y_gpu.device)].float().cpu().numpy().astype(np.float64)
-    rms = float(np.sqrt(np.mean(y_ref ** 2)))
-    err = float(np.abs(y - y_ref).max())
+    err, rms, used = output_error(y, y_ref)
     assert rms > 0
-    assert err <= Y_TOL * rms, f"output error {err:.3e} > {Y_TOL} x RMS {rms:.3e}"
+    assert used <= 1.0, (f"output error {err:.3e} exceeds {Y_TOL} x RMS {rms:.3e} + half a bf16 "
+                         f"ulp ({used:.2f} of the bound)")
     return dict(near_tie=rep.near_tie, differing=len(rep.differing_sets), w_err=rep.max_w_err,
-                y_err=err, y_rms=rms, y_rel=err / rms)
+                y_err=err, y_rms=rms, y_rel=err / rms, bound_used=used)

@@ -41,12 +41,21 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineLaunch a) {
             for (int j = 0; j < 8; ++j) acc[j] = 0.f;
         }
         if (a.y_sorted) {
-            const uint4* ys = reinterpret_cast<const uint4*>(a.y_sorted);
+            const float4* ys = reinterpret_cast<const float4*>(a.y_sorted);
             for (int k = 0; k < a.K; ++k) {
                 const int slot = t * a.K + k;
                 const int row = __ldg(a.slot_to_row + slot);
                 const float w = a.topk_w ? __ldg(a.topk_w + slot) : 1.f;
-                add8(acc, __ldg(ys + static_cast<size_t>(row) * vec + c), w);
+                const size_t o = 2 * (static_cast<size_t>(row) * vec + c);
+                const float4 lo = __ldg(ys + o), hi = __ldg(ys + o + 1);
+                acc[0] = fmaf(w, lo.x, acc[0]);
+                acc[1] = fmaf(w, lo.y, acc[1]);
+                acc[2] = fmaf(w, lo.z, acc[2]);
+                acc[3] = fmaf(w, lo.w, acc[3]);
+                acc[4] = fmaf(w, hi.x, acc[4]);
+                acc[5] = fmaf(w, hi.y, acc[5]);
+                acc[6] = fmaf(w, hi.z, acc[6]);
+                acc[7] = fmaf(w, hi.w, acc[7]);
             }
         }
         if (a.shared_out) {

@@ -86,14 +86,14 @@ struct GroupedGemmLaunch {
     int rows, E, D, f;
     bf16* h_out;                // gate_up: [rows, f]
     float* acc_out;             // down: [T, D] scatter-add target or NULL
-    bf16* y_out;                // down: [rows, D] or NULL
+    float* y_out;               // down: [rows, D] fp32 or NULL
     int* status;
 };
 cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s);
 
 struct CombineLaunch {
     const float* out_acc;
-    const bf16* y_sorted;
+    const float* y_sorted;
     const int32_t* slot_to_row;
     const float* topk_w;
     const bf16* shared_out;

@@ -18,7 +18,7 @@
 // Warp 0 issues TMA loads into a STAGES-deep ring, warp 1 issues tcgen05.mma (one
 // thread) and owns the TMEM allocation, warps 2-5 drain TMEM (tcgen05.ld) and run the
 // epilogue: h = SiLU(g) * u -> bf16 for gate_up; w * v -> fp32 red.add into the token's
-// output row (and/or bf16 y_sorted) for down.
+// output row (and/or fp32 y_sorted) for down.
 // The work list (group, feature block, row block) is derived on the device from the
 // group offsets, so no host synchronisation is needed.  Every wait is bounded.
 #include <cudaTypedefs.h>
@@ -70,7 +70,7 @@ struct Params {
     int out_cols;      // gate_up: f (h row length); down: D (output row length)
     bf16* h_out;
     float* acc_out;
-    bf16* y_out;
+    float* y_out;
     int* status;
 };
 
@@ -296,8 +296,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                             const int tok = p.sorted_token ? __ldg(p.sorted_token + row) : row;
                             red_add_f32(p.acc_out + static_cast<size_t>(tok) * p.out_cols + feat, v);
                         }
-                        if (p.y_out)
-                            p.y_out[static_cast<size_t>(row) * p.out_cols + feat] = __float2bfloat16_rn(v);
+                        if (p.y_out) p.y_out[static_cast<size_t>(row) * p.out_cols + feat] = v;
                     }
                 }
             }

@@ -65,7 +65,7 @@ Layout layout(long long T, long long D, long long E, long long K, long long f, l
     L.h = take(2 * T * K * f);
     L.h_s = take(2 * T * fs);
     L.out_acc = take(sizeof(float) * T * D);
-    L.y_sorted = take(2 * T * K * D);
+    L.y_sorted = take(sizeof(float) * T * K * D);
     L.total = o;
     return L;
 }
@@ -173,7 +173,7 @@ int moe_permute(const int32_t* topk_idx, const float* topk_w, const int32_t* exp
 int moe_grouped_swiglu(const moe_bf16* x, const int32_t* sorted_token,
                        const int32_t* expert_offsets, const float* sorted_w,
                        const moe_bf16* w_gate_up, const moe_bf16* w_down, int T, int rows, int D,
-                       int E, int f, moe_bf16* y_sorted, float* out_acc, void* workspace,
+                       int E, int f, float* y_sorted, float* out_acc, void* workspace,
                        size_t ws_bytes, void* stream) {
     int rc = check_shape(T, D, E, 1, f, 0);
     if (rc) return rc;
@@ -217,12 +217,12 @@ int moe_grouped_swiglu(const moe_bf16* x, const int32_t* sorted_token,
     dn.sorted_w = sorted_w;
     dn.rows = rows; dn.E = E; dn.D = D; dn.f = f;
     dn.acc_out = out_acc;
-    dn.y_out = reinterpret_cast<bf16*>(y_sorted);
+    dn.y_out = y_sorted;
     dn.status = status;
     return launch_grouped_gemm(dn, sms, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-int moe_combine(const float* out_acc, const moe_bf16* y_sorted, const int32_t* slot_to_row,
+int moe_combine(const float* out_acc, const float* y_sorted, const int32_t* slot_to_row,
                 const float* topk_w, const moe_bf16* shared_out, const float* shared_gate, int T,
                 int D, int K, moe_bf16* out, void* stream) {
     if (T < 0 || D <= 0 || D % 8 || K < 0) return MOE_ERR_ARG;
@@ -233,7 +233,7 @@ int moe_combine(const float* out_acc, const moe_bf16* y_sorted, const int32_t* s
         return MOE_ERR_ALIGN;
     CombineLaunch a{};
     a.out_acc = out_acc;
-    a.y_sorted = reinterpret_cast<const bf16*>(y_sorted);
+    a.y_sorted = y_sorted;
     a.slot_to_row = slot_to_row;
     a.topk_w = topk_w;
     a.shared_out = reinterpret_cast<const bf16*>(shared_out);
@@ -251,7 +251,8 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     int rc = check_shape(T, D, E, K, f, fs);
     if (rc) return rc;
     const bool shared = fs > 0;
-    if (!p->x || !p->w_router || !p->w_gate_up || !p->w_down || !out) return MOE_ERR_ARG;
+    if (!p->w_router || !p->w_gate_up || !p->w_down) return MOE_ERR_ARG;
+    if (T > 0 && (!p->x || !out)) return MOE_ERR_ARG;
     if (shared && (!p->w_shared_gate || !p->w_shared_gate_up || !p->w_shared_down)) return MOE_ERR_ARG;
     if (!shared && (p->w_shared_gate || p->w_shared_gate_up || p->w_shared_down)) return MOE_ERR_ARG;
     if (!aligned16(p->x) || !aligned16(p->w_router) || !aligned16(p->w_gate_up) ||
@@ -339,7 +340,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     dn.sorted_w = det ? nullptr : pm.sorted_w;
     dn.rows = rows; dn.E = E; dn.D = D; dn.f = f;
     dn.acc_out = det ? nullptr : out_acc;
-    dn.y_out = det ? at<bf16>(workspace, L.y_sorted) : nullptr;
+    dn.y_out = det ? at<float>(workspace, L.y_sorted) : nullptr;
     dn.status = status;
     if (!mark(MOE_EV_DOWN) || launch_grouped_gemm(dn, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -369,7 +370,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
 
     CombineLaunch c{};
     c.out_acc = (!det || shared) ? out_acc : nullptr;
-    c.y_sorted = det ? at<bf16>(workspace, L.y_sorted) : nullptr;
+    c.y_sorted = det ? at<float>(workspace, L.y_sorted) : nullptr;
     c.slot_to_row = pm.slot_to_row;
     c.topk_w = det ? tw : nullptr;
     c.T = T; c.D = D; c.K = K;
