@@ -101,6 +101,30 @@ MOE_API int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* 
               void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * moe_route_noalloc: the router of moe_route (same kernel, same outputs, same argument
+ * rules) for callers that cannot allocate device memory: code hosted by a framework that
+ * owns every device allocation and hands its plugins no allocator, or latency-critical
+ * code that cannot afford the device-wide synchronisation of cudaMalloc/cudaFree.  The
+ * source pages have no counterpart to this entry point; it exists only for such callers.
+ *   - No workspace argument.  The router's scratch (fp32 logits [T, E+1] and one ticket
+ *     per 8 tokens) lives in a 1 MiB array that the library declares in device memory;
+ *     every GPU that loads the library holds that 1 MiB until the process exits.
+ *   - Limit: 256-byte-rounded 4*T*(E+1) bytes plus 4*ceil(T/8) bytes must fit in 1 MiB
+ *     (for example T <= 1019 at E = 256, T <= 2030 at E = 128); larger calls return
+ *     MOE_ERR_UNSUPPORTED before anything is enqueued.
+ *   - The first call on a device looks up the array's device address (once per device,
+ *     with that device current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array and it keeps the last call's contents:
+ *     the call clears the tickets itself, but calls whose work overlaps on the GPU (other
+ *     streams, other host threads) race on the array and must be serialised by the caller.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+MOE_API int moe_route_noalloc(const moe_bf16* x, const moe_bf16* w_router,
+                              const float* logit_bias, const moe_bf16* w_shared_gate,
+                              int T, int D, int E, int K, int32_t* topk_idx, float* topk_w,
+                              int32_t* expert_counts, float* shared_gate, void* stream);
+
+/*
  * Permutation: group the T*K (token, slot) pairs by expert ("MoE", section 3.2: each
  * routed expert gathers the tokens routed to it).  Row order inside a group is by
  * ascending token (stable).

@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
         L.moe_layer_forward.restype = I
         L.moe_read_device_status.argtypes = [P, P]
         L.moe_read_device_status.restype = I
+        L.moe_route_noalloc.argtypes = [P, P, P, P, I, I, I, I, P, P, P, P, P]
+        L.moe_route_noalloc.restype = I
         L.moe_launch_count.argtypes = []
         L.moe_launch_count.restype = ctypes.c_ulonglong
         _lib = L
@@ -134,6 +136,23 @@ def route(x, w_router, K, logit_bias=None, w_shared_gate=None, workspace=None, s
     rc = lib().moe_route(_p(x), _p(w_router), _p(logit_bias), _p(w_shared_gate), T, D, E, K,
                          _p(idx), _p(w), _p(counts), _p(sg), _p(ws), ws.numel(), _stream(stream))
     _check(rc, "moe_route")
+    return idx, w, counts, sg
+
+
+def route_noalloc(x, w_router, K, logit_bias=None, w_shared_gate=None, stream=None):
+    """Router step with no workspace: the library's own 1 MiB device scratch is used (see
+    moe_route_noalloc in moe_api.h for the size limit and the sharing rules).  Only the
+    outputs are allocated here, by the caller's side of the binding."""
+    T, D = x.shape
+    E = w_router.shape[0]
+    dev = x.device
+    idx = torch.empty((T, K), dtype=torch.int32, device=dev)
+    w = torch.empty((T, K), dtype=torch.float32, device=dev)
+    counts = torch.empty((E,), dtype=torch.int32, device=dev)
+    sg = torch.empty((T,), dtype=torch.float32, device=dev) if w_shared_gate is not None else None
+    rc = lib().moe_route_noalloc(_p(x), _p(w_router), _p(logit_bias), _p(w_shared_gate), T, D,
+                                 E, K, _p(idx), _p(w), _p(counts), _p(sg), _stream(stream))
+    _check(rc, "moe_route_noalloc")
     return idx, w, counts, sg
 
 
