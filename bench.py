@@ -107,6 +107,25 @@ def ncu_traffic(kernel: str, workload: str):
         return None
 
 
+# ---------------------------------------------------------------- ranks
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """The slowest rank's figure (all-reduce MAX); x itself without a process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, tokens_per_rank: int, steps: int, slowest_ms: float) -> float:
+    """Tokens of all ranks over the slowest rank's device time, per second."""
+    return world * tokens_per_rank * steps / (slowest_ms / 1e3)
+
+
 # ---------------------------------------------------------------- clocks
 
 
@@ -245,6 +264,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--deterministic", action="store_true")
+    ap.add_argument("--flush-mib", type=int, default=FLUSH_BYTES >> 20,
+                    help="L2 flush buffer written before each timed step (0: none, for "
+                         "profiler runs that flush caches themselves)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -278,7 +300,9 @@ def main():
     idx = torch.empty((T, K), dtype=torch.int32, device=dev)
     tw = torch.empty((T, K), dtype=torch.float32, device=dev)
     counts = torch.empty((E,), dtype=torch.int32, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = torch.empty(max(args.flush_mib, 1) << 20, dtype=torch.uint8, device=dev)
+    if args.flush_mib == 0:
+        flush = flush[:0]
     stream = torch.cuda.current_stream()
 
     def events():
@@ -322,12 +346,9 @@ def main():
         total_ms += evs[0].elapsed_time(evs[-1])
         for j, n in enumerate(names[1:-1], start=1):
             per_kernel[n] += evs[j].elapsed_time(evs[j + 1])
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms / args.steps
-    value = world * T * args.steps / (total_ms / 1e3)
+    value = whole_job_rate(world, T, args.steps, total_ms)
 
     # ---- end to end through the public API: pinned host x in, pinned host y out
     x_host = inp.x.cpu().pin_memory()
@@ -346,14 +367,11 @@ def main():
         layer.forward_host(x_host, y_host, x_dev, out)
         e_b[i].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in zip(e_a, e_b))
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(e_a, e_b)), dev)
     if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
         dist.destroy_process_group()
-    e2e = {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+    e2e = {"value": whole_job_rate(world, T, args.steps, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
            "d2h_bytes_per_step": y_host.numel() * y_host.element_size()}
 
