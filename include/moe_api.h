@@ -160,8 +160,9 @@ MOE_API int moe_permute(const int32_t* topk_idx, const float* topk_w, const int3
  *   w_down       [E, D, f] bf16
  * `rows` is the number of sorted rows (T*K for routed experts; T for a dense expert
  * given as E = 1, identity tokens and offsets {0, T}).
- * workspace: at least moe_workspace_size(T, D, E, K, f, 0) bytes with K = rows / T
- * rounded up (holds the gathered token rows and h).
+ * The token rows are gathered from x inside the gate_up kernel (no permuted copy).
+ * workspace: at least 256 + 2*rows*f bytes rounded up to 256 (holds h); for example
+ * moe_workspace_size(T, D, E, K, f, 0) with K = rows / T rounded up.
  */
 MOE_API int moe_grouped_swiglu(const moe_bf16* x, const int32_t* sorted_token,
                        const int32_t* expert_offsets, const float* sorted_w,
@@ -207,14 +208,13 @@ typedef struct moe_layer_params {
  * layer).  Steps absent from a call (no shared expert) get a zero-length interval.
  */
 enum {
-    MOE_EV_START = 0,    /* before the workspace clears */
-    MOE_EV_ROUTER,       /* router kernel */
+    MOE_EV_START = 0,    /* before the workspace clear */
+    MOE_EV_ROUTER,       /* router kernel (also clears the fp32 accumulator) */
     MOE_EV_PERMUTE,      /* permutation kernel */
-    MOE_EV_GATHER,       /* gather of token rows into expert order */
-    MOE_EV_GATE_UP,      /* grouped gate_up GEMM + SwiGLU */
-    MOE_EV_DOWN,         /* grouped down GEMM + weighted scatter */
+    MOE_EV_GATE_UP,      /* grouped gate_up GEMM + SwiGLU (gathers the token rows) */
+    MOE_EV_DOWN,         /* grouped down GEMM + weighted scatter-add */
     MOE_EV_SHARED,       /* shared expert (gate_up and down) */
-    MOE_EV_COMBINE,      /* combine / bf16 output */
+    MOE_EV_COMBINE,      /* combine to the bf16 output */
     MOE_EV_END,
     MOE_NUM_STEP_EVENTS
 };

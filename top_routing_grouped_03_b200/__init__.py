@@ -43,8 +43,8 @@ class LayerParams(ctypes.Structure):
 
 
 # Step boundaries recorded by moe_layer_forward when step_events is given.
-STEP_EVENT_NAMES = ("start", "router", "permute", "gather", "gate_up", "down", "shared",
-                    "combine", "end")
+STEP_EVENT_NAMES = ("start", "router", "permute", "gate_up", "down", "shared", "combine",
+                    "end")
 NUM_STEP_EVENTS = len(STEP_EVENT_NAMES)
 
 

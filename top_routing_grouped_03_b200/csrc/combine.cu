@@ -25,6 +25,8 @@ __device__ __forceinline__ void add8(float (&acc)[8], const uint4 v, float w) {
 }
 
 __global__ void __launch_bounds__(256) combine_kernel(CombineLaunch a) {
+    grid_dep_wait();  // the rows to combine come from the grouped GEMM
+    grid_dep_launch();
     const int vec = a.D / 8;
     const long long n = static_cast<long long>(a.T) * vec;
     for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n; i += 256ll * gridDim.x) {
@@ -73,13 +75,13 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineLaunch a) {
 
 }  // namespace
 
-cudaError_t launch_combine(const CombineLaunch& a, int num_sms, cudaStream_t s) {
+cudaError_t launch_combine(const CombineLaunch& a, int num_sms, cudaStream_t s, bool pdl) {
     if (a.T == 0) return cudaSuccess;
     const long long n = static_cast<long long>(a.T) * (a.D / 8);
     const int blocks = static_cast<int>(std::min<long long>((n + 255) / 256, 8ll * num_sms));
-    combine_kernel<<<blocks, 256, 0, s>>>(a);
+    cudaError_t err = launch_kernel(combine_kernel, dim3(blocks), dim3(256), 0, s, pdl, a);
     count_launches(1);
-    return cudaGetLastError();
+    return err;
 }
 
 }  // namespace moe

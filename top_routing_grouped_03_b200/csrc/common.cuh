@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <utility>
 
 #include "../../include/moe_api.h"
 
@@ -32,6 +33,34 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Programmatic dependent launch: a kernel launched with launch_kernel(..., pdl = true) may
+// start while its predecessor on the stream is still running; it must call grid_dep_wait()
+// before touching anything the predecessor writes (a no-op when launched without PDL).
+// grid_dep_launch() lets the successor start as soon as every CTA of this grid issued it.
+__device__ __forceinline__ void grid_dep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t s, bool pdl, Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Host-side count of kernel launches issued by the library (read by moe_launch_count).
 void count_launches(unsigned n);
 
@@ -51,8 +80,12 @@ struct RouterLaunch {
     int32_t* counts;      // zeroed before the launch
     float* shared_gate;
     int* status;
+    // optional: rows [T, zero_cols] of zero_acc are cleared by the router kernel (the
+    // layer's fp32 accumulator)
+    float* zero_acc;
+    int zero_cols;
 };
-cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s);
+cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bool pdl = false);
 
 struct PermuteLaunch {
     const int32_t* topk_idx;
@@ -66,20 +99,13 @@ struct PermuteLaunch {
     int32_t* dense_offsets;  // optional [2] = {0, T} for a dense (shared) expert group
     int* status;
 };
-cudaError_t launch_permute(const PermuteLaunch& a, cudaStream_t s);
+cudaError_t launch_permute(const PermuteLaunch& a, cudaStream_t s, bool pdl = false);
 
-struct GatherLaunch {
-    const bf16* x;
-    const int32_t* sorted_token;
-    int rows, D;
-    bf16* x_sorted;
-};
-cudaError_t launch_gather(const GatherLaunch& a, int num_sms, cudaStream_t s);
 
 struct GroupedGemmLaunch {
     bool gate_up;               // true: SiLU(gate)*up epilogue -> h; false: down epilogue
     const void* w;              // weights: gate_up [E, 2f, D] or down [E, D, f]
-    const void* act;            // activations in row order: x_sorted [rows, D] or h [rows, f]
+    const void* act;            // activations: x [T, D] (gathered via gather_tok) or h [rows, f]
     const int32_t* offsets;     // [E+1]
     const int32_t* sorted_token;  // down only; NULL = identity
     const float* sorted_w;      // down only; NULL = 1
@@ -88,8 +114,12 @@ struct GroupedGemmLaunch {
     float* acc_out;             // down: [T, D] scatter-add target or NULL
     float* y_out;               // down: [rows, D] fp32 or NULL
     int* status;
+    // gate_up only: when gather_tok != NULL, act is the token matrix x [T, D] and row r of
+    // the expert-ordered problem is x[gather_tok[r]] (gathered inside the kernel)
+    const int32_t* gather_tok;
 };
-cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s);
+cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s,
+                                bool pdl = false);
 
 struct CombineLaunch {
     const float* out_acc;
@@ -101,6 +131,6 @@ struct CombineLaunch {
     int T, D, K;
     bf16* out;
 };
-cudaError_t launch_combine(const CombineLaunch& a, int num_sms, cudaStream_t s);
+cudaError_t launch_combine(const CombineLaunch& a, int num_sms, cudaStream_t s, bool pdl = false);
 
 }  // namespace moe

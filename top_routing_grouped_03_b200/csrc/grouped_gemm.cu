@@ -18,7 +18,10 @@
 // Warp 0 issues TMA loads into a STAGES-deep ring, warp 1 issues tcgen05.mma (one
 // thread) and owns the TMEM allocation, warps 2-5 drain TMEM (tcgen05.ld) and run the
 // epilogue: h = SiLU(g) * u -> bf16 for gate_up; w * v -> fp32 red.add into the token's
-// output row (and/or fp32 y_sorted) for down.
+// output row (and/or fp32 y_sorted) for down.  When the gate_up rows are tokens of x in
+// expert order, the producer warp gathers them itself with cp.async (16-byte chunks
+// written in the 128-byte swizzle the MMA descriptor expects), so no permuted copy of x is
+// ever materialised.
 // The work list (group, feature block, row block) is derived on the device from the
 // group offsets, so no host synchronisation is needed.  Every wait is bounded.
 #include <cudaTypedefs.h>
@@ -72,7 +75,25 @@ struct Params {
     float* acc_out;
     float* y_out;
     int* status;
+    const int32_t* gather_tok;  // gate_up: B rows are x[gather_tok[row]] (cp.async), or NULL
+    const bf16* x;              // the token matrix the gather reads, [*, K] bf16
 };
+
+
+// The same barrier with an AND across the epilogue threads: all of them take the same
+// branch afterwards, so none can be left waiting at a later epilogue_bar().
+__device__ __forceinline__ bool epilogue_bar_and(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, 1, %2, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(v)), "n"(kEpiThreads)
+        : "memory");
+    return r != 0;
+}
 
 struct Tile {
     int g, i, row0, row_end;
@@ -119,9 +140,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    // gate_up with gathered rows: the 32 producer lanes also arrive (after their cp.async)
+    const bool gather = GATE_UP && p.gather_tok != nullptr;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], gather ? 1 + 32 : 1);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -134,12 +157,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&map_w);
-        tma_prefetch_desc(&map_act);
+        if (!gather) tma_prefetch_desc(&map_act);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
+    // everything above overlaps the previous kernel's tail; the offsets, the activations
+    // and the accumulator are produced by earlier kernels of the stream
+    grid_dep_wait();
+    grid_dep_launch();
     for (int i = threadIdx.x; i <= p.G; i += kThreads) g_off[i] = p.offsets[i];
     __syncthreads();
     if (warp == 2) {
@@ -171,37 +198,74 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
     const int total = *total_slot;
 
     if (warp == 0) {
-        // ---------------------------------------------------------------- TMA producer
-        if (lane == 0) {
+        // ---------------------------------------------------------------- producer
+        // Weights (operand A) always by TMA from lane 0.  Activation rows (operand B): one
+        // TMA box when they are contiguous in expert order; otherwise (gather) each lane
+        // copies 16-byte chunks of x[gather_tok[row]] with cp.async into the swizzled tile:
+        // chunk c of tile row r lands at r*128 + ((c ^ (r % 8)) * 16).  Lane l always owns
+        // chunk c = l % 8 of rows l/8 + 4u.
+        constexpr int kChunks = BN * 8 / 32;
+        if (gather || lane == 0) {
             const uint64_t pol_w = policy_evict_first();  // weights stream through once
             const uint64_t pol_a = policy_evict_last();   // activations are re-read
+            const uint32_t a_bytes = C::kNumA * C::kABytes;
+            const int c = lane & 7;
             int stage = 0;
             uint32_t phase = 0, filled = 0, fill_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
                 const Tile t = decode_tile(tile, g_tile, g_off, p.G, BN);
                 const int wr0 = t.g * p.w_group_rows + t.i * kBM;
+                uint32_t src_off[kChunks];  // element offset of the chunk in x (< 2^31)
+                uint32_t valid_mask = 0;
+                if (gather) {
+#pragma unroll
+                    for (int u = 0; u < kChunks; ++u) {
+                        const int row = t.row0 + (lane >> 3) + 4 * u;
+                        const bool valid = row < t.row_end;
+                        const int tok = valid ? __ldg(p.gather_tok + row) : 0;
+                        src_off[u] = static_cast<uint32_t>(tok) * (p.nk * kBK) + c * 8;
+                        valid_mask |= (valid ? 1u : 0u) << u;
+                    }
+                }
                 for (int kk = 0; kk < p.nk; ++kk) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1u, kWaitBudgetNs, abort_flag)) {
+                    bool got = mbar_wait(&empty[stage], phase ^ 1u, kWaitBudgetNs, abort_flag);
+                    if (gather) got = __all_sync(0xffffffffu, got);
+                    if (!got) {
                         set_status(p.status, MOE_ERR_TIMEOUT);
                         *abort_flag = 1;
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
                     uint8_t* st = smem + stage * C::kStageBytes;
-                    tma_load_2d(st, &map_w, &full[stage], kk * kBK, wr0, pol_w);
-                    if (GATE_UP)
-                        tma_load_2d(st + C::kABytes, &map_w, &full[stage], kk * kBK,
-                                    wr0 + p.up_rows, pol_w);
-                    tma_load_2d(st + C::kNumA * C::kABytes, &map_act, &full[stage], kk * kBK,
-                                t.row0, pol_a);
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&full[stage], gather ? a_bytes : C::kStageBytes);
+                        tma_load_2d(st, &map_w, &full[stage], kk * kBK, wr0, pol_w);
+                        if (GATE_UP)
+                            tma_load_2d(st + C::kABytes, &map_w, &full[stage], kk * kBK,
+                                        wr0 + p.up_rows, pol_w);
+                        if (!gather)
+                            tma_load_2d(st + a_bytes, &map_act, &full[stage], kk * kBK, t.row0,
+                                        pol_a);
+                    }
+                    if (gather) {
+                        const uint32_t b0 = smem_u32(st + a_bytes);
+#pragma unroll
+                        for (int u = 0; u < kChunks; ++u) {
+                            const int r = (lane >> 3) + 4 * u;
+                            cp_async_16(b0 + r * 128 + ((c ^ (r & 7)) << 4),
+                                        p.x + src_off[u] + kk * kBK,
+                                        ((valid_mask >> u) & 1u) ? 16u : 0u);
+                        }
+                        cp_async_mbar_arrive_noinc(&full[stage]);
+                    }
                     filled |= 1u << stage;
                     fill_phase = (fill_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
                 }
             }
-            if (!ok) {  // let the copies already in flight land before the CTA exits
+            if (gather) cp_async_wait_all();
+            if (!ok && lane == 0) {  // let the copies already in flight land before exiting
                 for (int s = 0; s < C::kStages; ++s)
                     if (filled & (1u << s))
                         mbar_wait(&full[s], (fill_phase >> s) & 1u, kDrainBudgetNs, nullptr);
@@ -232,6 +296,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                         break;
                     }
                     tc_fence_after();
+                    if (gather) fence_proxy_async_smem();
                     const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
                     const uint32_t a1 = a0 + C::kABytes;
                     const uint32_t b0 = a0 + C::kNumA * C::kABytes;
@@ -264,7 +329,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
         uint32_t abuf = 0, aphase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             const Tile t = decode_tile(tile, g_tile, g_off, p.G, BN);
-            if (!mbar_wait(&tfull[abuf], aphase, kWaitBudgetNs, abort_flag)) {
+            const bool ready = mbar_wait(&tfull[abuf], aphase, kWaitBudgetNs, abort_flag);
+            if (!epilogue_bar_and(ready)) {
                 set_status(p.status, MOE_ERR_TIMEOUT);
                 *abort_flag = 1;
                 break;
@@ -347,7 +413,7 @@ cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
 
 template <int BN, bool GATE_UP>
 cudaError_t launch_tpl(const CUtensorMap& mw, const CUtensorMap& ma, const Params& p, int grid,
-                       cudaStream_t s) {
+                       cudaStream_t s, bool pdl) {
     using C = Cfg<BN, GATE_UP>;
     const size_t smem = 1024 + static_cast<size_t>(C::kStages) * C::kStageBytes +
                         (2 * C::kStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int);
@@ -355,9 +421,9 @@ cudaError_t launch_tpl(const CUtensorMap& mw, const CUtensorMap& ma, const Param
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    kfn<<<grid, kThreads, smem, s>>>(mw, ma, p);
+    err = launch_kernel(kfn, dim3(grid), dim3(kThreads), smem, s, pdl, mw, ma, p);
     count_launches(1);
-    return cudaGetLastError();
+    return err;
 }
 
 }  // namespace
@@ -370,7 +436,8 @@ int pick_block_rows(int rows, int groups) {
     return 128;
 }
 
-cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s) {
+cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s,
+                                bool pdl) {
     if (a.rows == 0 || a.E == 0) return cudaSuccess;
     if (a.E > kMaxGroups) return cudaErrorInvalidValue;
     cudaError_t err = get_encoder();
@@ -380,7 +447,11 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
     const uint64_t w_group_rows = a.gate_up ? 2ull * a.f : static_cast<uint64_t>(a.D);
     CUtensorMap mw, ma;
     if ((err = make_map(&mw, a.w, w_group_rows * a.E, K, kBM)) != cudaSuccess) return err;
-    if ((err = make_map(&ma, a.act, a.rows, K, BN)) != cudaSuccess) return err;
+    // the activation map is only read when the rows are contiguous (no gather); with a
+    // gather it still has to be a valid descriptor, so it covers the first row of x
+    const bool gather = a.gate_up && a.gather_tok != nullptr;
+    if ((err = make_map(&ma, a.act, gather ? 1 : a.rows, K, gather ? 1 : BN)) != cudaSuccess)
+        return err;
     Params p{};
     p.offsets = a.offsets;
     p.sorted_token = a.sorted_token;
@@ -395,13 +466,15 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
     p.acc_out = a.acc_out;
     p.y_out = a.y_out;
     p.status = a.status;
+    p.gather_tok = a.gate_up ? a.gather_tok : nullptr;
+    p.x = reinterpret_cast<const bf16*>(a.act);
     const long long max_tiles = (static_cast<long long>(ceil_div(a.rows, BN)) + a.E) * p.nf;
     const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
     switch (BN) {
-        case 16: return a.gate_up ? launch_tpl<16, true>(mw, ma, p, grid, s) : launch_tpl<16, false>(mw, ma, p, grid, s);
-        case 32: return a.gate_up ? launch_tpl<32, true>(mw, ma, p, grid, s) : launch_tpl<32, false>(mw, ma, p, grid, s);
-        case 64: return a.gate_up ? launch_tpl<64, true>(mw, ma, p, grid, s) : launch_tpl<64, false>(mw, ma, p, grid, s);
-        default: return a.gate_up ? launch_tpl<128, true>(mw, ma, p, grid, s) : launch_tpl<128, false>(mw, ma, p, grid, s);
+        case 16: return a.gate_up ? launch_tpl<16, true>(mw, ma, p, grid, s, pdl) : launch_tpl<16, false>(mw, ma, p, grid, s, pdl);
+        case 32: return a.gate_up ? launch_tpl<32, true>(mw, ma, p, grid, s, pdl) : launch_tpl<32, false>(mw, ma, p, grid, s, pdl);
+        case 64: return a.gate_up ? launch_tpl<64, true>(mw, ma, p, grid, s, pdl) : launch_tpl<64, false>(mw, ma, p, grid, s, pdl);
+        default: return a.gate_up ? launch_tpl<128, true>(mw, ma, p, grid, s, pdl) : launch_tpl<128, false>(mw, ma, p, grid, s, pdl);
     }
 }
 

@@ -36,7 +36,7 @@ int num_sms_current() {
 // Workspace of the whole layer.  The status word is always at offset 0.
 struct Layout {
     size_t status, counters, counts, logits, offsets, dense_offsets, topk_idx, topk_w, sgate,
-        sorted_token, sorted_w, slot_to_row, x_sorted, h, h_s, out_acc, y_sorted, total;
+        sorted_token, sorted_w, slot_to_row, h, h_s, out_acc, y_sorted, total;
     size_t zero_end;  // [0, zero_end) is cleared at the start of a layer call
 };
 
@@ -61,7 +61,6 @@ Layout layout(long long T, long long D, long long E, long long K, long long f, l
     L.sorted_token = take(sizeof(int32_t) * T * K);
     L.sorted_w = take(sizeof(float) * T * K);
     L.slot_to_row = take(sizeof(int32_t) * T * K);
-    L.x_sorted = take(2 * T * K * D);
     L.h = take(2 * T * K * f);
     L.h_s = take(2 * T * fs);
     L.out_acc = take(sizeof(float) * T * D);
@@ -184,25 +183,18 @@ int moe_grouped_swiglu(const moe_bf16* x, const int32_t* sorted_token,
         (y_sorted && !aligned16(y_sorted)))
         return MOE_ERR_ALIGN;
     if (!workspace) return MOE_ERR_WORKSPACE;
-    const size_t xs_off = kAlign;
-    const size_t h_off = align_up(xs_off + 2ull * rows * D);
+    const size_t h_off = kAlign;
     const size_t need = align_up(h_off + 2ull * rows * f);
     if (ws_bytes < need) return MOE_ERR_WORKSPACE;
     if (rows == 0) return MOE_OK;
     cudaStream_t s = as_stream(stream);
     const int sms = num_sms_current();
     int* status = at<int>(workspace, 0);
-    const bf16* act = reinterpret_cast<const bf16*>(x);
-    if (sorted_token) {
-        GatherLaunch g{reinterpret_cast<const bf16*>(x), sorted_token, rows, D,
-                       at<bf16>(workspace, xs_off)};
-        if (launch_gather(g, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
-        act = at<bf16>(workspace, xs_off);
-    }
     GroupedGemmLaunch up{};
     up.gate_up = true;
     up.w = w_gate_up;
-    up.act = act;
+    up.act = x;
+    up.gather_tok = sorted_token;
     up.offsets = expert_offsets;
     up.rows = rows; up.E = E; up.D = D; up.f = f;
     up.h_out = at<bf16>(workspace, h_off);
@@ -219,7 +211,7 @@ int moe_grouped_swiglu(const moe_bf16* x, const int32_t* sorted_token,
     dn.acc_out = out_acc;
     dn.y_out = y_sorted;
     dn.status = status;
-    return launch_grouped_gemm(dn, sms, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_grouped_gemm(dn, sms, s, true) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int moe_combine(const float* out_acc, const float* y_sorted, const int32_t* slot_to_row,
@@ -281,12 +273,12 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     float* out_acc = at<float>(workspace, L.out_acc);
 
     if (!mark(MOE_EV_START)) return MOE_ERR_CUDA;
+    // the only clear: status word, router tickets, expert counts (a few KB); the router
+    // kernel clears the fp32 accumulator itself
     if (cudaMemsetAsync(workspace, 0, L.zero_end, s) != cudaSuccess) return MOE_ERR_CUDA;
     if (p->expert_counts_out && cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s) != cudaSuccess)
         return MOE_ERR_CUDA;
-    if ((!det || shared) &&
-        cudaMemsetAsync(out_acc, 0, sizeof(float) * static_cast<size_t>(T) * D, s) != cudaSuccess)
-        return MOE_ERR_CUDA;
+    const bool use_acc = !det || shared;
 
     RouterLaunch r{};
     r.x = reinterpret_cast<const bf16*>(p->x);
@@ -301,7 +293,9 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     r.counts = counts;
     r.shared_gate = sgate;
     r.status = status;
-    if (!mark(MOE_EV_ROUTER) || launch_router(r, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    r.zero_acc = use_acc ? out_acc : nullptr;
+    r.zero_cols = D;
+    if (!mark(MOE_EV_ROUTER) || launch_router(r, sms, s, false) != cudaSuccess) return MOE_ERR_CUDA;
 
     PermuteLaunch pm{};
     pm.topk_idx = idx;
@@ -314,22 +308,20 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     pm.slot_to_row = at<int32_t>(workspace, L.slot_to_row);
     pm.dense_offsets = at<int32_t>(workspace, L.dense_offsets);
     pm.status = status;
-    if (!mark(MOE_EV_PERMUTE) || launch_permute(pm, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!mark(MOE_EV_PERMUTE) || launch_permute(pm, s, true) != cudaSuccess) return MOE_ERR_CUDA;
 
     const int rows = T * K;
-    GatherLaunch g{reinterpret_cast<const bf16*>(p->x), pm.sorted_token, rows, D,
-                   at<bf16>(workspace, L.x_sorted)};
-    if (!mark(MOE_EV_GATHER) || launch_gather(g, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
-
     GroupedGemmLaunch up{};
     up.gate_up = true;
     up.w = p->w_gate_up;
-    up.act = g.x_sorted;
+    up.act = p->x;
+    up.gather_tok = pm.sorted_token;
     up.offsets = pm.offsets;
     up.rows = rows; up.E = E; up.D = D; up.f = f;
     up.h_out = at<bf16>(workspace, L.h);
     up.status = status;
-    if (!mark(MOE_EV_GATE_UP) || launch_grouped_gemm(up, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!mark(MOE_EV_GATE_UP) || launch_grouped_gemm(up, sms, s, true) != cudaSuccess)
+        return MOE_ERR_CUDA;
 
     GroupedGemmLaunch dn{};
     dn.gate_up = false;
@@ -342,7 +334,8 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     dn.acc_out = det ? nullptr : out_acc;
     dn.y_out = det ? at<float>(workspace, L.y_sorted) : nullptr;
     dn.status = status;
-    if (!mark(MOE_EV_DOWN) || launch_grouped_gemm(dn, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!mark(MOE_EV_DOWN) || launch_grouped_gemm(dn, sms, s, true) != cudaSuccess)
+        return MOE_ERR_CUDA;
 
     if (!mark(MOE_EV_SHARED)) return MOE_ERR_CUDA;
     if (shared) {
@@ -354,7 +347,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
         su.rows = T; su.E = 1; su.D = D; su.f = fs;
         su.h_out = at<bf16>(workspace, L.h_s);
         su.status = status;
-        if (launch_grouped_gemm(su, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+        if (launch_grouped_gemm(su, sms, s, true) != cudaSuccess) return MOE_ERR_CUDA;
         GroupedGemmLaunch sd{};
         sd.gate_up = false;
         sd.w = p->w_shared_down;
@@ -365,17 +358,18 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
         sd.rows = T; sd.E = 1; sd.D = D; sd.f = fs;
         sd.acc_out = out_acc;
         sd.status = status;
-        if (launch_grouped_gemm(sd, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+        if (launch_grouped_gemm(sd, sms, s, true) != cudaSuccess) return MOE_ERR_CUDA;
     }
 
+    // bf16 output: out_acc alone, or (fixed order) out_acc's shared part + the routed rows
     CombineLaunch c{};
-    c.out_acc = (!det || shared) ? out_acc : nullptr;
+    c.out_acc = use_acc ? out_acc : nullptr;
     c.y_sorted = det ? at<float>(workspace, L.y_sorted) : nullptr;
     c.slot_to_row = pm.slot_to_row;
     c.topk_w = det ? tw : nullptr;
     c.T = T; c.D = D; c.K = K;
     c.out = reinterpret_cast<bf16*>(out);
-    if (!mark(MOE_EV_COMBINE) || launch_combine(c, sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!mark(MOE_EV_COMBINE) || launch_combine(c, sms, s, true) != cudaSuccess) return MOE_ERR_CUDA;
     return mark(MOE_EV_END) ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -1,5 +1,4 @@
-// permute.cu -- group the (token, slot) pairs by expert, build the inverse map, and
-// gather the token rows into expert order.
+// permute.cu -- group the (token, slot) pairs by expert and build the inverse map.
 //
 // "MoE" (llm.rainlin.net), section 3.2: each routed expert gathers the tokens routed to
 // it (the expert loop's torch.where over the expert mask, then hidden_states[token_idx]).
@@ -10,9 +9,7 @@
 //   offsets[e] = sum_{e' < e} counts[e']            (block reduction over <= 512 counts)
 //   a block-wide ballot scan walks the T*K routing entries in order and writes the
 //   entries equal to e to rows offsets[e] + rank  -> ascending token order (stable).
-// gather_kernel: x_sorted[r] = x[sorted_token[r]], 16-byte vectors, grid-stride.
-#include <algorithm>
-
+// The token rows themselves are never copied: the grouped GEMM gathers them from x.
 #include "common.cuh"
 
 namespace moe {
@@ -28,6 +25,9 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteLaunch a) 
     const int e = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int total = a.T * a.K;
+
+    grid_dep_wait();  // routing and counts come from the router
+    grid_dep_launch();
 
     int v = 0;
     for (int i = tid; i < e; i += kPermThreads) v += a.counts[i];
@@ -89,36 +89,15 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteLaunch a) 
         __syncthreads();
     }
     if (tid == 0 && base != n_e) set_status(a.status, MOE_ERR_DEVICE);
-}
 
-__global__ void __launch_bounds__(256) gather_kernel(GatherLaunch a) {
-    const int vec = a.D / 8;
-    const long long n = static_cast<long long>(a.rows) * vec;
-    const uint4* src = reinterpret_cast<const uint4*>(a.x);
-    uint4* dst = reinterpret_cast<uint4*>(a.x_sorted);
-    for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n; i += 256ll * gridDim.x) {
-        const int r = static_cast<int>(i / vec);
-        const int c = static_cast<int>(i - static_cast<long long>(r) * vec);
-        const int t = __ldg(a.sorted_token + r);
-        dst[i] = __ldg(src + static_cast<size_t>(t) * vec + c);
-    }
 }
 
 }  // namespace
 
-cudaError_t launch_permute(const PermuteLaunch& a, cudaStream_t s) {
-    permute_kernel<<<a.E, kPermThreads, 0, s>>>(a);
+cudaError_t launch_permute(const PermuteLaunch& a, cudaStream_t s, bool pdl) {
+    cudaError_t err = launch_kernel(permute_kernel, dim3(a.E), dim3(kPermThreads), 0, s, pdl, a);
     count_launches(1);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_gather(const GatherLaunch& a, int num_sms, cudaStream_t s) {
-    if (a.rows == 0) return cudaSuccess;
-    const long long n = static_cast<long long>(a.rows) * (a.D / 8);
-    const int blocks = static_cast<int>(std::min<long long>((n + 255) / 256, 8ll * num_sms));
-    gather_kernel<<<blocks, 256, 0, s>>>(a);
-    count_launches(1);
-    return cudaGetLastError();
+    return err;
 }
 
 }  // namespace moe

@@ -6,8 +6,9 @@
 //
 // One kernel.  CTA (tb, eb) computes the fp32 logits of 8 tokens against a slab of
 // experts (the shared gate vector rides along as expert index E) and writes them to a
-// workspace.  The CTA that finishes a token block last (atomic ticket, no waiting) then
-// runs the selection for those 8 tokens, one warp per token, in registers:
+// workspace; in the layer call it also clears its tokens' rows of the fp32 accumulator.
+// The CTA that finishes a token block last (atomic ticket, no waiting) then runs the
+// selection for those 8 tokens, one warp per token, in registers:
 //   * TopK on the logits: the softmax is strictly increasing, so the K largest
 //     probabilities are the K largest logits; ties go to the lower expert index.
 //   * alpha_k = exp(r_k - r_max) / sum_{j in I} exp(r_j - r_max): the full softmax
@@ -35,6 +36,18 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
     const int nt = min(kTokensPerCta, a.T - t0);
     const int rows_total = E + (a.w_shared_gate ? 1 : 0);
 
+    grid_dep_wait();     // x and the zeroed tickets/counts come from earlier stream work
+    grid_dep_launch();
+
+    // ---- clear this token block's slice of the layer accumulator
+    if (a.zero_acc) {
+        const int n4 = nt * a.zero_cols / 4;
+        const int per = (n4 + gridDim.y - 1) / gridDim.y;
+        float4* dst = reinterpret_cast<float4*>(a.zero_acc + static_cast<size_t>(t0) * a.zero_cols);
+        const int b = blockIdx.y * per, e = min(b + per, n4);
+        for (int i = b + tid; i < e; i += kRouterThreads) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+
     // ---- stage the 8 token rows (zeros past T)
     const int vec_per_row = D / 8;
     const uint4* xsrc = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0) * D);
@@ -44,7 +57,9 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
     }
     __syncthreads();
 
-    // ---- logits of this CTA's expert slab: one warp per expert row
+    // ---- logits of this CTA's expert slab: one warp per expert row; each lane keeps up
+    //      to kUnroll independent 16-byte weight loads in flight
+    constexpr int kUnroll = 8;
     const int e_begin = blockIdx.y * experts_per_cta;
     const int e_end = min(e_begin + experts_per_cta, rows_total);
     for (int e = e_begin + warp; e < e_end; e += kRouterThreads / 32) {
@@ -53,23 +68,34 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
         float acc[kTokensPerCta];
 #pragma unroll
         for (int t = 0; t < kTokensPerCta; ++t) acc[t] = 0.f;
-        for (int c = lane; c < vec_per_row; c += 32) {
-            const uint4 w = __ldg(wv + c);
-            const float w0 = bf16_lo(w.x), w1 = bf16_hi(w.x), w2 = bf16_lo(w.y), w3 = bf16_hi(w.y);
-            const float w4 = bf16_lo(w.z), w5 = bf16_hi(w.z), w6 = bf16_lo(w.w), w7 = bf16_hi(w.w);
+        for (int c0 = lane; c0 < vec_per_row; c0 += 32 * kUnroll) {
+            uint4 w[kUnroll];
 #pragma unroll
-            for (int t = 0; t < kTokensPerCta; ++t) {
-                const uint4 xv = xs[t * vec_per_row + c];
-                float s = acc[t];
-                s = fmaf(w0, bf16_lo(xv.x), s);
-                s = fmaf(w1, bf16_hi(xv.x), s);
-                s = fmaf(w2, bf16_lo(xv.y), s);
-                s = fmaf(w3, bf16_hi(xv.y), s);
-                s = fmaf(w4, bf16_lo(xv.z), s);
-                s = fmaf(w5, bf16_hi(xv.z), s);
-                s = fmaf(w6, bf16_lo(xv.w), s);
-                s = fmaf(w7, bf16_hi(xv.w), s);
-                acc[t] = s;
+            for (int u = 0; u < kUnroll; ++u) {
+                const int c = c0 + 32 * u;
+                w[u] = (c < vec_per_row) ? __ldg(wv + c) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int c = c0 + 32 * u;
+                if (c >= vec_per_row) break;
+                const float w0 = bf16_lo(w[u].x), w1 = bf16_hi(w[u].x), w2 = bf16_lo(w[u].y);
+                const float w3 = bf16_hi(w[u].y), w4 = bf16_lo(w[u].z), w5 = bf16_hi(w[u].z);
+                const float w6 = bf16_lo(w[u].w), w7 = bf16_hi(w[u].w);
+#pragma unroll
+                for (int t = 0; t < kTokensPerCta; ++t) {
+                    const uint4 xv = xs[t * vec_per_row + c];
+                    float s = acc[t];
+                    s = fmaf(w0, bf16_lo(xv.x), s);
+                    s = fmaf(w1, bf16_hi(xv.x), s);
+                    s = fmaf(w2, bf16_lo(xv.y), s);
+                    s = fmaf(w3, bf16_hi(xv.y), s);
+                    s = fmaf(w4, bf16_lo(xv.z), s);
+                    s = fmaf(w5, bf16_hi(xv.z), s);
+                    s = fmaf(w6, bf16_lo(xv.w), s);
+                    s = fmaf(w7, bf16_hi(xv.w), s);
+                    acc[t] = s;
+                }
             }
         }
 #pragma unroll
@@ -145,7 +171,7 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
 
 }  // namespace
 
-cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s) {
+cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bool pdl) {
     if (a.T == 0) return cudaSuccess;
     const int n_tb = ceil_div(a.T, kTokensPerCta);
     const int rows_total = a.E + (a.w_shared_gate ? 1 : 0);
@@ -159,9 +185,10 @@ cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s) {
     cudaError_t err = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    router_kernel<<<dim3(n_tb, n_eb), kRouterThreads, smem, s>>>(a, per_cta);
+    err = launch_kernel(router_kernel, dim3(n_tb, n_eb), dim3(kRouterThreads), smem, s, pdl, a,
+                        per_cta);
     count_launches(1);
-    return cudaGetLastError();
+    return err;
 }
 
 }  // namespace moe
