@@ -79,9 +79,9 @@ struct Params {
     const bf16* x;              // the token matrix the gather reads, [*, K] bf16
 };
 
-
-// The same barrier with an AND across the epilogue threads: all of them take the same
-// branch afterwards, so none can be left waiting at a later epilogue_bar().
+// Named barrier 1 of the four epilogue warps with an AND across their threads: all of
+// them take the same branch afterwards, so a wait that gives up in one warp makes every
+// epilogue warp unwind together.
 __device__ __forceinline__ bool epilogue_bar_and(bool v) {
     uint32_t r;
     asm volatile(
