@@ -264,6 +264,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--deterministic", action="store_true")
+    ap.add_argument("--events", default="roofline", choices=["roofline", "ends", "all"],
+                    help="step boundaries recorded in the timed steps: start/gate_up/down/end "
+                         "(default), start/end only, or every kernel boundary")
     ap.add_argument("--flush-mib", type=int, default=FLUSH_BYTES >> 20,
                     help="L2 flush buffer written before each timed step (0: none, for "
                          "profiler runs that flush caches themselves)")
@@ -305,10 +308,15 @@ def main():
         flush = flush[:0]
     stream = torch.cuda.current_stream()
 
-    def events():
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(moe.NUM_STEP_EVENTS)]
+    names = moe.STEP_EVENT_NAMES
+    recorded = {"roofline": {"start", "gate_up", "down", "end"}, "ends": {"start", "end"},
+                "all": set(names)}[args.events]
+
+    def events(which):
+        evs = [torch.cuda.Event(enable_timing=True) if n in which else None for n in names]
         for e in evs:
-            e.record(stream)  # creates the handle; the library re-records it
+            if e is not None:
+                e.record(stream)  # creates the handle; the library re-records it
         return evs
 
     for i in range(args.warmup):
@@ -318,7 +326,7 @@ def main():
     if layer.device_status() != 0:
         raise RuntimeError("device status after warm-up is not ok")
 
-    step_evs = [events() for _ in range(args.steps)]
+    step_evs = [events(recorded) for _ in range(args.steps)]
     arrs = [moe.event_array(e) for e in step_evs]
     torch.cuda.synchronize()
     props = torch.cuda.get_device_properties(dev)
@@ -339,13 +347,28 @@ def main():
     if layer.device_status() != 0:
         raise RuntimeError("device status after the timed steps is not ok")
 
-    names = moe.STEP_EVENT_NAMES
+    ix = {n: i for i, n in enumerate(names)}
+    total_ms = sum(evs[0].elapsed_time(evs[-1]) for evs in step_evs)
+    gu_total = (sum(e[ix["gate_up"]].elapsed_time(e[ix["down"]]) for e in step_evs)
+                if "gate_up" in recorded else None)
+
+    # per-kernel breakdown: a separate pass with every boundary recorded (those marks keep
+    # each kernel from overlapping its predecessor, so the pass is slower than the step)
+    n_bd = min(args.steps, 100)
+    bd_evs = [events(set(names)) for _ in range(n_bd)]
+    bd_arrs = [moe.event_array(e) for e in bd_evs]
+    torch.cuda.synchronize()
+    for i in range(n_bd):
+        flush.fill_(i & 0xFF)
+        layer(inp.x, out=out, topk_idx=idx, topk_w=tw, counts=counts, step_events=bd_arrs[i])
+    torch.cuda.synchronize()
     per_kernel = {n: 0.0 for n in names[1:-1]}
-    total_ms = 0.0
-    for evs in step_evs:
-        total_ms += evs[0].elapsed_time(evs[-1])
+    for evs in bd_evs:
         for j, n in enumerate(names[1:-1], start=1):
             per_kernel[n] += evs[j].elapsed_time(evs[j + 1])
+    bd_step_ms = sum(e[0].elapsed_time(e[-1]) for e in bd_evs) / n_bd
+    if gu_total is None:
+        gu_total = per_kernel["gate_up"] * args.steps / n_bd
     total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms / args.steps
     value = whole_job_rate(world, T, args.steps, total_ms)
@@ -381,7 +404,7 @@ def main():
     cnt = counts.cpu()
     U = int((cnt > 0).sum())
     peaks, peak_src = load_peaks()
-    gu_ms = per_kernel["gate_up"] / args.steps
+    gu_ms = gu_total / args.steps
     gu_bytes = gate_up_bytes(cfg, U)
     achieved_gbs = gu_bytes / (gu_ms / 1e3) / 1e9
     traffic = ncu_traffic("grouped_gemm_gate_up", cfg.name)
@@ -412,7 +435,10 @@ def main():
             "achieved_tflops": F / (ms_per_step / 1e3) / 1e12,
             "achieved_gbs": B / (ms_per_step / 1e3) / 1e9,
         },
-        "kernel_ms": {n: v / args.steps for n, v in per_kernel.items()},
+        "kernel_ms": {n: v / n_bd for n, v in per_kernel.items()},
+        "kernel_ms_note": f"separate {n_bd}-step pass with every kernel boundary recorded "
+                          f"({bd_step_ms:.4f} ms/step there); timed steps recorded "
+                          f"{sorted(recorded)}",
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,

@@ -205,11 +205,13 @@ typedef struct moe_layer_params {
 /*
  * Step boundaries at which moe_layer_forward records p->step_events[i] on its stream when
  * step_events is not NULL (events created by the caller; used to time each kernel of the
- * layer).  Steps absent from a call (no shared expert) get a zero-length interval.
+ * layer; a NULL entry is skipped).  Steps absent from a call (no shared expert) get a
+ * zero-length interval.  An event recorded between two kernels stops the second from
+ * starting early (programmatic dependent launch), so record only the boundaries needed.
  */
 enum {
     MOE_EV_START = 0,    /* before the workspace clear */
-    MOE_EV_ROUTER,       /* router kernel (also clears the fp32 accumulator) */
+    MOE_EV_ROUTER,       /* router (one kernel, or GEMM + selection for T >= 256) */
     MOE_EV_PERMUTE,      /* permutation kernel */
     MOE_EV_GATE_UP,      /* grouped gate_up GEMM + SwiGLU (gathers the token rows) */
     MOE_EV_DOWN,         /* grouped down GEMM + weighted scatter-add */

@@ -47,6 +47,10 @@ SMALL_LAYERS = {
     "dense_E1": LayerConfig("dense_E1", T=33, D=256, E=1, K=1, f=384, seed=5),
     "all_experts": LayerConfig("all_experts", T=50, D=256, E=8, K=8, f=128, seed=6),
     "hot_rows": LayerConfig("hot_rows", T=300, D=256, E=4, K=2, f=128, seed=7),
+    # T >= 256 and E % 128 == 0: router logits on the tensor cores, shared gate in the
+    # selection kernel
+    "tc_router_shared": LayerConfig("tc_router_shared", T=300, D=384, E=128, K=6, f=128,
+                                    f_s=256, seed=8),
 }
 
 
@@ -90,7 +94,10 @@ def test_route_ties_go_to_lower_index(moe):
 
 
 @pytest.mark.parametrize("T,D,E,K", [(1, 128, 16, 4), (9, 256, 16, 16), (37, 1024, 64, 8),
-                                     (130, 512, 512, 10), (64, 2048, 256, 8), (5, 8192, 32, 3)])
+                                     (130, 512, 512, 10), (64, 2048, 256, 8), (5, 8192, 32, 3),
+                                     # tensor-core logits (T >= 256, E % 128 == 0)
+                                     (256, 128, 128, 8), (1000, 2048, 256, 8),
+                                     (777, 512, 512, 10), (4099, 4096, 128, 8)])
 def test_route_shapes(moe, oracle_mod, T, D, E, K):
     cfg = LayerConfig("r", T=T, D=D, E=E, K=K, f=128, seed=T + E)
     inp = make_inputs(cfg).to("cuda")

@@ -201,10 +201,14 @@ def launch_count() -> int:
 
 
 def event_array(events):
-    """ctypes array of raw cudaEvent_t handles of recorded ``torch.cuda.Event`` objects."""
+    """ctypes array of raw cudaEvent_t handles of recorded ``torch.cuda.Event`` objects
+    (None entries are not recorded by the layer)."""
     assert len(events) == NUM_STEP_EVENTS
     arr = (ctypes.c_void_p * NUM_STEP_EVENTS)()
     for i, e in enumerate(events):
+        if e is None:
+            arr[i] = None
+            continue
         if not e.cuda_event:
             raise ValueError("record each event once before passing it (creates the handle)")
         arr[i] = e.cuda_event

@@ -87,6 +87,12 @@ struct RouterLaunch {
 };
 cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bool pdl = false);
 
+// Router for many tokens: the logits x W_r^T [T, E] (fp32) on the tensor cores through the
+// grouped GEMM (one dense group), then a selection kernel.  Needs E % 128 == 0 and
+// a.logits with room for T*E floats.
+bool router_uses_tensor_cores(int T, int E);
+cudaError_t launch_router_tc(const RouterLaunch& a, int num_sms, cudaStream_t s, bool pdl = false);
+
 struct PermuteLaunch {
     const int32_t* topk_idx;
     const float* topk_w;
@@ -106,7 +112,7 @@ struct GroupedGemmLaunch {
     bool gate_up;               // true: SiLU(gate)*up epilogue -> h; false: down epilogue
     const void* w;              // weights: gate_up [E, 2f, D] or down [E, D, f]
     const void* act;            // activations: x [T, D] (gathered via gather_tok) or h [rows, f]
-    const int32_t* offsets;     // [E+1]
+    const int32_t* offsets;     // [E+1]; NULL: one dense group of `rows` rows (E must be 1)
     const int32_t* sorted_token;  // down only; NULL = identity
     const float* sorted_w;      // down only; NULL = 1
     int rows, E, D, f;
@@ -117,6 +123,7 @@ struct GroupedGemmLaunch {
     // gate_up only: when gather_tok != NULL, act is the token matrix x [T, D] and row r of
     // the expert-ordered problem is x[gather_tok[r]] (gathered inside the kernel)
     const int32_t* gather_tok;
+    int block_rows;  // rows per tile (16/32/64/128); 0 picks from the average group size
 };
 cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s,
                                 bool pdl = false);

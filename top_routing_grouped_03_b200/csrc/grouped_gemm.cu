@@ -62,7 +62,8 @@ struct Cfg {
 };
 
 struct Params {
-    const int32_t* offsets;
+    const int32_t* offsets;  // [G+1] row ranges; NULL: one group of rows_total rows
+    int rows_total;
     const int32_t* sorted_token;
     const float* sorted_w;
     int G;             // groups
@@ -167,7 +168,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
     // and the accumulator are produced by earlier kernels of the stream
     grid_dep_wait();
     grid_dep_launch();
-    for (int i = threadIdx.x; i <= p.G; i += kThreads) g_off[i] = p.offsets[i];
+    for (int i = threadIdx.x; i <= p.G; i += kThreads)
+        g_off[i] = p.offsets ? p.offsets[i] : (i == 0 ? 0 : p.rows_total);
     __syncthreads();
     if (warp == 2) {
         // tile prefix over groups: lane l owns a contiguous run of groups
@@ -442,7 +444,8 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
     if (a.E > kMaxGroups) return cudaErrorInvalidValue;
     cudaError_t err = get_encoder();
     if (err != cudaSuccess) return err;
-    const int BN = pick_block_rows(a.rows, a.E);
+    const int BN = a.block_rows ? a.block_rows : pick_block_rows(a.rows, a.E);
+    if (BN != 16 && BN != 32 && BN != 64 && BN != 128) return cudaErrorInvalidValue;
     const int K = a.gate_up ? a.D : a.f;
     const uint64_t w_group_rows = a.gate_up ? 2ull * a.f : static_cast<uint64_t>(a.D);
     CUtensorMap mw, ma;
@@ -454,6 +457,7 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
         return err;
     Params p{};
     p.offsets = a.offsets;
+    p.rows_total = a.rows;
     p.sorted_token = a.sorted_token;
     p.sorted_w = a.sorted_w;
     p.G = a.E;

@@ -145,7 +145,10 @@ int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* logit_bi
     a.counts = expert_counts;
     a.shared_gate = shared_gate;
     a.status = at<int>(workspace, L.status);
-    return launch_router(a, num_sms_current(), s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    const int sms = num_sms_current();
+    const cudaError_t err = router_uses_tensor_cores(T, E) ? launch_router_tc(a, sms, s)
+                                                           : launch_router(a, sms, s);
+    return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int moe_permute(const int32_t* topk_idx, const float* topk_w, const int32_t* expert_counts, int T,
@@ -262,7 +265,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     const int sms = num_sms_current();
     const bool det = (p->flags & MOE_FLAG_DETERMINISTIC) != 0;
     auto mark = [&](int i) {
-        return p->step_events == nullptr ||
+        return p->step_events == nullptr || p->step_events[i] == nullptr ||
                cudaEventRecord(reinterpret_cast<cudaEvent_t>(p->step_events[i]), s) == cudaSuccess;
     };
     int* status = at<int>(workspace, L.status);
@@ -295,7 +298,10 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     r.status = status;
     r.zero_acc = use_acc ? out_acc : nullptr;
     r.zero_cols = D;
-    if (!mark(MOE_EV_ROUTER) || launch_router(r, sms, s, false) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!mark(MOE_EV_ROUTER)) return MOE_ERR_CUDA;
+    if ((router_uses_tensor_cores(T, E) ? launch_router_tc(r, sms, s) : launch_router(r, sms, s)) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
 
     PermuteLaunch pm{};
     pm.topk_idx = idx;

@@ -15,6 +15,9 @@
 //     denominator cancels in the renormalisation, so only the K selected terms are
 //     exponentiated.
 //   * expert_counts[e] += 1 per selected expert (global atomics, for the permutation).
+// For many tokens (T >= 256, E a multiple of 128) the logits instead come from the
+// tcgen05 grouped GEMM as one dense [T, E] product, and router_select_kernel runs the
+// same selection with one warp per token.
 #include <cfloat>
 
 #include "common.cuh"
@@ -25,6 +28,52 @@ namespace {
 constexpr int kTokensPerCta = 8;
 constexpr int kRouterThreads = 256;
 constexpr int kMaxExpertsPerLane = 16;  // E <= 512
+
+// TopK of one token's logits by one warp, in registers, then the renormalised weights.
+// lg: the token's E logits (bias already added when add_bias is NULL).  Writes idx/w of
+// the token and adds its K experts to the counts.
+__device__ __forceinline__ void select_topk_warp(const float* lg, const float* add_bias, int E,
+                                                 int K, int token, int lane, int32_t* topk_idx,
+                                                 float* topk_w, int32_t* counts) {
+    float v[kMaxExpertsPerLane];
+#pragma unroll
+    for (int j = 0; j < kMaxExpertsPerLane; ++j) {
+        const int e = j * 32 + lane;
+        v[j] = (e < E) ? __ldcg(lg + e) + (add_bias ? __ldg(add_bias + e) : 0.f) : -FLT_MAX;
+    }
+    float my_v = -FLT_MAX;
+    int my_i = 0;
+    for (int k = 0; k < K; ++k) {
+        float bv = -FLT_MAX;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < kMaxExpertsPerLane; ++j) {
+            const int e = j * 32 + lane;
+            if (e < E && v[j] > bv) { bv = v[j]; bi = e; }  // strict: lowest e per lane
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+        }
+        if (lane == k) { my_v = bv; my_i = bi; }
+        // retire the winner (owner lane only); -inf never wins against finite logits
+#pragma unroll
+        for (int j = 0; j < kMaxExpertsPerLane; ++j)
+            if (j * 32 + lane == bi) v[j] = -INFINITY;
+    }
+    const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
+    const float ex = (lane < K) ? expf(my_v - vmax) : 0.f;
+    float sum = ex;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane < K) {
+        topk_idx[static_cast<size_t>(token) * K + lane] = my_i;
+        topk_w[static_cast<size_t>(token) * K + lane] = ex / sum;
+        atomicAdd(&counts[my_i], 1);
+    }
+}
 
 __global__ void __launch_bounds__(kRouterThreads)
 router_kernel(RouterLaunch a, int experts_per_cta) {
@@ -124,48 +173,51 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
     for (int t = warp; t < nt; t += kRouterThreads / 32) {
         const int token = t0 + t;
         const float* lg = a.logits + static_cast<size_t>(token) * (E + 1);
-        float v[kMaxExpertsPerLane];
-#pragma unroll
-        for (int j = 0; j < kMaxExpertsPerLane; ++j) {
-            const int e = j * 32 + lane;
-            v[j] = (e < E) ? __ldcg(lg + e) : -FLT_MAX;
-        }
-        float my_v = -FLT_MAX;
-        int my_i = 0;
-        for (int k = 0; k < a.K; ++k) {
-            float bv = -FLT_MAX;
-            int bi = 0x7fffffff;
-#pragma unroll
-            for (int j = 0; j < kMaxExpertsPerLane; ++j) {
-                const int e = j * 32 + lane;
-                if (e < E && v[j] > bv) { bv = v[j]; bi = e; }  // strict: lowest e per lane
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-                if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-            }
-            if (lane == k) { my_v = bv; my_i = bi; }
-            // retire the winner (owner lane only); -inf never wins against finite logits
-#pragma unroll
-            for (int j = 0; j < kMaxExpertsPerLane; ++j)
-                if (j * 32 + lane == bi) v[j] = -INFINITY;
-        }
-        const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
-        float ex = (lane < a.K) ? expf(my_v - vmax) : 0.f;
-        float sum = ex;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        if (lane < a.K) {
-            a.topk_idx[static_cast<size_t>(token) * a.K + lane] = my_i;
-            a.topk_w[static_cast<size_t>(token) * a.K + lane] = ex / sum;
-            atomicAdd(&a.counts[my_i], 1);
-        }
+        select_topk_warp(lg, nullptr, E, a.K, token, lane, a.topk_idx, a.topk_w, a.counts);
         if (a.w_shared_gate && lane == 0) {
             const float g = __ldcg(lg + E);
             a.shared_gate[token] = 1.f / (1.f + expf(-g));
         }
+    }
+}
+
+
+// Selection after the tensor-core logits: one warp per token over logits [T, E] (no bias
+// yet), the bias added on load; the shared gate's dot product w_s . x_t is done here by
+// the same warp; the block also clears its tokens' rows of the layer accumulator.
+__global__ void __launch_bounds__(kRouterThreads) router_select_kernel(RouterLaunch a) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = blockIdx.x * (kRouterThreads / 32);
+    const int nt = min(kRouterThreads / 32, a.T - t0);
+    grid_dep_wait();  // logits come from the GEMM
+    grid_dep_launch();
+    if (a.zero_acc) {
+        float4* dst = reinterpret_cast<float4*>(a.zero_acc + static_cast<size_t>(t0) * a.zero_cols);
+        for (int i = threadIdx.x; i < nt * a.zero_cols / 4; i += kRouterThreads)
+            dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (warp >= nt) return;
+    const int token = t0 + warp;
+    select_topk_warp(a.logits + static_cast<size_t>(token) * a.E, a.logit_bias, a.E, a.K, token,
+                     lane, a.topk_idx, a.topk_w, a.counts);
+    if (a.w_shared_gate) {
+        const uint4* xv = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(token) * a.D);
+        const uint4* wv = reinterpret_cast<const uint4*>(a.w_shared_gate);
+        float acc = 0.f;
+        for (int c = lane; c < a.D / 8; c += 32) {
+            const uint4 x8 = __ldg(xv + c), w8 = __ldg(wv + c);
+            acc = fmaf(bf16_lo(x8.x), bf16_lo(w8.x), acc);
+            acc = fmaf(bf16_hi(x8.x), bf16_hi(w8.x), acc);
+            acc = fmaf(bf16_lo(x8.y), bf16_lo(w8.y), acc);
+            acc = fmaf(bf16_hi(x8.y), bf16_hi(w8.y), acc);
+            acc = fmaf(bf16_lo(x8.z), bf16_lo(w8.z), acc);
+            acc = fmaf(bf16_hi(x8.z), bf16_hi(w8.z), acc);
+            acc = fmaf(bf16_lo(x8.w), bf16_lo(w8.w), acc);
+            acc = fmaf(bf16_hi(x8.w), bf16_hi(w8.w), acc);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) a.shared_gate[token] = 1.f / (1.f + expf(-acc));
     }
 }
 
@@ -187,6 +239,35 @@ cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bo
     if (err != cudaSuccess) return err;
     err = launch_kernel(router_kernel, dim3(n_tb, n_eb), dim3(kRouterThreads), smem, s, pdl, a,
                         per_cta);
+    count_launches(1);
+    return err;
+}
+
+
+bool router_uses_tensor_cores(int T, int E) { return T >= 256 && E % 128 == 0; }
+
+cudaError_t launch_router_tc(const RouterLaunch& a, int num_sms, cudaStream_t s, bool pdl) {
+    if (a.T == 0) return cudaSuccess;
+    // logits = x W_r^T: W_r's E rows on the MMA's M side, tokens on N, one dense group;
+    // the tile height is chosen so that the (E/128) x (T/rows) tiles cover the GPU
+    GroupedGemmLaunch g{};
+    g.gate_up = false;
+    g.w = a.w_router;
+    g.act = a.x;
+    g.offsets = nullptr;
+    g.rows = a.T;
+    g.E = 1;
+    g.D = a.E;  // output features
+    g.f = a.D;  // reduction length
+    g.y_out = a.logits;
+    g.status = a.status;
+    g.block_rows = 16;
+    for (int bn = 128; bn >= 16; bn /= 2)
+        if ((a.E / 128) * ceil_div(a.T, bn) >= num_sms) { g.block_rows = bn; break; }
+    cudaError_t err = launch_grouped_gemm(g, num_sms, s, pdl);
+    if (err != cudaSuccess) return err;
+    err = launch_kernel(router_select_kernel, dim3(ceil_div(a.T, kRouterThreads / 32)),
+                        dim3(kRouterThreads), 0, s, true, a);
     count_launches(1);
     return err;
 }
