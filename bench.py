@@ -6,7 +6,8 @@
 One step = one whole layer call (router, permutation, gather, grouped gate_up + SwiGLU,
 grouped down + weighted combine, bf16 output) over one batch of synthetic tokens already
 resident in HBM.  L2 is flushed (512 MiB write) before every timed step, outside the timed
-interval; each step is timed with CUDA events recorded by the library on its own stream,
+interval (the flush writes one 512 MiB buffer and reads another, so L2 starts each step
+with clean lines); each step is timed with CUDA events recorded by the library on its stream,
 and the per-kernel intervals come from the same events.  With N > 1 (torchrun, one
 process per GPU) every rank runs an independent replica of the batch (no exchange): the
 reported value is all ranks' tokens over the slowest rank's time.
@@ -303,9 +304,22 @@ def main():
     idx = torch.empty((T, K), dtype=torch.int32, device=dev)
     tw = torch.empty((T, K), dtype=torch.float32, device=dev)
     counts = torch.empty((E,), dtype=torch.int32, device=dev)
-    flush = torch.empty(max(args.flush_mib, 1) << 20, dtype=torch.uint8, device=dev)
-    if args.flush_mib == 0:
-        flush = flush[:0]
+    # L2 flush between timed steps: write one buffer larger than L2, then read another,
+    # so L2 holds clean lines when a step starts (the write-back of the dirty lines the
+    # write leaves happens during the read, outside the timed interval)
+    nflush = max(args.flush_mib, 1) << 20
+    flush_w = torch.empty(nflush, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(nflush // 4, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    class _Flush:
+        def fill_(self, v):
+            if args.flush_mib == 0:
+                return
+            flush_w.fill_(v)
+            torch.sum(flush_r, dim=0, out=flush_sink)
+
+    flush = _Flush()
     stream = torch.cuda.current_stream()
 
     names = moe.STEP_EVENT_NAMES
@@ -417,8 +431,8 @@ def main():
         "config": {
             "workload": describe(cfg), "global_batch": world * T, "tokens_per_gpu": T,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "l2": "flushed before every timed step (512 MiB write); expert weights read per "
-                  "step exceed L2",
+            "l2": "flushed before every timed step (512 MiB write, then 512 MiB read), "
+                  "outside the timed interval; expert weights read per step exceed L2",
             "routing_U": U, "max_rows_per_expert": int(cnt.max()),
             "deterministic_combine": bool(args.deterministic),
         },

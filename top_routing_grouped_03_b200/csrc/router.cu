@@ -158,6 +158,7 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
                 a.logits[static_cast<size_t>(t0 + t) * (E + 1) + e] = acc[t] + b;
         }
     }
+    __threadfence();  // this thread's logits are visible device-wide before the ticket
 
     // ---- ticket: the last CTA of this token block does the selection
     __syncthreads();
