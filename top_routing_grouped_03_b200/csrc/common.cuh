@@ -123,7 +123,8 @@ struct GroupedGemmLaunch {
     // gate_up only: when gather_tok != NULL, act is the token matrix x [T, D] and row r of
     // the expert-ordered problem is x[gather_tok[r]] (gathered inside the kernel)
     const int32_t* gather_tok;
-    int block_rows;  // rows per tile (16/32/64/128); 0 picks from the average group size
+    int block_rows;   // rows per tile (16/32/64/128); 0 picks from the average group size
+    int orientation;  // 0: auto; 1: weights on the MMA's M side; 2: tokens on M
 };
 cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s,
                                 bool pdl = false);

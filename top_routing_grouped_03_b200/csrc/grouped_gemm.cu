@@ -119,6 +119,75 @@ __device__ __forceinline__ Tile decode_tile(int tile, const int* g_tile, const i
     return t;
 }
 
+// The group table every role of a CTA walks: g_off = row offsets of the groups (from the
+// device, or {0, rows_total} for one dense group); g_tile[g] = first tile of group g, where a
+// group of n rows has ceil(n / rows_per_tile) * nf tiles; g_tile[G] = total.
+__device__ __forceinline__ void build_tile_table(const Params& p, int rows_per_tile, int* g_off,
+                                                 int* g_tile, int* total_slot, int warp,
+                                                 int lane) {
+    for (int i = threadIdx.x; i <= p.G; i += kThreads)
+        g_off[i] = p.offsets ? p.offsets[i] : (i == 0 ? 0 : p.rows_total);
+    __syncthreads();
+    if (warp == 2) {
+        // tile prefix over groups: lane l owns a contiguous run of groups
+        const int per = (p.G + 31) / 32;
+        const int gb = min(lane * per, p.G), ge = min(gb + per, p.G);
+        int local = 0;
+        for (int g = gb; g < ge; ++g)
+            local += ((g_off[g + 1] - g_off[g] + rows_per_tile - 1) / rows_per_tile) * p.nf;
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - local;
+        for (int g = gb; g < ge; ++g) {
+            g_tile[g] = run;
+            run += ((g_off[g + 1] - g_off[g] + rows_per_tile - 1) / rows_per_tile) * p.nf;
+        }
+        if (lane == 31) {
+            g_tile[p.G] = incl;
+            *total_slot = incl;
+        }
+    }
+}
+
+// Per-lane plan for gathering ROWS token rows of x into a 128-byte-swizzled operand tile
+// with cp.async: lane l owns 16-byte chunk c = l % 8 of tile rows l/8 + 4u; that chunk of
+// tile row r lands at r*128 + ((c ^ (r % 8)) * 16).
+template <int ROWS>
+struct RowGather {
+    static constexpr int kChunks = ROWS * 8 / 32;
+    uint32_t src_off[kChunks];  // element offset of the chunk's row in x (< 2^31)
+    uint32_t valid;
+
+    __device__ __forceinline__ void plan(const int32_t* tok, int row0, int row_end, int row_len,
+                                         int lane) {
+        valid = 0;
+#pragma unroll
+        for (int u = 0; u < kChunks; ++u) {
+            const int row = row0 + (lane >> 3) + 4 * u;
+            const bool ok = row < row_end;
+            const int t = ok ? __ldg(tok + row) : 0;
+            src_off[u] = static_cast<uint32_t>(t) * row_len + (lane & 7) * 8;
+            valid |= (ok ? 1u : 0u) << u;
+        }
+    }
+
+    // copies columns [k0, k0 + 64) of the planned rows into the tile at smem_tile
+    __device__ __forceinline__ void issue(uint32_t smem_tile, const bf16* x, int k0,
+                                          int lane) const {
+        const int c = lane & 7;
+#pragma unroll
+        for (int u = 0; u < kChunks; ++u) {
+            const int r = (lane >> 3) + 4 * u;
+            cp_async_16(smem_tile + r * 128 + ((c ^ (r & 7)) << 4), x + src_off[u] + k0,
+                        ((valid >> u) & 1u) ? 16u : 0u);
+        }
+    }
+};
+
 template <int BN, bool GATE_UP>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
@@ -168,31 +237,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
     // and the accumulator are produced by earlier kernels of the stream
     grid_dep_wait();
     grid_dep_launch();
-    for (int i = threadIdx.x; i <= p.G; i += kThreads)
-        g_off[i] = p.offsets ? p.offsets[i] : (i == 0 ? 0 : p.rows_total);
-    __syncthreads();
-    if (warp == 2) {
-        // tile prefix over groups: lane l owns a contiguous run of groups
-        const int per = (p.G + 31) / 32;
-        const int gb = min(lane * per, p.G), ge = min(gb + per, p.G);
-        int local = 0;
-        for (int g = gb; g < ge; ++g) local += ((g_off[g + 1] - g_off[g] + BN - 1) / BN) * p.nf;
-        int incl = local;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        int run = incl - local;
-        for (int g = gb; g < ge; ++g) {
-            g_tile[g] = run;
-            run += ((g_off[g + 1] - g_off[g] + BN - 1) / BN) * p.nf;
-        }
-        if (lane == 31) {
-            g_tile[p.G] = incl;
-            *total_slot = incl;
-        }
-    }
+    build_tile_table(p, BN, g_off, g_tile, total_slot, warp, lane);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -203,33 +248,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
         // ---------------------------------------------------------------- producer
         // Weights (operand A) always by TMA from lane 0.  Activation rows (operand B): one
         // TMA box when they are contiguous in expert order; otherwise (gather) each lane
-        // copies 16-byte chunks of x[gather_tok[row]] with cp.async into the swizzled tile:
-        // chunk c of tile row r lands at r*128 + ((c ^ (r % 8)) * 16).  Lane l always owns
-        // chunk c = l % 8 of rows l/8 + 4u.
-        constexpr int kChunks = BN * 8 / 32;
+        // copies 16-byte chunks of x[gather_tok[row]] with cp.async into the swizzled tile
+        // (RowGather).
         if (gather || lane == 0) {
             const uint64_t pol_w = policy_evict_first();  // weights stream through once
             const uint64_t pol_a = policy_evict_last();   // activations are re-read
             const uint32_t a_bytes = C::kNumA * C::kABytes;
-            const int c = lane & 7;
             int stage = 0;
             uint32_t phase = 0, filled = 0, fill_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
                 const Tile t = decode_tile(tile, g_tile, g_off, p.G, BN);
                 const int wr0 = t.g * p.w_group_rows + t.i * kBM;
-                uint32_t src_off[kChunks];  // element offset of the chunk in x (< 2^31)
-                uint32_t valid_mask = 0;
-                if (gather) {
-#pragma unroll
-                    for (int u = 0; u < kChunks; ++u) {
-                        const int row = t.row0 + (lane >> 3) + 4 * u;
-                        const bool valid = row < t.row_end;
-                        const int tok = valid ? __ldg(p.gather_tok + row) : 0;
-                        src_off[u] = static_cast<uint32_t>(tok) * (p.nk * kBK) + c * 8;
-                        valid_mask |= (valid ? 1u : 0u) << u;
-                    }
-                }
+                RowGather<BN> rg;
+                if (gather) rg.plan(p.gather_tok, t.row0, t.row_end, p.nk * kBK, lane);
                 for (int kk = 0; kk < p.nk; ++kk) {
                     bool got = mbar_wait(&empty[stage], phase ^ 1u, kWaitBudgetNs, abort_flag);
                     if (gather) got = __all_sync(0xffffffffu, got);
@@ -251,14 +283,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                                         pol_a);
                     }
                     if (gather) {
-                        const uint32_t b0 = smem_u32(st + a_bytes);
-#pragma unroll
-                        for (int u = 0; u < kChunks; ++u) {
-                            const int r = (lane >> 3) + 4 * u;
-                            cp_async_16(b0 + r * 128 + ((c ^ (r & 7)) << 4),
-                                        p.x + src_off[u] + kk * kBK,
-                                        ((valid_mask >> u) & 1u) ? 16u : 0u);
-                        }
+                        rg.issue(smem_u32(st + a_bytes), p.x, kk * kBK, lane);
                         cp_async_mbar_arrive_noinc(&full[stage]);
                     }
                     filled |= 1u << stage;
@@ -383,6 +408,272 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
     }
 }
 
+// ---------------------------------------------------------------- tokens-on-M variant
+// For groups with many rows: the MMA's M side holds 128 token rows and its N side 256
+// weight rows (gate_up: the gate and up rows of the same 128 features; down: 256 output
+// features), one tcgen05.mma of 128 x 256 x 16 per 16 of K.  Per tile: 128 rows x 128 h
+// features (gate_up) or 128 rows x 256 output features (down).  Each epilogue thread owns
+// one row, so h is written with 16-byte stores and the down epilogue reduces 16-byte
+// vectors (red.global.add.v4.f32) into the token's output row.
+constexpr int kTmRows = 128;  // token rows per tile (MMA M)
+constexpr int kTmN = 256;     // weight rows per tile (MMA N)
+
+template <bool GATE_UP>
+struct CfgTm {
+    static constexpr int kABytes = kTmRows * kBK * 2;  // 16 KB of token rows
+    static constexpr int kBBytes = kTmN * kBK * 2;     // 32 KB of weight rows
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = 4;
+    static constexpr int kAccCols = kTmN;
+    static constexpr int kTmemCols = 2 * kAccCols;
+    static_assert(kTmemCols <= 512, "accumulators exceed tensor memory");
+};
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+                 "f"(c), "f"(d)
+                 : "memory");
+}
+
+template <bool GATE_UP>
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
+                       const __grid_constant__ CUtensorMap map_act, Params p) {
+    using C = CfgTm<GATE_UP>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+    uint64_t* empty = full + C::kStages;
+    uint64_t* tfull = empty + C::kStages;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* total_slot = reinterpret_cast<int*>(tmem_slot + 2);
+    int* g_off = reinterpret_cast<int*>(tmem_slot + 4);
+    int* g_tile = g_off + (p.G + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const bool gather = GATE_UP && p.gather_tok != nullptr;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], gather ? 1 + 32 : 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], kEpiThreads);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&map_w);
+        if (!gather) tma_prefetch_desc(&map_act);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    grid_dep_wait();
+    grid_dep_launch();
+    build_tile_table(p, kTmRows, g_off, g_tile, total_slot, warp, lane);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = *total_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        // token rows (A): one TMA box of 128 rows when contiguous, else the lanes gather
+        // them with cp.async; weight rows (B): two TMA boxes of 128 rows.
+        if (gather || lane == 0) {
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_a = policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0, filled = 0, fill_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const Tile t = decode_tile(tile, g_tile, g_off, p.G, kTmRows);
+                // gate_up: gate rows g*2f + i*128 and up rows g*2f + f + i*128;
+                // down: rows g*D + i*256 and the next 128
+                const int wr0 = t.g * p.w_group_rows + t.i * (GATE_UP ? kBM : kTmN);
+                const int wr1 = GATE_UP ? wr0 + p.up_rows : wr0 + kBM;
+                RowGather<kTmRows> rg;
+                if (gather) rg.plan(p.gather_tok, t.row0, t.row_end, p.nk * kBK, lane);
+                for (int kk = 0; kk < p.nk; ++kk) {
+                    bool got = mbar_wait(&empty[stage], phase ^ 1u, kWaitBudgetNs, abort_flag);
+                    if (gather) got = __all_sync(0xffffffffu, got);
+                    if (!got) {
+                        set_status(p.status, MOE_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* st = smem + stage * C::kStageBytes;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&full[stage], gather ? C::kBBytes : C::kStageBytes);
+                        if (!gather)
+                            tma_load_2d(st, &map_act, &full[stage], kk * kBK, t.row0, pol_a);
+                        tma_load_2d(st + C::kABytes, &map_w, &full[stage], kk * kBK, wr0, pol_w);
+                        tma_load_2d(st + C::kABytes + kBM * kBK * 2, &map_w, &full[stage],
+                                    kk * kBK, wr1, pol_w);
+                    }
+                    if (gather) {
+                        rg.issue(smem_u32(st), p.x, kk * kBK, lane);
+                        cp_async_mbar_arrive_noinc(&full[stage]);
+                    }
+                    filled |= 1u << stage;
+                    fill_phase = (fill_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (gather) cp_async_wait_all();
+            if (!ok && lane == 0) {
+                for (int s = 0; s < C::kStages; ++s)
+                    if (filled & (1u << s))
+                        mbar_wait(&full[s], (fill_phase >> s) & 1u, kDrainBudgetNs, nullptr);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(kTmRows, kTmN);
+            int stage = 0;
+            uint32_t phase = 0, abuf = 0, aphase = 0;
+            bool ok = true, issued = false;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                if (!mbar_wait(&tempty[abuf], aphase ^ 1u, kWaitBudgetNs, abort_flag)) {
+                    set_status(p.status, MOE_ERR_TIMEOUT);
+                    *abort_flag = 1;
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + abuf * C::kAccCols;
+                for (int kk = 0; kk < p.nk; ++kk) {
+                    if (!mbar_wait(&full[stage], phase, kWaitBudgetNs, abort_flag)) {
+                        set_status(p.status, MOE_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (gather) fence_proxy_async_smem();
+                    const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
+                    const uint32_t b0 = a0 + C::kABytes;
+#pragma unroll
+                    for (int s = 0; s < kBK / 16; ++s)
+                        umma_bf16(d0, sdesc_k_sw128(a0 + s * 32), sdesc_k_sw128(b0 + s * 32), idesc,
+                                  (kk | s) != 0 ? 1u : 0u);
+                    issued = true;
+                    umma_commit(&empty[stage]);
+                    if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                umma_commit(&tfull[abuf]);
+                abuf ^= 1u;
+                if (abuf == 0) aphase ^= 1u;
+            }
+            if (!ok && issued) {
+                umma_commit(drain);
+                mbar_wait(drain, 0, kDrainBudgetNs, nullptr);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- epilogue
+        const int q = warp & 3;
+        uint32_t abuf = 0, aphase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const Tile t = decode_tile(tile, g_tile, g_off, p.G, kTmRows);
+            const bool ready = mbar_wait(&tfull[abuf], aphase, kWaitBudgetNs, abort_flag);
+            if (!epilogue_bar_and(ready)) {
+                set_status(p.status, MOE_ERR_TIMEOUT);
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   abuf * C::kAccCols;
+            const int row = t.row0 + q * 32 + lane;
+            const bool valid = row < t.row_end;
+            if (GATE_UP) {
+                bf16* hrow = p.h_out + static_cast<size_t>(row) * p.out_cols + t.i * kBM;
+#pragma unroll 1
+                for (int c0 = 0; c0 < kBM; c0 += 16) {
+                    uint32_t gv[16], uv[16];
+                    tmem_ld16(tbase + c0, gv);
+                    tmem_ld16(tbase + kBM + c0, uv);
+                    tmem_ld_wait();
+                    if (valid) {
+                        uint32_t pk[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float g0 = __uint_as_float(gv[2 * j]);
+                            const float g1 = __uint_as_float(gv[2 * j + 1]);
+                            const float h0 = g0 / (1.f + __expf(-g0)) * __uint_as_float(uv[2 * j]);
+                            const float h1 = g1 / (1.f + __expf(-g1)) * __uint_as_float(uv[2 * j + 1]);
+                            pk[j] = pack_bf16x2(h0, h1);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(hrow + c0);
+                        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    }
+                }
+            } else {
+                const float w = (valid && p.sorted_w) ? __ldg(p.sorted_w + row) : 1.f;
+                const int tok = valid ? (p.sorted_token ? __ldg(p.sorted_token + row) : row) : 0;
+                const int col0 = t.i * kTmN;
+#pragma unroll 1
+                for (int c0 = 0; c0 < kTmN; c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld16(tbase + c0, v);
+                    tmem_ld_wait();
+                    if (valid) {
+                        if (p.acc_out) {
+                            float* dst = p.acc_out + static_cast<size_t>(tok) * p.out_cols + col0 + c0;
+#pragma unroll
+                            for (int j = 0; j < 16; j += 4)
+                                red_add_v4(dst + j, w * __uint_as_float(v[j]),
+                                           w * __uint_as_float(v[j + 1]),
+                                           w * __uint_as_float(v[j + 2]),
+                                           w * __uint_as_float(v[j + 3]));
+                        }
+                        if (p.y_out) {
+                            float4* dst = reinterpret_cast<float4*>(
+                                p.y_out + static_cast<size_t>(row) * p.out_cols + col0 + c0);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                dst[j] = make_float4(w * __uint_as_float(v[4 * j]),
+                                                     w * __uint_as_float(v[4 * j + 1]),
+                                                     w * __uint_as_float(v[4 * j + 2]),
+                                                     w * __uint_as_float(v[4 * j + 3]));
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[abuf]);
+            abuf ^= 1u;
+            if (abuf == 0) aphase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
 // ---------------------------------------------------------------- host side
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -428,6 +719,21 @@ cudaError_t launch_tpl(const CUtensorMap& mw, const CUtensorMap& ma, const Param
     return err;
 }
 
+template <bool GATE_UP>
+cudaError_t launch_tm(const CUtensorMap& mw, const CUtensorMap& ma, const Params& p, int grid,
+                      cudaStream_t s, bool pdl) {
+    using C = CfgTm<GATE_UP>;
+    const size_t smem = 1024 + static_cast<size_t>(C::kStages) * C::kStageBytes +
+                        (2 * C::kStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int);
+    auto kfn = grouped_gemm_tm_kernel<GATE_UP>;
+    cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    err = launch_kernel(kfn, dim3(grid), dim3(kThreads), smem, s, pdl, mw, ma, p);
+    count_launches(1);
+    return err;
+}
+
 }  // namespace
 
 int pick_block_rows(int rows, int groups) {
@@ -444,12 +750,17 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
     if (a.E > kMaxGroups) return cudaErrorInvalidValue;
     cudaError_t err = get_encoder();
     if (err != cudaSuccess) return err;
-    const int BN = a.block_rows ? a.block_rows : pick_block_rows(a.rows, a.E);
+    // orientation: tokens on the MMA's M side once the groups average a full 128-row tile
+    // (and the output width splits into 256-wide blocks for down); weights on M otherwise
+    const bool tm_ok = a.gate_up ? (a.f % 128 == 0) : (a.D % 256 == 0);
+    const bool tm = tm_ok && (a.orientation == 2 ||
+                              (a.orientation == 0 && a.block_rows == 0 && a.rows / a.E >= 128));
+    const int BN = tm ? kTmRows : (a.block_rows ? a.block_rows : pick_block_rows(a.rows, a.E));
     if (BN != 16 && BN != 32 && BN != 64 && BN != 128) return cudaErrorInvalidValue;
     const int K = a.gate_up ? a.D : a.f;
     const uint64_t w_group_rows = a.gate_up ? 2ull * a.f : static_cast<uint64_t>(a.D);
     CUtensorMap mw, ma;
-    if ((err = make_map(&mw, a.w, w_group_rows * a.E, K, kBM)) != cudaSuccess) return err;
+    if ((err = make_map(&mw, a.w, w_group_rows * a.E, K, kBM)) != cudaSuccess) return err;  // 128-row boxes
     // the activation map is only read when the rows are contiguous (no gather); with a
     // gather it still has to be a valid descriptor, so it covers the first row of x
     const bool gather = a.gate_up && a.gather_tok != nullptr;
@@ -461,7 +772,7 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
     p.sorted_token = a.sorted_token;
     p.sorted_w = a.sorted_w;
     p.G = a.E;
-    p.nf = (a.gate_up ? a.f : a.D) / kBM;
+    p.nf = a.gate_up ? a.f / kBM : a.D / (tm ? kTmN : kBM);
     p.nk = K / kBK;
     p.w_group_rows = static_cast<int>(w_group_rows);
     p.up_rows = a.f;
@@ -474,6 +785,8 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
     p.x = reinterpret_cast<const bf16*>(a.act);
     const long long max_tiles = (static_cast<long long>(ceil_div(a.rows, BN)) + a.E) * p.nf;
     const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
+    if (tm) return a.gate_up ? launch_tm<true>(mw, ma, p, grid, s, pdl)
+                             : launch_tm<false>(mw, ma, p, grid, s, pdl);
     switch (BN) {
         case 16: return a.gate_up ? launch_tpl<16, true>(mw, ma, p, grid, s, pdl) : launch_tpl<16, false>(mw, ma, p, grid, s, pdl);
         case 32: return a.gate_up ? launch_tpl<32, true>(mw, ma, p, grid, s, pdl) : launch_tpl<32, false>(mw, ma, p, grid, s, pdl);

@@ -63,6 +63,9 @@ CONFIGS = {
     "prefill": LayerConfig("prefill", T=8192, D=4096, E=128, K=8, f=1536),
     "finegrained": LayerConfig("finegrained", T=4096, D=4096, E=512, K=10, f=1024, f_s=1024),
 }
+# the prefill layer's per-expert shape (512 rows per expert, D=4096, f=1536) with 32 experts:
+# the same kernels and tiles on ~1.2 GB of weights, small enough for profiler captures
+CONFIGS["prefill_e32"] = LayerConfig("prefill_e32", T=2048, D=4096, E=32, K=8, f=1536)
 ZIPF_TOKENS = (1, 16, 128, 1024, 16384)
 for _t in ZIPF_TOKENS:
     CONFIGS[f"zipf@T{_t}"] = LayerConfig(f"zipf@T{_t}", T=_t, D=4096, E=128, K=8, f=1536,
