@@ -125,6 +125,11 @@ struct GroupedGemmLaunch {
     const int32_t* gather_tok;
     int block_rows;   // rows per tile (16/32/64/128); 0 picks from the average group size
     int orientation;  // 0: auto; 1: weights on the MMA's M side; 2: tokens on M
+    // down with acc_out: when final_out and done are set, the kernel converts acc_out
+    // [final_rows, D] to bf16 in final_out after all its CTAs finished (done = 0 at launch)
+    bf16* final_out;
+    int final_rows;
+    unsigned* done;
 };
 cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s,
                                 bool pdl = false);

@@ -78,7 +78,50 @@ struct Params {
     int* status;
     const int32_t* gather_tok;  // gate_up: B rows are x[gather_tok[row]] (cp.async), or NULL
     const bf16* x;              // the token matrix the gather reads, [*, K] bf16
+    bf16* final_out;            // down: when set, convert acc_out [final_rows, out_cols] to
+    int final_rows;             //   bf16 here once every CTA of the grid has added its tiles
+    unsigned* done;             //   (grid barrier counter, zero at launch)
 };
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// The layer's last down launch finishes the output: every thread fences its reductions,
+// each CTA takes a ticket, all CTAs wait (bounded) until the whole grid has arrived --
+// the grid is persistent with at most one CTA per SM, so all of it is resident -- and
+// then convert a grid-stride share of the fp32 accumulator to bf16.
+__device__ __noinline__ void finalize_output(const Params& p) {
+    __shared__ int s_ok;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        atomicAdd(p.done, 1u);
+        int ok = 1;
+        const uint64_t t0 = global_timer_ns();
+        while (ld_acquire_gpu(p.done) < gridDim.x) {
+            if (global_timer_ns() - t0 > kWaitBudgetNs) {
+                set_status(p.status, MOE_ERR_TIMEOUT);
+                ok = 0;
+                break;
+            }
+            __nanosleep(64);
+        }
+        s_ok = ok;
+    }
+    __syncthreads();
+    if (!s_ok) return;
+    const long long n4 = static_cast<long long>(p.final_rows) * p.out_cols / 4;
+    const float4* src = reinterpret_cast<const float4*>(p.acc_out);
+    uint2* dst = reinterpret_cast<uint2*>(p.final_out);
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const float4 v = __ldcg(src + i);
+        dst[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+    }
+}
 
 // Named barrier 1 of the four epilogue warps with an AND across their threads: all of
 // them take the same branch afterwards, so a wait that gives up in one warp makes every
@@ -406,6 +449,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
         tc_fence_after();
         tmem_dealloc(tmem_base, C::kTmemCols);
     }
+    if (!GATE_UP && p.final_out != nullptr) finalize_output(p);
 }
 
 // ---------------------------------------------------------------- tokens-on-M variant
@@ -672,6 +716,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
         tc_fence_after();
         tmem_dealloc(tmem_base, C::kTmemCols);
     }
+    if (!GATE_UP && p.final_out != nullptr) finalize_output(p);
 }
 
 // ---------------------------------------------------------------- host side
@@ -783,6 +828,9 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
     p.status = a.status;
     p.gather_tok = a.gate_up ? a.gather_tok : nullptr;
     p.x = reinterpret_cast<const bf16*>(a.act);
+    p.final_out = (!a.gate_up && a.acc_out && a.done) ? a.final_out : nullptr;
+    p.final_rows = a.final_rows;
+    p.done = a.done;
     const long long max_tiles = (static_cast<long long>(ceil_div(a.rows, BN)) + a.E) * p.nf;
     const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
     if (tm) return a.gate_up ? launch_tm<true>(mw, ma, p, grid, s, pdl)

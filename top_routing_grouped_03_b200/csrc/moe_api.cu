@@ -340,6 +340,13 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     dn.acc_out = det ? nullptr : out_acc;
     dn.y_out = det ? at<float>(workspace, L.y_sorted) : nullptr;
     dn.status = status;
+    // without the fixed-order combine, the last down launch also writes the bf16 output
+    unsigned* done = at<unsigned>(workspace, L.status + 64);  // inside the cleared header
+    if (!det && !shared) {
+        dn.final_out = reinterpret_cast<bf16*>(out);
+        dn.final_rows = T;
+        dn.done = done;
+    }
     if (!mark(MOE_EV_DOWN) || launch_grouped_gemm(dn, sms, s, true) != cudaSuccess)
         return MOE_ERR_CUDA;
 
@@ -364,10 +371,16 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
         sd.rows = T; sd.E = 1; sd.D = D; sd.f = fs;
         sd.acc_out = out_acc;
         sd.status = status;
+        if (!det) {
+            sd.final_out = reinterpret_cast<bf16*>(out);
+            sd.final_rows = T;
+            sd.done = done;
+        }
         if (launch_grouped_gemm(sd, sms, s, true) != cudaSuccess) return MOE_ERR_CUDA;
     }
 
-    // bf16 output: out_acc alone, or (fixed order) out_acc's shared part + the routed rows
+    if (!det) return mark(MOE_EV_COMBINE) && mark(MOE_EV_END) ? MOE_OK : MOE_ERR_CUDA;
+    // fixed order: out_acc's shared part (if any) + the routed rows in slot order
     CombineLaunch c{};
     c.out_acc = use_acc ? out_acc : nullptr;
     c.y_sorted = det ? at<float>(workspace, L.y_sorted) : nullptr;

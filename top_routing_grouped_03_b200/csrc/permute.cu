@@ -9,6 +9,7 @@
 //   offsets[e] = sum_{e' < e} counts[e']            (block reduction over <= 512 counts)
 //   a block-wide ballot scan walks the T*K routing entries in order and writes the
 //   entries equal to e to rows offsets[e] + rank  -> ascending token order (stable).
+// permute_small_kernel: the same result from one CTA when T*K <= 4096 (decode sizes).
 // The token rows themselves are never copied: the grouped GEMM gathers them from x.
 #include "common.cuh"
 
@@ -92,10 +93,115 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteLaunch a) 
 
 }
 
+
+// Small problems (T*K <= kSmallEntries): one CTA of 1024 threads does the whole
+// permutation.  offsets = exclusive scan of the counts; then the entries are walked in
+// chunks of 1024 in order, and an entry's row is offsets[e] + (entries of e in earlier
+// chunks) + (entries of e in earlier warps of this chunk) + (its rank among the lanes of
+// its warp holding e, from __match_any_sync) -- ascending token order, as the
+// one-CTA-per-expert kernel gives.
+constexpr int kSmallEntries = 4096;
+constexpr int kSmallThreads = 1024;
+constexpr int kSmallWarps = kSmallThreads / 32;
+
+__global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(PermuteLaunch a) {
+    extern __shared__ int sm[];
+    int* warp_cnt = sm;                          // [kSmallWarps][E]
+    int* base = warp_cnt + kSmallWarps * a.E;    // [E] rows of e placed so far
+    int* off = base + a.E;                       // [E + 1]
+    __shared__ int warp_sums[kSmallWarps];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int E = a.E, total = a.T * a.K;
+
+    grid_dep_wait();
+    grid_dep_launch();
+
+    // offsets: exclusive scan of counts (E <= 512 < kSmallThreads)
+    const int c = tid < E ? a.counts[tid] : 0;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int s = warp_sums[lane];
+        int ws = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, ws, o);
+            if (lane >= o) ws += v;
+        }
+        warp_sums[lane] = ws - s;  // exclusive prefix of the warps
+    }
+    __syncthreads();
+    if (tid < E) {
+        off[tid] = warp_sums[warp] + incl - c;
+        base[tid] = 0;
+        a.offsets[tid] = off[tid];
+    }
+    if (tid == 0) {
+        off[E] = total;
+        a.offsets[E] = total;
+        if (a.dense_offsets) {
+            a.dense_offsets[0] = 0;
+            a.dense_offsets[1] = a.T;
+        }
+    }
+    const unsigned lt = (1u << lane) - 1u;
+    for (int j0 = 0; j0 < total; j0 += kSmallThreads) {
+        for (int i = tid; i < kSmallWarps * E; i += kSmallThreads) warp_cnt[i] = 0;
+        __syncthreads();
+        const int j = j0 + tid;
+        const bool live = j < total;
+        const int e = live ? __ldg(a.topk_idx + j) : -1;
+        const bool ok = live && e >= 0 && e < E;
+        const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
+        const int rank = __popc(peers & lt);
+        if (ok && rank == 0) warp_cnt[warp * E + e] = __popc(peers);
+        if (live && !ok) set_status(a.status, MOE_ERR_DEVICE);
+        __syncthreads();
+        if (tid < E) {  // prefix over the warps of this chunk, per expert
+            int run = base[tid];
+            for (int w = 0; w < kSmallWarps; ++w) {
+                const int v = warp_cnt[w * E + tid];
+                warp_cnt[w * E + tid] = run;
+                run += v;
+            }
+            base[tid] = run;
+        }
+        __syncthreads();
+        if (ok) {
+            const int row = off[e] + warp_cnt[warp * E + e] + rank;
+            if (row < off[e + 1]) {
+                a.sorted_token[row] = j / a.K;
+                if (a.topk_w) a.sorted_w[row] = __ldg(a.topk_w + j);
+                a.slot_to_row[j] = row;
+            } else {
+                set_status(a.status, MOE_ERR_DEVICE);
+            }
+        }
+        __syncthreads();
+    }
+    if (tid < E && base[tid] != off[tid + 1] - off[tid]) set_status(a.status, MOE_ERR_DEVICE);
+}
+
 }  // namespace
 
 cudaError_t launch_permute(const PermuteLaunch& a, cudaStream_t s, bool pdl) {
-    cudaError_t err = launch_kernel(permute_kernel, dim3(a.E), dim3(kPermThreads), 0, s, pdl, a);
+    cudaError_t err;
+    if (static_cast<long long>(a.T) * a.K <= kSmallEntries) {
+        const size_t smem = sizeof(int) * (static_cast<size_t>(kSmallWarps) * a.E + 2 * a.E + 1);
+        err = cudaFuncSetAttribute(permute_small_kernel,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(smem));
+        if (err != cudaSuccess) return err;
+        err = launch_kernel(permute_small_kernel, dim3(1), dim3(kSmallThreads), smem, s, pdl, a);
+    } else {
+        err = launch_kernel(permute_kernel, dim3(a.E), dim3(kPermThreads), 0, s, pdl, a);
+    }
     count_launches(1);
     return err;
 }

@@ -27,17 +27,19 @@ namespace {
 
 constexpr int kTokensPerCta = 8;
 constexpr int kRouterThreads = 256;
-constexpr int kMaxExpertsPerLane = 16;  // E <= 512
+// E <= 512: at most 16 logits per lane in the selection (select_topk_warp)
+constexpr int kExpertsPerWarp = 2;
 
 // TopK of one token's logits by one warp, in registers, then the renormalised weights.
 // lg: the token's E logits (bias already added when add_bias is NULL).  Writes idx/w of
 // the token and adds its K experts to the counts.
-__device__ __forceinline__ void select_topk_warp(const float* lg, const float* add_bias, int E,
-                                                 int K, int token, int lane, int32_t* topk_idx,
-                                                 float* topk_w, int32_t* counts) {
-    float v[kMaxExpertsPerLane];
+template <int NV>
+__device__ __forceinline__ void select_topk_nv(const float* lg, const float* add_bias, int E,
+                                               int K, int token, int lane, int32_t* topk_idx,
+                                               float* topk_w, int32_t* counts) {
+    float v[NV];
 #pragma unroll
-    for (int j = 0; j < kMaxExpertsPerLane; ++j) {
+    for (int j = 0; j < NV; ++j) {
         const int e = j * 32 + lane;
         v[j] = (e < E) ? __ldcg(lg + e) + (add_bias ? __ldg(add_bias + e) : 0.f) : -FLT_MAX;
     }
@@ -47,7 +49,7 @@ __device__ __forceinline__ void select_topk_warp(const float* lg, const float* a
         float bv = -FLT_MAX;
         int bi = 0x7fffffff;
 #pragma unroll
-        for (int j = 0; j < kMaxExpertsPerLane; ++j) {
+        for (int j = 0; j < NV; ++j) {
             const int e = j * 32 + lane;
             if (e < E && v[j] > bv) { bv = v[j]; bi = e; }  // strict: lowest e per lane
         }
@@ -60,7 +62,7 @@ __device__ __forceinline__ void select_topk_warp(const float* lg, const float* a
         if (lane == k) { my_v = bv; my_i = bi; }
         // retire the winner (owner lane only); -inf never wins against finite logits
 #pragma unroll
-        for (int j = 0; j < kMaxExpertsPerLane; ++j)
+        for (int j = 0; j < NV; ++j)
             if (j * 32 + lane == bi) v[j] = -INFINITY;
     }
     const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
@@ -73,6 +75,18 @@ __device__ __forceinline__ void select_topk_warp(const float* lg, const float* a
         topk_w[static_cast<size_t>(token) * K + lane] = ex / sum;
         atomicAdd(&counts[my_i], 1);
     }
+}
+
+// NV = logits per lane = ceil(E / 32), so the selection loops run exactly as far as E needs.
+__device__ __forceinline__ void select_topk_warp(const float* lg, const float* add_bias, int E,
+                                                 int K, int token, int lane, int32_t* topk_idx,
+                                                 float* topk_w, int32_t* counts) {
+    const int nv = (E + 31) / 32;
+    if (nv <= 1) select_topk_nv<1>(lg, add_bias, E, K, token, lane, topk_idx, topk_w, counts);
+    else if (nv <= 2) select_topk_nv<2>(lg, add_bias, E, K, token, lane, topk_idx, topk_w, counts);
+    else if (nv <= 4) select_topk_nv<4>(lg, add_bias, E, K, token, lane, topk_idx, topk_w, counts);
+    else if (nv <= 8) select_topk_nv<8>(lg, add_bias, E, K, token, lane, topk_idx, topk_w, counts);
+    else select_topk_nv<16>(lg, add_bias, E, K, token, lane, topk_idx, topk_w, counts);
 }
 
 __global__ void __launch_bounds__(kRouterThreads)
@@ -106,56 +120,87 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
     }
     __syncthreads();
 
-    // ---- logits of this CTA's expert slab: one warp per expert row; each lane keeps up
-    //      to kUnroll independent 16-byte weight loads in flight
-    constexpr int kUnroll = 8;
+    // ---- logits of this CTA's expert slab: each warp takes kExpertsPerWarp expert rows at
+    //      a time (one unpack of x serves all of them), each lane keeps kUnroll chunks of
+    //      16-byte weight loads per row in flight
+    constexpr int kUnroll = 4;
     const int e_begin = blockIdx.y * experts_per_cta;
     const int e_end = min(e_begin + experts_per_cta, rows_total);
-    for (int e = e_begin + warp; e < e_end; e += kRouterThreads / 32) {
-        const bf16* wrow = (e < E) ? a.w_router + static_cast<size_t>(e) * D : a.w_shared_gate;
-        const uint4* wv = reinterpret_cast<const uint4*>(wrow);
-        float acc[kTokensPerCta];
+    for (int e0 = e_begin + warp * kExpertsPerWarp; e0 < e_end;
+         e0 += (kRouterThreads / 32) * kExpertsPerWarp) {
+        const uint4* wv[kExpertsPerWarp];
+        bool has[kExpertsPerWarp];
 #pragma unroll
-        for (int t = 0; t < kTokensPerCta; ++t) acc[t] = 0.f;
+        for (int u = 0; u < kExpertsPerWarp; ++u) {
+            const int e = e0 + u;
+            has[u] = e < e_end;
+            const bf16* wrow = (e < E) ? a.w_router + static_cast<size_t>(e) * D : a.w_shared_gate;
+            wv[u] = reinterpret_cast<const uint4*>(has[u] ? wrow : a.w_router);
+        }
+        float acc[kExpertsPerWarp][kTokensPerCta];
+#pragma unroll
+        for (int u = 0; u < kExpertsPerWarp; ++u)
+#pragma unroll
+            for (int t = 0; t < kTokensPerCta; ++t) acc[u][t] = 0.f;
         for (int c0 = lane; c0 < vec_per_row; c0 += 32 * kUnroll) {
-            uint4 w[kUnroll];
+            uint4 w[kUnroll][kExpertsPerWarp];
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int c = c0 + 32 * u;
-                w[u] = (c < vec_per_row) ? __ldg(wv + c) : make_uint4(0, 0, 0, 0);
-            }
+            for (int v = 0; v < kUnroll; ++v)
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int c = c0 + 32 * u;
+                for (int u = 0; u < kExpertsPerWarp; ++u) {
+                    const int c = c0 + 32 * v;
+                    w[v][u] = (c < vec_per_row && has[u]) ? __ldg(wv[u] + c) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+            for (int v = 0; v < kUnroll; ++v) {
+                const int c = c0 + 32 * v;
                 if (c >= vec_per_row) break;
-                const float w0 = bf16_lo(w[u].x), w1 = bf16_hi(w[u].x), w2 = bf16_lo(w[u].y);
-                const float w3 = bf16_hi(w[u].y), w4 = bf16_lo(w[u].z), w5 = bf16_hi(w[u].z);
-                const float w6 = bf16_lo(w[u].w), w7 = bf16_hi(w[u].w);
+                float wf[kExpertsPerWarp][8];
+#pragma unroll
+                for (int u = 0; u < kExpertsPerWarp; ++u) {
+                    wf[u][0] = bf16_lo(w[v][u].x); wf[u][1] = bf16_hi(w[v][u].x);
+                    wf[u][2] = bf16_lo(w[v][u].y); wf[u][3] = bf16_hi(w[v][u].y);
+                    wf[u][4] = bf16_lo(w[v][u].z); wf[u][5] = bf16_hi(w[v][u].z);
+                    wf[u][6] = bf16_lo(w[v][u].w); wf[u][7] = bf16_hi(w[v][u].w);
+                }
 #pragma unroll
                 for (int t = 0; t < kTokensPerCta; ++t) {
                     const uint4 xv = xs[t * vec_per_row + c];
-                    float s = acc[t];
-                    s = fmaf(w0, bf16_lo(xv.x), s);
-                    s = fmaf(w1, bf16_hi(xv.x), s);
-                    s = fmaf(w2, bf16_lo(xv.y), s);
-                    s = fmaf(w3, bf16_hi(xv.y), s);
-                    s = fmaf(w4, bf16_lo(xv.z), s);
-                    s = fmaf(w5, bf16_hi(xv.z), s);
-                    s = fmaf(w6, bf16_lo(xv.w), s);
-                    s = fmaf(w7, bf16_hi(xv.w), s);
-                    acc[t] = s;
+                    const float x0 = bf16_lo(xv.x), x1 = bf16_hi(xv.x), x2 = bf16_lo(xv.y);
+                    const float x3 = bf16_hi(xv.y), x4 = bf16_lo(xv.z), x5 = bf16_hi(xv.z);
+                    const float x6 = bf16_lo(xv.w), x7 = bf16_hi(xv.w);
+#pragma unroll
+                    for (int u = 0; u < kExpertsPerWarp; ++u) {
+                        float s2 = acc[u][t];
+                        s2 = fmaf(wf[u][0], x0, s2);
+                        s2 = fmaf(wf[u][1], x1, s2);
+                        s2 = fmaf(wf[u][2], x2, s2);
+                        s2 = fmaf(wf[u][3], x3, s2);
+                        s2 = fmaf(wf[u][4], x4, s2);
+                        s2 = fmaf(wf[u][5], x5, s2);
+                        s2 = fmaf(wf[u][6], x6, s2);
+                        s2 = fmaf(wf[u][7], x7, s2);
+                        acc[u][t] = s2;
+                    }
                 }
             }
         }
 #pragma unroll
-        for (int t = 0; t < kTokensPerCta; ++t) {
+        for (int u = 0; u < kExpertsPerWarp; ++u)
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
-        }
+            for (int t = 0; t < kTokensPerCta; ++t)
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+                    acc[u][t] += __shfl_xor_sync(0xffffffffu, acc[u][t], off);
         if (lane == 0) {
-            const float b = (e < E && a.logit_bias) ? a.logit_bias[e] : 0.f;
-            for (int t = 0; t < nt; ++t)
-                a.logits[static_cast<size_t>(t0 + t) * (E + 1) + e] = acc[t] + b;
+#pragma unroll
+            for (int u = 0; u < kExpertsPerWarp; ++u) {
+                const int e = e0 + u;
+                if (!has[u]) continue;
+                const float b = (e < E && a.logit_bias) ? a.logit_bias[e] : 0.f;
+                for (int t = 0; t < nt; ++t)
+                    a.logits[static_cast<size_t>(t0 + t) * (E + 1) + e] = acc[u][t] + b;
+            }
         }
     }
     __threadfence();  // this thread's logits are visible device-wide before the ticket
@@ -228,11 +273,11 @@ cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bo
     if (a.T == 0) return cudaSuccess;
     const int n_tb = ceil_div(a.T, kTokensPerCta);
     const int rows_total = a.E + (a.w_shared_gate ? 1 : 0);
-    const int warps = kRouterThreads / 32;
-    // split the experts so that the grid covers about two waves of the GPU
-    int n_eb = ceil_div(2 * num_sms, n_tb);
-    n_eb = max(1, min(n_eb, ceil_div(rows_total, warps)));
-    int per_cta = ceil_div(ceil_div(rows_total, n_eb), warps) * warps;
+    const int rows_per_pass = (kRouterThreads / 32) * kExpertsPerWarp;
+    // split the experts so that the grid covers about one wave of the GPU
+    int n_eb = ceil_div(num_sms, n_tb);
+    n_eb = max(1, min(n_eb, ceil_div(rows_total, rows_per_pass)));
+    int per_cta = ceil_div(ceil_div(rows_total, n_eb), rows_per_pass) * rows_per_pass;
     n_eb = ceil_div(rows_total, per_cta);
     const size_t smem = static_cast<size_t>(kTokensPerCta) * a.D * sizeof(bf16);
     cudaError_t err = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
