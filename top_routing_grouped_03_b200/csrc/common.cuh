@@ -124,13 +124,18 @@ struct GroupedGemmLaunch {
     // the expert-ordered problem is x[gather_tok[r]] (gathered inside the kernel)
     const int32_t* gather_tok;
     int block_rows;   // rows per tile (16/32/64/128); 0 picks from the average group size
-    int orientation;  // 0: auto; 1: weights on the MMA's M side; 2: tokens on M
+    int orientation;  // 0: auto; 1: weights on M; 2: tokens on M (one CTA); 3: CTA pairs
     // down with acc_out: when final_out and done are set, the kernel converts acc_out
     // [final_rows, D] to bf16 in final_out after all its CTAs finished (done = 0 at launch)
     bf16* final_out;
     int final_rows;
     unsigned* done;
+    // gate_up with gather_tok: room for the rows in expert order [rows, D]; when given, the
+    // CTA-pair kernel may be used (rows gathered by a copy kernel first)
+    bf16* gather_buf;
 };
+cudaError_t launch_gather_rows(const bf16* x, const int32_t* tok, int rows, int D, bf16* out,
+                               int num_sms, cudaStream_t s, bool pdl);
 cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s,
                                 bool pdl = false);
 

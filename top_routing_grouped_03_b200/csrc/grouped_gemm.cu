@@ -26,6 +26,7 @@
 // group offsets, so no host synchronisation is needed.  Every wait is bounded.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -126,6 +127,7 @@ __device__ __noinline__ void finalize_output(const Params& p) {
 // Named barrier 1 of the four epilogue warps with an AND across their threads: all of
 // them take the same branch afterwards, so a wait that gives up in one warp makes every
 // epilogue warp unwind together.
+template <int kThreadsInBar = kEpiThreads>
 __device__ __forceinline__ bool epilogue_bar_and(bool v) {
     uint32_t r;
     asm volatile(
@@ -134,7 +136,7 @@ __device__ __forceinline__ bool epilogue_bar_and(bool v) {
         "bar.red.and.pred p, 1, %2, q;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(r)
-        : "r"(static_cast<uint32_t>(v)), "n"(kEpiThreads)
+        : "r"(static_cast<uint32_t>(v)), "n"(kThreadsInBar)
         : "memory");
     return r != 0;
 }
@@ -168,7 +170,7 @@ __device__ __forceinline__ Tile decode_tile(int tile, const int* g_tile, const i
 __device__ __forceinline__ void build_tile_table(const Params& p, int rows_per_tile, int* g_off,
                                                  int* g_tile, int* total_slot, int warp,
                                                  int lane) {
-    for (int i = threadIdx.x; i <= p.G; i += kThreads)
+    for (int i = threadIdx.x; i <= p.G; i += blockDim.x)
         g_off[i] = p.offsets ? p.offsets[i] : (i == 0 ? 0 : p.rows_total);
     __syncthreads();
     if (warp == 2) {
@@ -461,6 +463,78 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
 // vectors (red.global.add.v4.f32) into the token's output row.
 constexpr int kTmRows = 128;  // token rows per tile (MMA M)
 constexpr int kTmN = 256;     // weight rows per tile (MMA N)
+// 2 warps (producer, MMA) + 8 epilogue warps: two warps per tensor-memory lane quarter,
+// each draining half of the accumulator's columns
+constexpr int kTmThreads = 64 + 256;
+constexpr int kTmEpiThreads = 256;
+
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+                 "f"(c), "f"(d)
+                 : "memory");
+}
+
+// Epilogue of one tokens-on-M tile for one epilogue warp: `half` selects the columns this
+// warp drains (gate_up: features [64 half, 64 half + 64) of the tile's 128; down: output
+// columns [128 half, 128 half + 128) of its 256).  The warp's 32 lanes are 32 rows.
+template <bool GATE_UP>
+__device__ __forceinline__ void tm_epilogue(const Params& p, uint32_t tbase, int row, bool valid,
+                                            int tile_i, int half) {
+    if (GATE_UP) {
+        bf16* hrow = p.h_out + static_cast<size_t>(row) * p.out_cols + tile_i * kBM + half * 64;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+            uint32_t gv[32], uv[32];
+            tmem_ld32(tbase + half * 64 + c0, gv);
+            tmem_ld32(tbase + kBM + half * 64 + c0, uv);
+            tmem_ld_wait();
+            if (valid) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float g0 = __uint_as_float(gv[2 * j]);
+                    const float g1 = __uint_as_float(gv[2 * j + 1]);
+                    const float h0 = __fdividef(g0, 1.f + __expf(-g0)) * __uint_as_float(uv[2 * j]);
+                    const float h1 = __fdividef(g1, 1.f + __expf(-g1)) * __uint_as_float(uv[2 * j + 1]);
+                    pk[j] = pack_bf16x2(h0, h1);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(hrow + c0);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            }
+        }
+    } else {
+        const float w = (valid && p.sorted_w) ? __ldg(p.sorted_w + row) : 1.f;
+        const int tok = valid ? (p.sorted_token ? __ldg(p.sorted_token + row) : row) : 0;
+        const int col0 = tile_i * kTmN + half * 128;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(tbase + half * 128 + c0, v);
+            tmem_ld_wait();
+            if (valid) {
+                if (p.acc_out) {
+                    float* dst = p.acc_out + static_cast<size_t>(tok) * p.out_cols + col0 + c0;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        red_add_v4(dst + j, w * __uint_as_float(v[j]), w * __uint_as_float(v[j + 1]),
+                                   w * __uint_as_float(v[j + 2]), w * __uint_as_float(v[j + 3]));
+                }
+                if (p.y_out) {
+                    float4* dst = reinterpret_cast<float4*>(
+                        p.y_out + static_cast<size_t>(row) * p.out_cols + col0 + c0);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        dst[j] = make_float4(w * __uint_as_float(v[4 * j]), w * __uint_as_float(v[4 * j + 1]),
+                                             w * __uint_as_float(v[4 * j + 2]),
+                                             w * __uint_as_float(v[4 * j + 3]));
+                }
+            }
+        }
+    }
+}
 
 template <bool GATE_UP>
 struct CfgTm {
@@ -473,14 +547,9 @@ struct CfgTm {
     static_assert(kTmemCols <= 512, "accumulators exceed tensor memory");
 };
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-                 "f"(c), "f"(d)
-                 : "memory");
-}
 
 template <bool GATE_UP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kTmThreads, 1)
 grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
                        const __grid_constant__ CUtensorMap map_act, Params p) {
     using C = CfgTm<GATE_UP>;
@@ -509,7 +578,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], kEpiThreads);
+            mbar_init(&tempty[b], kTmEpiThreads);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -638,7 +707,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             const Tile t = decode_tile(tile, g_tile, g_off, p.G, kTmRows);
             const bool ready = mbar_wait(&tfull[abuf], aphase, kWaitBudgetNs, abort_flag);
-            if (!epilogue_bar_and(ready)) {
+            if (!epilogue_bar_and<kTmEpiThreads>(ready)) {
                 set_status(p.status, MOE_ERR_TIMEOUT);
                 *abort_flag = 1;
                 break;
@@ -647,62 +716,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    abuf * C::kAccCols;
             const int row = t.row0 + q * 32 + lane;
-            const bool valid = row < t.row_end;
-            if (GATE_UP) {
-                bf16* hrow = p.h_out + static_cast<size_t>(row) * p.out_cols + t.i * kBM;
-#pragma unroll 1
-                for (int c0 = 0; c0 < kBM; c0 += 16) {
-                    uint32_t gv[16], uv[16];
-                    tmem_ld16(tbase + c0, gv);
-                    tmem_ld16(tbase + kBM + c0, uv);
-                    tmem_ld_wait();
-                    if (valid) {
-                        uint32_t pk[8];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const float g0 = __uint_as_float(gv[2 * j]);
-                            const float g1 = __uint_as_float(gv[2 * j + 1]);
-                            const float h0 = g0 / (1.f + __expf(-g0)) * __uint_as_float(uv[2 * j]);
-                            const float h1 = g1 / (1.f + __expf(-g1)) * __uint_as_float(uv[2 * j + 1]);
-                            pk[j] = pack_bf16x2(h0, h1);
-                        }
-                        uint4* dst = reinterpret_cast<uint4*>(hrow + c0);
-                        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                    }
-                }
-            } else {
-                const float w = (valid && p.sorted_w) ? __ldg(p.sorted_w + row) : 1.f;
-                const int tok = valid ? (p.sorted_token ? __ldg(p.sorted_token + row) : row) : 0;
-                const int col0 = t.i * kTmN;
-#pragma unroll 1
-                for (int c0 = 0; c0 < kTmN; c0 += 16) {
-                    uint32_t v[16];
-                    tmem_ld16(tbase + c0, v);
-                    tmem_ld_wait();
-                    if (valid) {
-                        if (p.acc_out) {
-                            float* dst = p.acc_out + static_cast<size_t>(tok) * p.out_cols + col0 + c0;
-#pragma unroll
-                            for (int j = 0; j < 16; j += 4)
-                                red_add_v4(dst + j, w * __uint_as_float(v[j]),
-                                           w * __uint_as_float(v[j + 1]),
-                                           w * __uint_as_float(v[j + 2]),
-                                           w * __uint_as_float(v[j + 3]));
-                        }
-                        if (p.y_out) {
-                            float4* dst = reinterpret_cast<float4*>(
-                                p.y_out + static_cast<size_t>(row) * p.out_cols + col0 + c0);
-#pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                dst[j] = make_float4(w * __uint_as_float(v[4 * j]),
-                                                     w * __uint_as_float(v[4 * j + 1]),
-                                                     w * __uint_as_float(v[4 * j + 2]),
-                                                     w * __uint_as_float(v[4 * j + 3]));
-                        }
-                    }
-                }
-            }
+            tm_epilogue<GATE_UP>(p, tbase, row, row < t.row_end, t.i, (warp - 2) >> 2);
             tc_fence_before();
             mbar_arrive(&tempty[abuf]);
             abuf ^= 1u;
@@ -715,6 +729,202 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+    if (!GATE_UP && p.final_out != nullptr) finalize_output(p);
+}
+
+// ---------------------------------------------------------------- CTA-pair variant
+// For groups with many rows, two CTAs of a cluster share one tcgen05.mma of 256 x 256 x 16
+// (cta_group::2): CTA r holds token rows [128 r, 128 r + 128) of a 256-row block (its half
+// of A) and weight rows [128 r, 128 r + 128) of the 256-row block (its half of B) -- for
+// gate_up the leader's half is the 128 gate rows and the peer's the 128 up rows of the same
+// features -- and receives its 128 rows x 256 columns of D in its own tensor memory.  Each
+// CTA loads 32 KB per K step instead of 48 KB, and 6 stages fit.  Both CTAs' TMA loads are
+// counted on the leader's full barrier; the leader's single MMA thread commits to the
+// empty and accumulator-full barriers of both CTAs; the peer's epilogue warps arrive on the
+// leader's accumulator-empty barrier.  A's rows must be contiguous (x gathered into expert
+// order beforehand for gate_up).
+struct CfgPair {
+    static constexpr int kABytes = kTmRows * kBK * 2;  // this CTA's 128 token rows: 16 KB
+    static constexpr int kBBytes = kBM * kBK * 2;      // this CTA's 128 weight rows: 16 KB
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = 6;
+    static constexpr int kAccCols = kTmN;
+    static constexpr int kTmemCols = 2 * kAccCols;
+    static constexpr int kPairRows = 2 * kTmRows;  // token rows per pair tile
+};
+
+template <bool GATE_UP>
+__global__ void __launch_bounds__(kTmThreads, 1)
+grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_w,
+                         const __grid_constant__ CUtensorMap map_act, Params p) {
+    using C = CfgPair;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+    uint64_t* empty = full + C::kStages;
+    uint64_t* tfull = empty + C::kStages;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* total_slot = reinterpret_cast<int*>(tmem_slot + 2);
+    int* g_off = reinterpret_cast<int*>(tmem_slot + 4);
+    int* g_tile = g_off + (p.G + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();  // 0: leader (issues the MMAs), 1: peer
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);   // leader: one expect-tx arrival; both CTAs' bytes
+            mbar_init(&empty[s], 1);  // both: the leader's multicast commit
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);    // both: the leader's multicast commit
+            mbar_init(&tempty[b], 16);  // leader: the 8 epilogue warps of each CTA
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&map_w);
+        tma_prefetch_desc(&map_act);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, C::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    grid_dep_wait();
+    grid_dep_launch();
+    build_tile_table(p, C::kPairRows, g_off, g_tile, total_slot, warp, lane);
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // both CTAs' barriers and tensor memory exist before any pair operation
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = *total_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer (both)
+        if (lane == 0) {
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_a = policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0, filled = 0, fill_phase = 0;
+            bool ok = true;
+            for (int tile = pair; tile < total && ok; tile += npairs) {
+                const Tile t = decode_tile(tile, g_tile, g_off, p.G, C::kPairRows);
+                const int arow = t.row0 + static_cast<int>(rank) * kTmRows;
+                // gate_up: leader = gate rows, peer = up rows of features i*128..+127;
+                // down: rows i*256 + 128*rank
+                const int wrow = GATE_UP ? t.g * p.w_group_rows + t.i * kBM + (rank ? p.up_rows : 0)
+                                         : t.g * p.w_group_rows + t.i * kTmN + rank * kBM;
+                for (int kk = 0; kk < p.nk; ++kk) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, kWaitBudgetNs, abort_flag)) {
+                        set_status(p.status, MOE_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* st = smem + stage * C::kStageBytes;
+                    const uint32_t leader_full = map_to_rank(smem_u32(&full[stage]), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
+                    tma_load_2d_pair(st, &map_act, leader_full, kk * kBK, arow, pol_a);
+                    tma_load_2d_pair(st + C::kABytes, &map_w, leader_full, kk * kBK, wrow, pol_w);
+                    filled |= 1u << stage;
+                    fill_phase = (fill_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok && rank == 0) {
+                for (int s = 0; s < C::kStages; ++s)
+                    if (filled & (1u << s))
+                        mbar_wait(&full[s], (fill_phase >> s) & 1u, kDrainBudgetNs, nullptr);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA (leader)
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(2 * kTmRows, kTmN);
+            int stage = 0;
+            uint32_t phase = 0, abuf = 0, aphase = 0;
+            bool ok = true, issued = false;
+            for (int tile = pair; tile < total && ok; tile += npairs) {
+                if (!mbar_wait(&tempty[abuf], aphase ^ 1u, kWaitBudgetNs, abort_flag)) {
+                    set_status(p.status, MOE_ERR_TIMEOUT);
+                    *abort_flag = 1;
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + abuf * C::kAccCols;
+                for (int kk = 0; kk < p.nk; ++kk) {
+                    if (!mbar_wait(&full[stage], phase, kWaitBudgetNs, abort_flag)) {
+                        set_status(p.status, MOE_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
+                    const uint32_t b0 = a0 + C::kABytes;
+#pragma unroll
+                    for (int s = 0; s < kBK / 16; ++s)
+                        umma_bf16_pair(d0, sdesc_k_sw128(a0 + s * 32), sdesc_k_sw128(b0 + s * 32),
+                                       idesc, (kk | s) != 0 ? 1u : 0u);
+                    issued = true;
+                    umma_commit_pair(&empty[stage]);
+                    if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                umma_commit_pair(&tfull[abuf]);
+                abuf ^= 1u;
+                if (abuf == 0) aphase ^= 1u;
+            }
+            if (!ok && issued) {
+                umma_commit_pair(drain);
+                mbar_wait(drain, 0, kDrainBudgetNs, nullptr);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- epilogue (both)
+        const int q = warp & 3;
+        const uint32_t leader_tempty0 = map_to_rank(smem_u32(&tempty[0]), 0);
+        uint32_t abuf = 0, aphase = 0;
+        for (int tile = pair; tile < total; tile += npairs) {
+            const Tile t = decode_tile(tile, g_tile, g_off, p.G, C::kPairRows);
+            const bool ready = mbar_wait(&tfull[abuf], aphase, kWaitBudgetNs, abort_flag);
+            if (!epilogue_bar_and<kTmEpiThreads>(ready)) {
+                set_status(p.status, MOE_ERR_TIMEOUT);
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   abuf * C::kAccCols;
+            const int row = t.row0 + static_cast<int>(rank) * kTmRows + q * 32 + lane;
+            tm_epilogue<GATE_UP>(p, tbase, row, row < t.row_end, t.i, (warp - 2) >> 2);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_tempty0 + abuf * 8);
+            abuf ^= 1u;
+            if (abuf == 0) aphase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // the pair's MMAs and remote arrivals are over before tensor memory goes
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::kTmemCols);
     }
     if (!GATE_UP && p.final_out != nullptr) finalize_output(p);
 }
@@ -774,7 +984,36 @@ cudaError_t launch_tm(const CUtensorMap& mw, const CUtensorMap& ma, const Params
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    err = launch_kernel(kfn, dim3(grid), dim3(kThreads), smem, s, pdl, mw, ma, p);
+    err = launch_kernel(kfn, dim3(grid), dim3(kTmThreads), smem, s, pdl, mw, ma, p);
+    count_launches(1);
+    return err;
+}
+
+template <bool GATE_UP>
+cudaError_t launch_pair(const CUtensorMap& mw, const CUtensorMap& ma, const Params& p,
+                        int npairs, cudaStream_t s, bool pdl) {
+    using C = CfgPair;
+    const size_t smem = 1024 + static_cast<size_t>(C::kStages) * C::kStageBytes +
+                        (2 * C::kStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int);
+    auto kfn = grouped_gemm_pair_kernel<GATE_UP>;
+    cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * npairs);
+    cfg.blockDim = dim3(kTmThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
+    err = cudaLaunchKernelEx(&cfg, kfn, mw, ma, p);
     count_launches(1);
     return err;
 }
@@ -798,8 +1037,13 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
     // orientation: tokens on the MMA's M side once the groups average a full 128-row tile
     // (and the output width splits into 256-wide blocks for down); weights on M otherwise
     const bool tm_ok = a.gate_up ? (a.f % 128 == 0) : (a.D % 256 == 0);
-    const bool tm = tm_ok && (a.orientation == 2 ||
+    const bool tm = tm_ok && (a.orientation >= 2 ||
                               (a.orientation == 0 && a.block_rows == 0 && a.rows / a.E >= 128));
+    // tokens on M: CTA pairs when A's rows are contiguous (always for down; for gate_up once
+    // x is gathered into expert order), unless a single CTA is asked for
+    const bool gathered = a.gate_up && a.gather_tok != nullptr;
+    const bool pairs = tm && a.orientation != 2 && (!gathered || a.gather_buf != nullptr) &&
+                       num_sms >= 2;
     const int BN = tm ? kTmRows : (a.block_rows ? a.block_rows : pick_block_rows(a.rows, a.E));
     if (BN != 16 && BN != 32 && BN != 64 && BN != 128) return cudaErrorInvalidValue;
     const int K = a.gate_up ? a.D : a.f;
@@ -808,8 +1052,16 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
     if ((err = make_map(&mw, a.w, w_group_rows * a.E, K, kBM)) != cudaSuccess) return err;  // 128-row boxes
     // the activation map is only read when the rows are contiguous (no gather); with a
     // gather it still has to be a valid descriptor, so it covers the first row of x
-    const bool gather = a.gate_up && a.gather_tok != nullptr;
-    if ((err = make_map(&ma, a.act, gather ? 1 : a.rows, K, gather ? 1 : BN)) != cudaSuccess)
+    const void* act = a.act;
+    bool gather = gathered;
+    if (pairs && gathered) {
+        err = launch_gather_rows(reinterpret_cast<const bf16*>(a.act), a.gather_tok, a.rows, a.D,
+                                 a.gather_buf, num_sms, s, pdl);
+        if (err != cudaSuccess) return err;
+        act = a.gather_buf;
+        gather = false;
+    }
+    if ((err = make_map(&ma, act, gather ? 1 : a.rows, K, gather ? 1 : BN)) != cudaSuccess)
         return err;
     Params p{};
     p.offsets = a.offsets;
@@ -826,13 +1078,20 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
     p.acc_out = a.acc_out;
     p.y_out = a.y_out;
     p.status = a.status;
-    p.gather_tok = a.gate_up ? a.gather_tok : nullptr;
-    p.x = reinterpret_cast<const bf16*>(a.act);
+    p.gather_tok = gather ? a.gather_tok : nullptr;
+    p.x = reinterpret_cast<const bf16*>(act);
     p.final_out = (!a.gate_up && a.acc_out && a.done) ? a.final_out : nullptr;
     p.final_rows = a.final_rows;
     p.done = a.done;
     const long long max_tiles = (static_cast<long long>(ceil_div(a.rows, BN)) + a.E) * p.nf;
     const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
+    if (pairs) {
+        const long long pair_tiles =
+            (static_cast<long long>(ceil_div(a.rows, CfgPair::kPairRows)) + a.E) * p.nf;
+        const int npairs = static_cast<int>(std::min<long long>(pair_tiles, num_sms / 2));
+        return a.gate_up ? launch_pair<true>(mw, ma, p, npairs, s, true)
+                         : launch_pair<false>(mw, ma, p, npairs, s, true);
+    }
     if (tm) return a.gate_up ? launch_tm<true>(mw, ma, p, grid, s, pdl)
                              : launch_tm<false>(mw, ma, p, grid, s, pdl);
     switch (BN) {

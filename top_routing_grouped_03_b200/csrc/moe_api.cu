@@ -36,7 +36,7 @@ int num_sms_current() {
 // Workspace of the whole layer.  The status word is always at offset 0.
 struct Layout {
     size_t status, counters, counts, logits, offsets, dense_offsets, topk_idx, topk_w, sgate,
-        sorted_token, sorted_w, slot_to_row, h, h_s, out_acc, y_sorted, total;
+        sorted_token, sorted_w, slot_to_row, x_sorted, h, h_s, out_acc, y_sorted, total;
     size_t zero_end;  // [0, zero_end) is cleared at the start of a layer call
 };
 
@@ -61,6 +61,7 @@ Layout layout(long long T, long long D, long long E, long long K, long long f, l
     L.sorted_token = take(sizeof(int32_t) * T * K);
     L.sorted_w = take(sizeof(float) * T * K);
     L.slot_to_row = take(sizeof(int32_t) * T * K);
+    L.x_sorted = take(2 * T * K * D);
     L.h = take(2 * T * K * f);
     L.h_s = take(2 * T * fs);
     L.out_acc = take(sizeof(float) * T * D);
@@ -322,6 +323,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     up.w = p->w_gate_up;
     up.act = p->x;
     up.gather_tok = pm.sorted_token;
+    up.gather_buf = at<bf16>(workspace, L.x_sorted);
     up.offsets = pm.offsets;
     up.rows = rows; up.E = E; up.D = D; up.f = f;
     up.h_out = at<bf16>(workspace, L.h);

@@ -11,6 +11,8 @@
 //   entries equal to e to rows offsets[e] + rank  -> ascending token order (stable).
 // permute_small_kernel: the same result from one CTA when T*K <= 4096 (decode sizes).
 // The token rows themselves are never copied: the grouped GEMM gathers them from x.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace moe {
@@ -188,6 +190,24 @@ __global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(PermuteLau
     if (tid < E && base[tid] != off[tid + 1] - off[tid]) set_status(a.status, MOE_ERR_DEVICE);
 }
 
+
+// x_sorted[r] = x[sorted_token[r]]: the token rows in expert order, 16-byte vectors,
+// grid-stride (for the CTA-pair GEMM, whose operand rows must be contiguous).
+__global__ void __launch_bounds__(256) gather_rows_kernel(const bf16* x, const int32_t* tok,
+                                                          int rows, int D, bf16* out) {
+    grid_dep_wait();
+    grid_dep_launch();
+    const int vec = D / 8;
+    const long long n = static_cast<long long>(rows) * vec;
+    const uint4* src = reinterpret_cast<const uint4*>(x);
+    uint4* dst = reinterpret_cast<uint4*>(out);
+    for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n; i += 256ll * gridDim.x) {
+        const int r = static_cast<int>(i / vec);
+        const int c = static_cast<int>(i - static_cast<long long>(r) * vec);
+        dst[i] = __ldg(src + static_cast<size_t>(__ldg(tok + r)) * vec + c);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_permute(const PermuteLaunch& a, cudaStream_t s, bool pdl) {
@@ -202,6 +222,17 @@ cudaError_t launch_permute(const PermuteLaunch& a, cudaStream_t s, bool pdl) {
     } else {
         err = launch_kernel(permute_kernel, dim3(a.E), dim3(kPermThreads), 0, s, pdl, a);
     }
+    count_launches(1);
+    return err;
+}
+
+cudaError_t launch_gather_rows(const bf16* x, const int32_t* tok, int rows, int D, bf16* out,
+                               int num_sms, cudaStream_t s, bool pdl) {
+    if (rows == 0) return cudaSuccess;
+    const long long n = static_cast<long long>(rows) * (D / 8);
+    const int blocks = static_cast<int>(std::min<long long>((n + 255) / 256, 8ll * num_sms));
+    cudaError_t err = launch_kernel(gather_rows_kernel, dim3(blocks), dim3(256), 0, s, pdl, x, tok,
+                                    rows, D, out);
     count_launches(1);
     return err;
 }
