@@ -45,6 +45,8 @@ def _load():
         P = ctypes.c_void_p
         I = ctypes.c_int
         lib.oracle_route.argtypes = [P, P, P, P, I, I, I, I, P, P, P, P, P]
+        lib.oracle_route_ex.argtypes = [P, P, P, P, I, I, I, I, I, P, I, P, P, P, P, P]
+        lib.oracle_route_ex.restype = ctypes.c_int
         lib.oracle_experts.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P, I, P]
         lib.oracle_dense_masked.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P]
         lib.oracle_permute.argtypes = [P, I, I, I, P, P, P, P, P]
@@ -75,23 +77,32 @@ def _ptr(a: Optional[np.ndarray]):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
 
-def route(x, w_router, K: int, logit_bias=None, w_shared_gate=None):
-    """Router: returns dict(idx [T,K] int32, alpha [T,K] f64, probs [T,E] f64,
-    gap [T] f64, shared_gate [T] f64 or None)."""
+def _f64_vec(v):
+    if v is None:
+        return None
+    return np.ascontiguousarray(np.asarray(v.cpu() if hasattr(v, "cpu") else v, dtype=np.float64))
+
+
+def route(x, w_router, K: int, logit_bias=None, w_shared_gate=None, score: str = "softmax",
+          select_bias=None, bf16_weights: bool = False):
+    """Router: returns dict(idx [T,K] int32, alpha [T,K] f64, probs [T,E] f64 (the scores:
+    softmax probabilities or sigmoid affinities), gap [T] f64 (of the selection keys),
+    shared_gate [T] f64 or None)."""
     xb, wb = bits(x), bits(w_router)
     T, D = xb.shape
     E = wb.shape[0]
-    bias = None if logit_bias is None else np.ascontiguousarray(
-        np.asarray(logit_bias.cpu() if hasattr(logit_bias, "cpu") else logit_bias,
-                   dtype=np.float64))
+    bias = _f64_vec(logit_bias)
+    sbias = _f64_vec(select_bias)
+    mode = {"softmax": 0, "sigmoid": 1}[score]
     sg = None if w_shared_gate is None else bits(w_shared_gate)
     idx = np.zeros((T, K), np.int32)
     alpha = np.zeros((T, K), np.float64)
     probs = np.zeros((T, E), np.float64)
     gap = np.zeros((T,), np.float64)
     sgate = np.zeros((T,), np.float64) if sg is not None else None
-    rc = _load().oracle_route(_ptr(xb), _ptr(wb), _ptr(bias), _ptr(sg), T, D, E, K,
-                              _ptr(idx), _ptr(alpha), _ptr(probs), _ptr(gap), _ptr(sgate))
+    rc = _load().oracle_route_ex(_ptr(xb), _ptr(wb), _ptr(bias), _ptr(sg), T, D, E, K, mode,
+                                 _ptr(sbias), int(bool(bf16_weights)), _ptr(idx), _ptr(alpha),
+                                 _ptr(probs), _ptr(gap), _ptr(sgate))
     if rc != 0:
         raise ValueError(f"oracle_route failed ({rc})")
     return dict(idx=idx, alpha=alpha, probs=probs, gap=gap, shared_gate=sgate)
@@ -161,10 +172,16 @@ def permute(idx, E: int):
                 sorted_slot=sorted_slot, slot_to_row=slot_to_row)
 
 
-def layer(inp, tokens=None):
+def layer(inp, tokens=None, score: str = "softmax", select_bias=None, bf16_weights=False,
+          residual=None):
     """Whole layer for a ``workloads.LayerInputs``: route every token, then the sparse
-    expert sum for ``tokens`` (all when None).  Returns (route dict, y [ntok, D])."""
-    r = route(inp.x, inp.w_router, inp.cfg.K, inp.logit_bias, inp.w_shared_gate)
+    expert sum for ``tokens`` (all when None), plus the residual h (bf16 [T, D]) when given
+    ("MoE", section 4: h_out = h + y).  Returns (route dict, y [ntok, D])."""
+    r = route(inp.x, inp.w_router, inp.cfg.K, inp.logit_bias, inp.w_shared_gate, score,
+              select_bias, bf16_weights)
     y = experts(inp.x, r["idx"], r["alpha"], inp.w_gate_up, inp.w_down, tokens,
                 inp.w_shared_gate_up, inp.w_shared_down, r["shared_gate"])
+    if residual is not None:
+        h = bf16_to_f64(residual)
+        y = y + (h if tokens is None else h[np.asarray(tokens)])
     return r, y

@@ -50,61 +50,96 @@ static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
 
 static double silu(double z) { return z * sigmoid(z); }
 
+/* bf16 rounding of a routing weight the way the reference casts it back to the model
+ * dtype: the fp32 weight rounded to the nearest bf16, ties to even ("MoE", section 2:
+ * the renormalised fp32 scores are converted to the model's bf16). */
+static double round_to_bf16(double v) {
+    float f = (float)v;
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    u = (u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
 /*
- * Router ("MoE", section 2).  For each token t:
+ * Router ("MoE", section 2; "1.6 混合专家（MoE）", section 2 top-k gating and section 3
+ * bias method).  For each token t:
  *   r_t[e]  = x_t . W_r[e]  (+ bias[e])
- *   p_t     = softmax(r_t)                       (max-subtracted, double)
- *   I_t     = the K largest p_t[e]; ties -> lower e; listed by descending p
- *   alpha   = p_t[I_t] / sum p_t[I_t]
- *   gap[t]  = p_(K) - p_(K+1)  (K-th minus (K+1)-th largest probability; +inf if K == E)
- *   sgate[t]= sigma(w_s . x_t)                   (shared-expert scalar gate, section 4)
- * Outputs idx [T*K], alpha [T*K]; probs [T*E], gap [T], sgate [T] are optional (NULL).
- * Returns 0, or -1 on bad arguments.
+ *   p_t     = softmax(r_t)          score_mode 0 (max-subtracted, double), or
+ *   p_t[e]  = sigma(r_t[e])         score_mode 1 (per-expert sigmoid affinity)
+ *   key[e]  = p_t[e] + select_bias[e]   (selection-only bias; 0 when NULL)
+ *   I_t     = the K largest keys; ties -> lower e; listed by descending key
+ *   alpha   = p_t[I_t] / sum p_t[I_t]   (the raw scores, never the bias)
+ *             rounded to bf16 when bf16_weights != 0
+ *   gap[t]  = key_(K) - key_(K+1)  (+inf if K == E)
+ *   sgate[t]= sigma(w_s . x_t)      (shared-expert scalar gate, "MoE" section 4)
+ * Outputs idx [T*K], alpha [T*K]; probs [T*E] (the scores p), gap [T], sgate [T] are
+ * optional (NULL).  Returns 0, or -1 on bad arguments.
  */
-int oracle_route(const uint16_t* x, const uint16_t* w_r, const double* bias,
-                 const uint16_t* w_sg, int T, int D, int E, int K,
-                 int32_t* idx, double* alpha, double* probs, double* gap, double* sgate) {
-    if (T < 0 || D <= 0 || E <= 0 || K <= 0 || K > E) return -1;
+int oracle_route_ex(const uint16_t* x, const uint16_t* w_r, const double* bias,
+                    const uint16_t* w_sg, int T, int D, int E, int K, int score_mode,
+                    const double* select_bias, int bf16_weights,
+                    int32_t* idx, double* alpha, double* probs, double* gap, double* sgate) {
+    if (T < 0 || D <= 0 || E <= 0 || K <= 0 || K > E || score_mode < 0 || score_mode > 1)
+        return -1;
     int bad = 0;
 #pragma omp parallel for schedule(dynamic, 1)
     for (int t = 0; t < T; ++t) {
         double* p = (double*)malloc(sizeof(double) * (size_t)E);
+        double* key = (double*)malloc(sizeof(double) * (size_t)E);
         char* taken = (char*)calloc((size_t)E, 1);
-        if (!p || !taken) { bad = 1; free(p); free(taken); continue; }
+        if (!p || !key || !taken) { bad = 1; free(p); free(key); free(taken); continue; }
         const uint16_t* xt = x + (size_t)t * D;
         double m = -INFINITY;
         for (int e = 0; e < E; ++e) {
             p[e] = dot_bf16(xt, w_r + (size_t)e * D, D) + (bias ? bias[e] : 0.0);
             if (p[e] > m) m = p[e];
         }
-        double z = 0.0;
-        for (int e = 0; e < E; ++e) { p[e] = exp(p[e] - m); z += p[e]; }
-        for (int e = 0; e < E; ++e) p[e] /= z;
+        if (score_mode == 0) {
+            double z = 0.0;
+            for (int e = 0; e < E; ++e) { p[e] = exp(p[e] - m); z += p[e]; }
+            for (int e = 0; e < E; ++e) p[e] /= z;
+        } else {
+            for (int e = 0; e < E; ++e) p[e] = sigmoid(p[e]);
+        }
+        for (int e = 0; e < E; ++e) key[e] = p[e] + (select_bias ? select_bias[e] : 0.0);
         if (probs) memcpy(probs + (size_t)t * E, p, sizeof(double) * (size_t)E);
 
-        /* TopK by repeated selection of the largest remaining probability. */
+        /* TopK by repeated selection of the largest remaining key. */
         double sel_sum = 0.0;
         for (int k = 0; k < K; ++k) {
             int best = -1;
             for (int e = 0; e < E; ++e)
-                if (!taken[e] && (best < 0 || p[e] > p[best])) best = e;
+                if (!taken[e] && (best < 0 || key[e] > key[best])) best = e;
             taken[best] = 1;
             idx[(size_t)t * K + k] = best;
             sel_sum += p[best];
         }
-        for (int k = 0; k < K; ++k)
-            alpha[(size_t)t * K + k] = p[idx[(size_t)t * K + k]] / sel_sum;
+        for (int k = 0; k < K; ++k) {
+            double a = p[idx[(size_t)t * K + k]] / sel_sum;
+            alpha[(size_t)t * K + k] = bf16_weights ? round_to_bf16(a) : a;
+        }
         if (gap) {
             double next = -INFINITY;
             for (int e = 0; e < E; ++e)
-                if (!taken[e] && p[e] > next) next = p[e];
-            gap[t] = (K == E) ? INFINITY : p[idx[(size_t)t * K + K - 1]] - next;
+                if (!taken[e] && key[e] > next) next = key[e];
+            gap[t] = (K == E) ? INFINITY : key[idx[(size_t)t * K + K - 1]] - next;
         }
         if (sgate) sgate[t] = w_sg ? sigmoid(dot_bf16(xt, w_sg, D)) : 0.0;
         free(p);
+        free(key);
         free(taken);
     }
     return bad ? -1 : 0;
+}
+
+/* The softmax router without selection bias and with fp32 weights (the layer's default). */
+int oracle_route(const uint16_t* x, const uint16_t* w_r, const double* bias,
+                 const uint16_t* w_sg, int T, int D, int E, int K,
+                 int32_t* idx, double* alpha, double* probs, double* gap, double* sgate) {
+    return oracle_route_ex(x, w_r, bias, w_sg, T, D, E, K, 0, NULL, 0, idx, alpha, probs, gap,
+                           sgate);
 }
 
 /*

@@ -17,9 +17,14 @@ MUTANTS = {
     "down_transposed": ("s += bf16_to_double(row[n]) * h[n];",
                         "s += bf16_to_double(w_d[(size_t)n * D + d]) * h[n];"),
     "drop_routing_weight": ("acc[d] += a * s;", "acc[d] += s;"),
-    "no_renormalisation": ("alpha[(size_t)t * K + k] = p[idx[(size_t)t * K + k]] / sel_sum;",
-                           "alpha[(size_t)t * K + k] = p[idx[(size_t)t * K + k]];"),
-    "ties_to_higher_index": ("p[e] > p[best]", "p[e] >= p[best]"),
+    "no_renormalisation": ("double a = p[idx[(size_t)t * K + k]] / sel_sum;",
+                           "double a = p[idx[(size_t)t * K + k]];"),
+    "ties_to_higher_index": ("key[e] > key[best]", "key[e] >= key[best]"),
+    "selection_bias_in_weights": ("sel_sum += p[best];", "sel_sum += key[best];"),
+    "sigmoid_scores_as_softmax": ("for (int e = 0; e < E; ++e) p[e] = sigmoid(p[e]);",
+                                  "for (int e = 0; e < E; ++e) p[e] = exp(p[e] - m);"),
+    "bf16_weights_truncated": ("u = (u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u;",
+                               "u = u & 0xFFFF0000u;"),
     "shared_gate_no_sigmoid": ("sgate[t] = w_sg ? sigmoid(dot_bf16(xt, w_sg, D)) : 0.0;",
                                "sgate[t] = w_sg ? dot_bf16(xt, w_sg, D) : 0.0;"),
     "drop_logit_bias": ("+ (bias ? bias[e] : 0.0)", "+ 0.0"),

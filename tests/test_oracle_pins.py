@@ -45,6 +45,88 @@ def test_renorm_worked_example(oracle_mod):
     assert r["alpha"][0].sum() == pytest.approx(float(g["weight_sum"]), abs=1e-15)
 
 
+def test_sigmoid_worked_example(oracle_mod):
+    """The worked example exactly as the page states it: sigmoid affinities (x = 0 and a
+    logit bias of logit(score) make s_i equal the printed scores), top-2, weights
+    0.90/1.50 = 0.60 and 0.40."""
+    g = golden("renorm_worked_example.txt")
+    E, K = int(g["E"]), int(g["K"])
+    scores = np.array([float(g[f"score {i}"]) for i in range(1, E + 1)])
+    x = torch.zeros((1, 8), dtype=torch.bfloat16)
+    w_r = torch.zeros((E, 8), dtype=torch.bfloat16)
+    r = oracle_mod.route(x, w_r, K, logit_bias=np.log(scores / (1 - scores)), score="sigmoid")
+    assert list(r["idx"][0]) == [1, 4]
+    np.testing.assert_allclose(r["probs"][0], scores, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(r["alpha"][0], [float(g["weight 2"]), float(g["weight 5"])],
+                               rtol=0, atol=1e-12)
+
+
+def test_selection_only_bias(oracle_mod):
+    """"1.6 混合专家（MoE）", section 三 (DeepSeek-V3 bias method): the bias b_i is added to the
+    affinity for selection only; the weights normalise the raw s_i.  With s = (0.2, 0.9,
+    0.3, 0.1, 0.6) and b = 0.55 on expert 3 (1-based) the keys are (0.2, 0.9, 0.85, 0.1,
+    0.6): experts 2 and 3 win, weighted 0.9/1.2 = 0.75 and 0.3/1.2 = 0.25 -- not by the
+    biased keys (0.9/1.75) and not the unbiased winners (2 and 5)."""
+    s = np.array([0.2, 0.9, 0.3, 0.1, 0.6])
+    b = np.array([0.0, 0.0, 0.55, 0.0, 0.0])
+    x = torch.zeros((1, 8), dtype=torch.bfloat16)
+    w_r = torch.zeros((5, 8), dtype=torch.bfloat16)
+    r = oracle_mod.route(x, w_r, 2, logit_bias=np.log(s / (1 - s)), score="sigmoid",
+                         select_bias=b)
+    assert list(r["idx"][0]) == [1, 2]
+    np.testing.assert_allclose(r["alpha"][0], [0.75, 0.25], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(r["gap"][0], 0.85 - 0.6, atol=1e-12)
+
+
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_sigmoid_router_matches_library(oracle_mod, with_bias):
+    """Sigmoid scores = scipy expit of the logits; selection = stable sort of the keys
+    (scores + selection bias); weights = selected raw scores over their sum."""
+    x, w = _random_router(23, 128, 32, seed=9)
+    b = np.linspace(-0.3, 0.3, 32) if with_bias else None
+    r = oracle_mod.route(x, w, 6, score="sigmoid", select_bias=b)
+    s = scipy.special.expit(_f64(x) @ _f64(w).T)
+    np.testing.assert_allclose(r["probs"], s, rtol=1e-13)
+    key = s + (b if with_bias else 0.0)
+    order = np.argsort(-key, axis=1, kind="stable")[:, :6]
+    np.testing.assert_array_equal(r["idx"], order)
+    sel = np.take_along_axis(s, order, axis=1)
+    np.testing.assert_allclose(r["alpha"], sel / sel.sum(1, keepdims=True), rtol=1e-12)
+
+
+def test_softmax_with_selection_bias(oracle_mod):
+    """Softmax scores with a selection-only bias: keys = p + b, weights from p alone."""
+    x, w = _random_router(15, 64, 16, seed=10)
+    b = np.linspace(0.0, 0.2, 16)
+    r = oracle_mod.route(x, w, 4, select_bias=b)
+    p = scipy.special.softmax(_f64(x) @ _f64(w).T, axis=1)
+    order = np.argsort(-(p + b), axis=1, kind="stable")[:, :4]
+    np.testing.assert_array_equal(r["idx"], order)
+    sel = np.take_along_axis(p, order, axis=1)
+    np.testing.assert_allclose(r["alpha"], sel / sel.sum(1, keepdims=True), rtol=1e-12)
+
+
+def test_bf16_routing_weights(oracle_mod):
+    """"MoE", section 2: the renormalised fp32 weights are cast back to the model dtype --
+    the fp64 weights rounded to fp32 and then to bf16 by torch (round to nearest even)."""
+    x, w = _random_router(31, 128, 24, seed=11)
+    ref = oracle_mod.route(x, w, 5)
+    r = oracle_mod.route(x, w, 5, bf16_weights=True)
+    np.testing.assert_array_equal(r["idx"], ref["idx"])
+    want = torch.tensor(ref["alpha"]).to(torch.float32).to(torch.bfloat16).to(torch.float64)
+    np.testing.assert_array_equal(r["alpha"], want.numpy())
+
+
+def test_residual_is_added(oracle_mod):
+    """"MoE", section 4: h_out = h + y_MoE."""
+    cfg = LayerConfig("res", T=6, D=64, E=4, K=2, f=32)
+    inp = make_inputs(cfg)
+    h = (torch.randn((6, 64), generator=torch.Generator().manual_seed(3))).to(torch.bfloat16)
+    _, y = oracle_mod.layer(inp)
+    _, yh = oracle_mod.layer(inp, residual=h)
+    np.testing.assert_allclose(yh, y + _f64(h), rtol=0, atol=0)
+
+
 def _random_router(T, D, E, seed):
     gen = torch.Generator().manual_seed(seed)
     x = torch.randn((T, D), generator=gen).to(torch.bfloat16)
