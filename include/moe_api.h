@@ -60,8 +60,14 @@ typedef enum {
     MOE_ERR_DEVICE = -7       /* device status only: inconsistent routing table seen */
 } moe_status;
 
-/* Flags of moe_layer_params.flags. */
+/* Flags of moe_layer_params.flags and moe_route_ex. */
 #define MOE_FLAG_DETERMINISTIC 1u /* combine by a fixed-order gather instead of fp32 atomics */
+#define MOE_FLAG_BF16_WEIGHTS 2u  /* round the routing weights to bf16 ("MoE", section 2:
+                                     the renormalised scores return to the model dtype) */
+
+/* Router score functions. */
+#define MOE_SCORE_SOFTMAX 0 /* p = softmax(r) over all experts ("MoE", section 2) */
+#define MOE_SCORE_SIGMOID 1 /* s_e = sigma(r_e) per expert ("1.6 混合专家（MoE）", section 2) */
 
 /* Human-readable name of a status code (static string). */
 MOE_API const char* moe_status_string(int status);
@@ -99,6 +105,21 @@ MOE_API int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* 
               const moe_bf16* w_shared_gate, int T, int D, int E, int K,
               int32_t* topk_idx, float* topk_w, int32_t* expert_counts, float* shared_gate,
               void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * moe_route with the router variants of "1.6 混合专家（MoE）", sections 2-3:
+ *   score_mode   MOE_SCORE_SOFTMAX (as moe_route) or MOE_SCORE_SIGMOID (s_e = sigma(r_e))
+ *   select_bias  [E] fp32 added to the scores for the TopK selection only (the DeepSeek-V3
+ *                bias method: the weights normalise the raw scores), or NULL
+ *   flags        MOE_FLAG_BF16_WEIGHTS to round the weights to bf16
+ * The weights are alpha_k = score_k / sum_{j in I} score_j; the selection keys are
+ * score + select_bias.  Other arguments, outputs and errors as moe_route.
+ */
+MOE_API int moe_route_ex(const moe_bf16* x, const moe_bf16* w_router, const float* logit_bias,
+                         const moe_bf16* w_shared_gate, int T, int D, int E, int K,
+                         int score_mode, const float* select_bias, unsigned flags,
+                         int32_t* topk_idx, float* topk_w, int32_t* expert_counts,
+                         float* shared_gate, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * moe_route_noalloc: the router of moe_route (same kernel, same outputs, same argument
@@ -200,6 +221,9 @@ typedef struct moe_layer_params {
     float* topk_w_out;                /* optional [T, K], or NULL */
     int32_t* expert_counts_out;       /* optional [E], or NULL */
     void* const* step_events;         /* optional: MOE_NUM_STEP_EVENTS cudaEvent_t handles */
+    int score_mode;                   /* MOE_SCORE_SOFTMAX (0) or MOE_SCORE_SIGMOID */
+    const float* select_bias;         /* [E] selection-only bias, or NULL (see moe_route_ex) */
+    const moe_bf16* residual;         /* [T, D] decoder residual h: out = h + y, or NULL */
 } moe_layer_params;
 
 /*
@@ -223,7 +247,8 @@ enum {
 
 /*
  * The whole layer: route, permute, grouped SwiGLU (routed experts and, when present, the
- * shared expert scaled by sigma(w_s . x)), combine to out [T, D] bf16.  No host
+ * shared expert scaled by sigma(w_s . x)), combine to out [T, D] bf16 -- plus the residual
+ * h when p->residual is set ("MoE", section 4: h_out = h + y_MoE).  No host
  * synchronisation; every step reads its sizes from the device, so the call can be
  * captured in a CUDA graph.  workspace: at least moe_workspace_size(T, D, E, K, f, f_s)
  * bytes, 256-byte aligned.

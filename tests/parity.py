@@ -47,10 +47,16 @@ def output_error(y_gpu_bf16: np.ndarray, y_ref: np.ndarray):
     return float(d.max()) if d.size else 0.0, rms, float((d / allow).max()) if d.size else 0.0
 
 
-def check_route(orc, gpu_idx, gpu_w, gpu_counts=None, E=None) -> RouteReport:
-    """orc: oracle.route(...) dict; gpu_*: numpy arrays."""
+def check_route(orc, gpu_idx, gpu_w, gpu_counts=None, select_bias=None,
+                bf16_weights=False) -> RouteReport:
+    """orc: oracle.route(...) dict; gpu_*: numpy arrays.  The selection keys are the scores
+    plus the selection-only bias; with bf16 weights both sides round independently, so one
+    bf16 ulp of the weight is allowed on top of W_TOL."""
     o_idx, o_alpha, probs, gap = orc["idx"], orc["alpha"], orc["probs"], orc["gap"]
     T, K = o_idx.shape
+    sb = None if select_bias is None else np.asarray(
+        select_bias.cpu() if hasattr(select_bias, "cpu") else select_bias, np.float64)
+    keys = probs if sb is None else probs + sb
     assert gpu_idx.shape == (T, K)
     assert np.all((gpu_idx >= 0) & (gpu_idx < probs.shape[1])), "index out of range"
     for t in range(T):
@@ -61,16 +67,18 @@ def check_route(orc, gpu_idx, gpu_w, gpu_counts=None, E=None) -> RouteReport:
     assert not bad.any(), f"selection differs on non-near-tie tokens {np.nonzero(bad)[0][:10]}"
     # near-tie tokens: the CUDA choice must be a valid top-K within the tie gap
     for t in np.nonzero(~same)[0]:
-        kth = probs[t, o_idx[t, K - 1]]
-        chosen = probs[t, gpu_idx[t]]
+        kth = keys[t, o_idx[t, K - 1]]
+        chosen = keys[t, gpu_idx[t]]
         assert np.all(chosen >= kth - NEAR_TIE), f"token {t}: invalid near-tie selection"
-    # weights: compare per expert; renormalise the oracle probs over the CUDA set
+    # weights: compare per expert; renormalise the oracle scores over the CUDA set
     sel = np.take_along_axis(probs, gpu_idx.astype(np.int64), axis=1)
     ref_w = sel / sel.sum(1, keepdims=True)
+    allow = W_TOL + (2 * half_ulp_bf16(ref_w) if bf16_weights else 0.0)
     w_err = float(np.abs(gpu_w - ref_w).max()) if T else 0.0
-    assert w_err <= W_TOL, f"routing weight error {w_err}"
-    # descending order of the CUDA list
-    assert np.all(np.diff(gpu_w, axis=1) <= 1e-6), "weights not in descending order"
+    assert np.all(np.abs(gpu_w - ref_w) <= allow), f"routing weight error {w_err}"
+    # the CUDA list is ordered by descending key
+    gk = np.take_along_axis(keys, gpu_idx.astype(np.int64), axis=1)
+    assert np.all(np.diff(gk, axis=1) <= 1e-6), "selection not in descending key order"
     if gpu_counts is not None:
         bc = np.bincount(gpu_idx.reshape(-1), minlength=len(gpu_counts))
         np.testing.assert_array_equal(gpu_counts, bc)
@@ -96,13 +104,15 @@ def oracle_outputs(orc_mod, inp, idx, alpha, tokens, shared_gate=None):
                            None if inp.w_shared_down is None else inp.w_shared_down.cpu(), sg)
 
 
-def check_layer(orc_mod, inp, y_gpu, gpu_idx, gpu_w, tokens=None, orc=None):
-    """Route on the oracle (all tokens), compare routing, then compare y on `tokens`
-    (all when None).  Returns a dict of measured errors."""
+def check_layer(orc_mod, inp, y_gpu, gpu_idx, gpu_w, tokens=None, orc=None, score="softmax",
+                select_bias=None, bf16_weights=False, residual=None):
+    """Route on the oracle (all tokens), compare routing, then compare y (+ residual) on
+    `tokens` (all when None).  Returns a dict of measured errors."""
     cfg = inp.cfg
     if orc is None:
-        orc = orc_mod.route(inp.x, inp.w_router, cfg.K, inp.logit_bias, inp.w_shared_gate)
-    rep = check_route(orc, gpu_idx, gpu_w)
+        orc = orc_mod.route(inp.x, inp.w_router, cfg.K, inp.logit_bias, inp.w_shared_gate,
+                            score, select_bias, bf16_weights)
+    rep = check_route(orc, gpu_idx, gpu_w, select_bias=select_bias, bf16_weights=bf16_weights)
     T = cfg.T
     toks = np.arange(T) if tokens is None else np.asarray(tokens)
     # forced routing: the oracle's own weights over the CUDA set for differing tokens
@@ -112,7 +122,11 @@ def check_layer(orc_mod, inp, y_gpu, gpu_idx, gpu_w, tokens=None, orc=None):
         idx[t] = gpu_idx[t]
         p = orc["probs"][t, gpu_idx[t]]
         alpha[t] = p / p.sum()
+        if bf16_weights:
+            alpha[t] = torch.tensor(alpha[t]).float().bfloat16().double().numpy()
     y_ref = oracle_outputs(orc_mod, inp, idx, alpha, toks, orc["shared_gate"])
+    if residual is not None:
+        y_ref = y_ref + residual[torch.as_tensor(toks, device=residual.device)].cpu().double().numpy()
     y = y_gpu[torch.as_tensor(toks, device=y_gpu.device)].float().cpu().numpy().astype(np.float64)
     err, rms, used = output_error(y, y_ref)
     assert rms > 0

@@ -288,3 +288,78 @@ def test_full_size_layer(moe, oracle_mod, name):
     rep = check_layer(oracle_mod, inp, y, gi, _np(w), tokens=toks)
     np.testing.assert_array_equal(_np(counts), np.bincount(gi.reshape(-1), minlength=cfg.E))
     print(name, rep, "U =", int((_np(counts) > 0).sum()))
+
+
+# ------------------------------------------------------------------ router variants, residual
+
+
+VARIANTS = [
+    dict(score="sigmoid"),
+    dict(score="sigmoid", select_bias=True),
+    dict(score="softmax", select_bias=True),
+    dict(score="softmax", bf16_weights=True),
+    dict(score="sigmoid", select_bias=True, bf16_weights=True),
+]
+
+
+def _variant(cfg, v):
+    sb = None
+    if v.get("select_bias"):
+        g = torch.Generator().manual_seed(21)
+        sb = (0.05 * torch.randn(cfg.E, generator=g)).float().cuda()
+    return dict(score=v.get("score", "softmax"), select_bias=sb,
+                bf16_weights=bool(v.get("bf16_weights", False)))
+
+
+@pytest.mark.parametrize("vi", range(len(VARIANTS)))
+@pytest.mark.parametrize("name", ["decode", "tc_router_shared", "single_token"])
+def test_route_variants(moe, oracle_mod, name, vi):
+    cfg = SMALL_LAYERS[name]
+    inp = make_inputs(cfg).to("cuda")
+    v = _variant(cfg, VARIANTS[vi])
+    idx, w, counts, sg = moe.route(inp.x, inp.w_router, cfg.K, inp.logit_bias, inp.w_shared_gate,
+                                   **v)
+    torch.cuda.synchronize()
+    orc = oracle_mod.route(inp.x, inp.w_router, cfg.K, inp.logit_bias, inp.w_shared_gate,
+                           v["score"], v["select_bias"], v["bf16_weights"])
+    check_route(orc, _np(idx), _np(w), _np(counts), select_bias=v["select_bias"],
+                bf16_weights=v["bf16_weights"])
+
+
+def test_route_sigmoid_worked_example(moe):
+    """The worked example in its own form: sigmoid affinities 0.9 and 0.6 win and are
+    renormalised to 0.6 and 0.4; a selection bias of 0.35 on the 0.3 expert makes it win
+    the second slot while the weights still use the raw scores (0.9/1.2, 0.3/1.2)."""
+    s = np.array([0.2, 0.9, 0.3, 0.1, 0.6, 0.05, 0.05, 0.05])
+    x = torch.zeros((2, 128), dtype=torch.bfloat16, device="cuda")
+    w_r = torch.zeros((8, 128), dtype=torch.bfloat16, device="cuda")
+    bias = torch.tensor(np.log(s / (1 - s)), dtype=torch.float32, device="cuda")
+    idx, w, _, _ = moe.route(x, w_r, 2, bias, score="sigmoid")
+    torch.cuda.synchronize()
+    assert _np(idx).tolist() == [[1, 4]] * 2
+    np.testing.assert_allclose(_np(w), [[0.6, 0.4]] * 2, atol=1e-6)
+    sb = torch.zeros(8, dtype=torch.float32, device="cuda")
+    sb[2] = 0.35
+    idx, w, _, _ = moe.route(x, w_r, 2, bias, score="sigmoid", select_bias=sb)
+    torch.cuda.synchronize()
+    assert _np(idx).tolist() == [[1, 2]] * 2
+    np.testing.assert_allclose(_np(w), [[0.75, 0.25]] * 2, atol=1e-6)
+
+
+@pytest.mark.parametrize("det", [False, True])
+@pytest.mark.parametrize("vi", [0, 2, 4])
+@pytest.mark.parametrize("name", ["tiny", "tc_router_shared"])
+def test_layer_variants_with_residual(moe, oracle_mod, name, vi, det):
+    cfg = SMALL_LAYERS[name]
+    inp = make_inputs(cfg).to("cuda")
+    v = _variant(cfg, VARIANTS[vi])
+    g = torch.Generator().manual_seed(31)
+    h = torch.randn((cfg.T, cfg.D), generator=g).to(torch.bfloat16).cuda()
+    layer = moe.MoELayer.from_inputs(inp, deterministic=det, **v)
+    idx = torch.empty((cfg.T, cfg.K), dtype=torch.int32, device="cuda")
+    w = torch.empty((cfg.T, cfg.K), dtype=torch.float32, device="cuda")
+    y = layer(inp.x, topk_idx=idx, topk_w=w, residual=h)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    rep = check_layer(oracle_mod, inp, y, _np(idx), _np(w), residual=h, **v)
+    print(name, VARIANTS[vi], det, rep)

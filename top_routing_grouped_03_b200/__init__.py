@@ -19,6 +19,8 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moe_api.h")
 
 MOE_FLAG_DETERMINISTIC = 1
+MOE_FLAG_BF16_WEIGHTS = 2
+SCORES = {"softmax": 0, "sigmoid": 1}
 
 _lib = None
 
@@ -39,6 +41,8 @@ class LayerParams(ctypes.Structure):
         ("f", ctypes.c_int), ("f_s", ctypes.c_int), ("flags", ctypes.c_uint),
         ("topk_idx_out", ctypes.c_void_p), ("topk_w_out", ctypes.c_void_p),
         ("expert_counts_out", ctypes.c_void_p), ("step_events", ctypes.c_void_p),
+        ("score_mode", ctypes.c_int), ("select_bias", ctypes.c_void_p),
+        ("residual", ctypes.c_void_p),
     ]
 
 
@@ -65,6 +69,9 @@ def lib() -> ctypes.CDLL:
         L.moe_workspace_size.restype = Z
         L.moe_route.argtypes = [P, P, P, P, I, I, I, I, P, P, P, P, P, Z, P]
         L.moe_route.restype = I
+        L.moe_route_ex.argtypes = [P, P, P, P, I, I, I, I, I, P, ctypes.c_uint, P, P, P, P, P,
+                                   Z, P]
+        L.moe_route_ex.restype = I
         L.moe_permute.argtypes = [P, P, P, I, I, I, P, P, P, P, P, P]
         L.moe_permute.restype = I
         L.moe_grouped_swiglu.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P, P, Z, P]
@@ -122,9 +129,11 @@ def alloc_workspace(T, D, E, K, f, f_s=0, device=None) -> torch.Tensor:
     return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
 
 
-def route(x, w_router, K, logit_bias=None, w_shared_gate=None, workspace=None, stream=None):
+def route(x, w_router, K, logit_bias=None, w_shared_gate=None, workspace=None, stream=None,
+          score="softmax", select_bias=None, bf16_weights=False):
     """Router step.  Returns (topk_idx [T,K] int32, topk_w [T,K] f32, expert_counts [E]
-    int32, shared_gate [T] f32 or None)."""
+    int32, shared_gate [T] f32 or None).  score / select_bias / bf16_weights select the
+    router variants of moe_route_ex."""
     T, D = x.shape
     E = w_router.shape[0]
     dev = x.device
@@ -133,8 +142,15 @@ def route(x, w_router, K, logit_bias=None, w_shared_gate=None, workspace=None, s
     w = torch.empty((T, K), dtype=torch.float32, device=dev)
     counts = torch.empty((E,), dtype=torch.int32, device=dev)
     sg = torch.empty((T,), dtype=torch.float32, device=dev) if w_shared_gate is not None else None
-    rc = lib().moe_route(_p(x), _p(w_router), _p(logit_bias), _p(w_shared_gate), T, D, E, K,
-                         _p(idx), _p(w), _p(counts), _p(sg), _p(ws), ws.numel(), _stream(stream))
+    if score == "softmax" and select_bias is None and not bf16_weights:
+        rc = lib().moe_route(_p(x), _p(w_router), _p(logit_bias), _p(w_shared_gate), T, D, E, K,
+                             _p(idx), _p(w), _p(counts), _p(sg), _p(ws), ws.numel(),
+                             _stream(stream))
+    else:
+        rc = lib().moe_route_ex(_p(x), _p(w_router), _p(logit_bias), _p(w_shared_gate), T, D, E,
+                                K, SCORES[score], _p(select_bias),
+                                MOE_FLAG_BF16_WEIGHTS if bf16_weights else 0, _p(idx), _p(w),
+                                _p(counts), _p(sg), _p(ws), ws.numel(), _stream(stream))
     _check(rc, "moe_route")
     return idx, w, counts, sg
 
@@ -226,7 +242,8 @@ class MoELayer:
     """
 
     def __init__(self, w_router, w_gate_up, w_down, K, logit_bias=None, w_shared_gate=None,
-                 w_shared_gate_up=None, w_shared_down=None, deterministic=False):
+                 w_shared_gate_up=None, w_shared_down=None, deterministic=False,
+                 score="softmax", select_bias=None, bf16_weights=False):
         self.w_router, self.w_gate_up, self.w_down = w_router, w_gate_up, w_down
         self.logit_bias = logit_bias
         self.w_shared_gate, self.w_shared_gate_up = w_shared_gate, w_shared_gate_up
@@ -235,14 +252,18 @@ class MoELayer:
         self.f = w_gate_up.shape[1] // 2
         self.f_s = 0 if w_shared_gate_up is None else w_shared_gate_up.shape[0] // 2
         self.K = K
-        self.flags = MOE_FLAG_DETERMINISTIC if deterministic else 0
+        self.flags = (MOE_FLAG_DETERMINISTIC if deterministic else 0) | \
+            (MOE_FLAG_BF16_WEIGHTS if bf16_weights else 0)
+        self.score_mode = SCORES[score]
+        self.select_bias = select_bias
         self._ws = None
         self._ws_T = -1
 
     @classmethod
-    def from_inputs(cls, inp, deterministic=False):
+    def from_inputs(cls, inp, deterministic=False, **router):
         return cls(inp.w_router, inp.w_gate_up, inp.w_down, inp.cfg.K, inp.logit_bias,
-                   inp.w_shared_gate, inp.w_shared_gate_up, inp.w_shared_down, deterministic)
+                   inp.w_shared_gate, inp.w_shared_gate_up, inp.w_shared_down, deterministic,
+                   **router)
 
     def workspace(self, T: int) -> torch.Tensor:
         if self._ws is None or self._ws_T < T:
@@ -251,25 +272,27 @@ class MoELayer:
             self._ws_T = T
         return self._ws
 
-    def params(self, x, topk_idx=None, topk_w=None, counts=None, events=None) -> LayerParams:
+    def params(self, x, topk_idx=None, topk_w=None, counts=None, events=None,
+               residual=None) -> LayerParams:
         T = x.shape[0]
         ev = None if events is None else ctypes.cast(events, ctypes.c_void_p)
         return LayerParams(_p(x), _p(self.w_router), _p(self.logit_bias), _p(self.w_gate_up),
                            _p(self.w_down), _p(self.w_shared_gate), _p(self.w_shared_gate_up),
                            _p(self.w_shared_down), T, self.D, self.E, self.K, self.f, self.f_s,
-                           self.flags, _p(topk_idx), _p(topk_w), _p(counts), ev)
+                           self.flags, _p(topk_idx), _p(topk_w), _p(counts), ev,
+                           self.score_mode, _p(self.select_bias), _p(residual))
 
     def __call__(self, x, out=None, topk_idx=None, topk_w=None, counts=None, stream=None,
-                 step_events=None):
-        """y = layer(x) on the device.  ``step_events``: an ``event_array(...)`` to time
-        each kernel of the call."""
+                 step_events=None, residual=None):
+        """y = layer(x) (+ residual h) on the device.  ``step_events``: an
+        ``event_array(...)`` to time each kernel of the call."""
         T = x.shape[0]
         if x.shape[1] != self.D:
             raise MoEError(-1, "moe_layer_forward (x has the wrong width)")
         out = out if out is not None else torch.empty((T, self.D), dtype=torch.bfloat16,
                                                       device=x.device)
         ws = self.workspace(T)
-        prm = self.params(x, topk_idx, topk_w, counts, step_events)
+        prm = self.params(x, topk_idx, topk_w, counts, step_events, residual)
         rc = lib().moe_layer_forward(ctypes.byref(prm), _p(out), _p(ws), ws.numel(),
                                      _stream(stream))
         _check(rc, "moe_layer_forward")

@@ -4,8 +4,8 @@
 // + sigma(w_s^T x_t) E_s(x_t); section 3.2: the expert outputs are index-added back to
 // their tokens.  One thread owns 8 consecutive features of one token (16-byte loads and
 // stores) and sums, in this fixed order: the fp32 accumulator row (if any), the K routed
-// rows in slot order, then the gated shared-expert row; the result is rounded once to
-// bf16 (round to nearest even).
+// rows in slot order, the gated shared-expert row, then the decoder residual h (section 4:
+// h_out = h + y); the result is rounded once to bf16 (round to nearest even).
 #include <algorithm>
 
 #include "common.cuh"
@@ -64,6 +64,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineLaunch a) {
             const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.shared_out) + i);
             add8(acc, v, __ldg(a.shared_gate + t));
         }
+        if (a.residual) add8(acc, __ldg(reinterpret_cast<const uint4*>(a.residual) + i), 1.f);
         uint4 o;
         o.x = pack_bf16x2(acc[0], acc[1]);
         o.y = pack_bf16x2(acc[2], acc[3]);

@@ -84,6 +84,9 @@ struct RouterLaunch {
     // layer's fp32 accumulator)
     float* zero_acc;
     int zero_cols;
+    int score_mode;           // 0: softmax over the experts; 1: per-expert sigmoid
+    const float* select_bias; // [E] added to the scores for the selection only, or NULL
+    int bf16_weights;         // round the renormalised weights to bf16
 };
 cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bool pdl = false);
 
@@ -130,6 +133,7 @@ struct GroupedGemmLaunch {
     bf16* final_out;
     int final_rows;
     unsigned* done;
+    const bf16* final_residual;  // [final_rows, D] added in the conversion, or NULL
     // gate_up with gather_tok: room for the rows in expert order [rows, D]; when given, the
     // CTA-pair kernel may be used (rows gathered by a copy kernel first)
     bf16* gather_buf;
@@ -140,6 +144,7 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
                                 bool pdl = false);
 
 struct CombineLaunch {
+    const bf16* residual;  // [T, D] added before the bf16 rounding, or NULL
     const float* out_acc;
     const float* y_sorted;
     const int32_t* slot_to_row;

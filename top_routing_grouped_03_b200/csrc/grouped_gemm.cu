@@ -82,6 +82,7 @@ struct Params {
     bf16* final_out;            // down: when set, convert acc_out [final_rows, out_cols] to
     int final_rows;             //   bf16 here once every CTA of the grid has added its tiles
     unsigned* done;             //   (grid barrier counter, zero at launch)
+    const bf16* final_residual; //   + this bf16 [final_rows, out_cols] when not NULL
 };
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
@@ -116,10 +117,15 @@ __device__ __noinline__ void finalize_output(const Params& p) {
     if (!s_ok) return;
     const long long n4 = static_cast<long long>(p.final_rows) * p.out_cols / 4;
     const float4* src = reinterpret_cast<const float4*>(p.acc_out);
+    const uint2* res = reinterpret_cast<const uint2*>(p.final_residual);
     uint2* dst = reinterpret_cast<uint2*>(p.final_out);
     for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
          i += static_cast<long long>(gridDim.x) * blockDim.x) {
-        const float4 v = __ldcg(src + i);
+        float4 v = __ldcg(src + i);
+        if (res) {
+            const uint2 r = __ldg(res + i);
+            v.x += bf16_lo(r.x); v.y += bf16_hi(r.x); v.z += bf16_lo(r.y); v.w += bf16_hi(r.y);
+        }
         dst[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
     }
 }
@@ -1083,6 +1089,7 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
     p.final_out = (!a.gate_up && a.acc_out && a.done) ? a.final_out : nullptr;
     p.final_rows = a.final_rows;
     p.done = a.done;
+    p.final_residual = a.final_residual;
     const long long max_tiles = (static_cast<long long>(ceil_div(a.rows, BN)) + a.E) * p.nf;
     const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
     if (pairs) {

@@ -120,8 +120,19 @@ int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* logit_bi
               const moe_bf16* w_shared_gate, int T, int D, int E, int K, int32_t* topk_idx,
               float* topk_w, int32_t* expert_counts, float* shared_gate, void* workspace,
               size_t ws_bytes, void* stream) {
+    return moe_route_ex(x, w_router, logit_bias, w_shared_gate, T, D, E, K, MOE_SCORE_SOFTMAX,
+                        nullptr, 0u, topk_idx, topk_w, expert_counts, shared_gate, workspace,
+                        ws_bytes, stream);
+}
+
+int moe_route_ex(const moe_bf16* x, const moe_bf16* w_router, const float* logit_bias,
+                 const moe_bf16* w_shared_gate, int T, int D, int E, int K, int score_mode,
+                 const float* select_bias, unsigned flags, int32_t* topk_idx, float* topk_w,
+                 int32_t* expert_counts, float* shared_gate, void* workspace, size_t ws_bytes,
+                 void* stream) {
     int rc = check_shape(T, D, E, K, 128, 0);
     if (rc) return rc;
+    if (score_mode != MOE_SCORE_SOFTMAX && score_mode != MOE_SCORE_SIGMOID) return MOE_ERR_ARG;
     if (!w_router || !expert_counts) return MOE_ERR_ARG;
     if (T > 0 && (!x || !topk_idx || !topk_w || (w_shared_gate && !shared_gate))) return MOE_ERR_ARG;
     if (!aligned16(x) || !aligned16(w_router) || (w_shared_gate && !aligned16(w_shared_gate)))
@@ -146,6 +157,9 @@ int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* logit_bi
     a.counts = expert_counts;
     a.shared_gate = shared_gate;
     a.status = at<int>(workspace, L.status);
+    a.score_mode = score_mode;
+    a.select_bias = select_bias;
+    a.bf16_weights = (flags & MOE_FLAG_BF16_WEIGHTS) ? 1 : 0;
     const int sms = num_sms_current();
     const cudaError_t err = router_uses_tensor_cores(T, E) ? launch_router_tc(a, sms, s)
                                                            : launch_router(a, sms, s);
@@ -251,8 +265,9 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     if (T > 0 && (!p->x || !out)) return MOE_ERR_ARG;
     if (shared && (!p->w_shared_gate || !p->w_shared_gate_up || !p->w_shared_down)) return MOE_ERR_ARG;
     if (!shared && (p->w_shared_gate || p->w_shared_gate_up || p->w_shared_down)) return MOE_ERR_ARG;
+    if (p->score_mode != MOE_SCORE_SOFTMAX && p->score_mode != MOE_SCORE_SIGMOID) return MOE_ERR_ARG;
     if (!aligned16(p->x) || !aligned16(p->w_router) || !aligned16(p->w_gate_up) ||
-        !aligned16(p->w_down) || !aligned16(out) ||
+        !aligned16(p->w_down) || !aligned16(out) || !aligned16(p->residual) ||
         (shared && (!aligned16(p->w_shared_gate) || !aligned16(p->w_shared_gate_up) ||
                     !aligned16(p->w_shared_down))))
         return MOE_ERR_ALIGN;
@@ -299,6 +314,9 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     r.status = status;
     r.zero_acc = use_acc ? out_acc : nullptr;
     r.zero_cols = D;
+    r.score_mode = p->score_mode;
+    r.select_bias = p->select_bias;
+    r.bf16_weights = (p->flags & MOE_FLAG_BF16_WEIGHTS) ? 1 : 0;
     if (!mark(MOE_EV_ROUTER)) return MOE_ERR_CUDA;
     if ((router_uses_tensor_cores(T, E) ? launch_router_tc(r, sms, s) : launch_router(r, sms, s)) !=
         cudaSuccess)
@@ -344,10 +362,12 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     dn.status = status;
     // without the fixed-order combine, the last down launch also writes the bf16 output
     unsigned* done = at<unsigned>(workspace, L.status + 64);  // inside the cleared header
+    const bf16* residual = reinterpret_cast<const bf16*>(p->residual);
     if (!det && !shared) {
         dn.final_out = reinterpret_cast<bf16*>(out);
         dn.final_rows = T;
         dn.done = done;
+        dn.final_residual = residual;
     }
     if (!mark(MOE_EV_DOWN) || launch_grouped_gemm(dn, sms, s, true) != cudaSuccess)
         return MOE_ERR_CUDA;
@@ -377,6 +397,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
             sd.final_out = reinterpret_cast<bf16*>(out);
             sd.final_rows = T;
             sd.done = done;
+            sd.final_residual = residual;
         }
         if (launch_grouped_gemm(sd, sms, s, true) != cudaSuccess) return MOE_ERR_CUDA;
     }
@@ -384,6 +405,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     if (!det) return mark(MOE_EV_COMBINE) && mark(MOE_EV_END) ? MOE_OK : MOE_ERR_CUDA;
     // fixed order: out_acc's shared part (if any) + the routed rows in slot order
     CombineLaunch c{};
+    c.residual = residual;
     c.out_acc = use_acc ? out_acc : nullptr;
     c.y_sorted = det ? at<float>(workspace, L.y_sorted) : nullptr;
     c.slot_to_row = pm.slot_to_row;

@@ -14,6 +14,10 @@
 //   * alpha_k = exp(r_k - r_max) / sum_{j in I} exp(r_j - r_max): the full softmax
 //     denominator cancels in the renormalisation, so only the K selected terms are
 //     exponentiated.
+//   * Variants ("1.6 混合专家（MoE）", sections 2-3): per-expert sigmoid affinities
+//     s = sigma(r) normalised over the selected experts, and a bias added to the scores
+//     for the selection only (the weights use the raw scores); optionally the weights are
+//     rounded to bf16 as the reference's cast to the model dtype does.
 //   * expert_counts[e] += 1 per selected expert (global atomics, for the permutation).
 // For many tokens (T >= 256, E a multiple of 128) the logits instead come from the
 // tcgen05 grouped GEMM as one dense [T, E] product, and router_select_kernel runs the
@@ -36,14 +40,50 @@ constexpr int kExpertsPerWarp = 2;
 template <int NV>
 __device__ __forceinline__ void select_topk_nv(const float* lg, const float* add_bias, int E,
                                                int K, int token, int lane, int32_t* topk_idx,
-                                               float* topk_w, int32_t* counts) {
-    float v[NV];
+                                               float* topk_w, int32_t* counts, int score_mode,
+                                               const float* select_bias, int bf16_weights) {
+    float v[NV];  // logits (+ the logit bias)
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
         const int e = j * 32 + lane;
         v[j] = (e < E) ? __ldcg(lg + e) + (add_bias ? __ldg(add_bias + e) : 0.f) : -FLT_MAX;
     }
-    float my_v = -FLT_MAX;
+    // scores and selection keys.  Softmax without selection bias: the key is the logit
+    // itself (softmax is increasing) and only the K selected terms are exponentiated.
+    // Otherwise the scores are the full softmax or the sigmoids, keys = scores + bias.
+    const bool on_logits = (score_mode == 0 && select_bias == nullptr);
+    float sc[NV], key[NV];
+    if (on_logits) {
+#pragma unroll
+        for (int j = 0; j < NV; ++j) { sc[j] = v[j]; key[j] = v[j]; }
+    } else {
+        if (score_mode == 0) {
+            float m = -FLT_MAX;
+#pragma unroll
+            for (int j = 0; j < NV; ++j) m = fmaxf(m, v[j]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+            float z = 0.f;
+#pragma unroll
+            for (int j = 0; j < NV; ++j) {
+                sc[j] = (j * 32 + lane < E) ? expf(v[j] - m) : 0.f;
+                z += sc[j];
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+#pragma unroll
+            for (int j = 0; j < NV; ++j) sc[j] /= z;
+        } else {
+#pragma unroll
+            for (int j = 0; j < NV; ++j) sc[j] = 1.f / (1.f + expf(-v[j]));
+        }
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const int e = j * 32 + lane;
+            key[j] = (e < E) ? sc[j] + (select_bias ? __ldg(select_bias + e) : 0.f) : -FLT_MAX;
+        }
+    }
+    float my_sc = 0.f;
     int my_i = 0;
     for (int k = 0; k < K; ++k) {
         float bv = -FLT_MAX;
@@ -51,7 +91,7 @@ __device__ __forceinline__ void select_topk_nv(const float* lg, const float* add
 #pragma unroll
         for (int j = 0; j < NV; ++j) {
             const int e = j * 32 + lane;
-            if (e < E && v[j] > bv) { bv = v[j]; bi = e; }  // strict: lowest e per lane
+            if (e < E && key[j] > bv) { bv = key[j]; bi = e; }  // strict: lowest e per lane
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
@@ -59,34 +99,47 @@ __device__ __forceinline__ void select_topk_nv(const float* lg, const float* add
             const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
             if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
         }
-        if (lane == k) { my_v = bv; my_i = bi; }
-        // retire the winner (owner lane only); -inf never wins against finite logits
+        // the winner's score comes from its owner lane, which also retires it
+        float wsc = 0.f;
 #pragma unroll
         for (int j = 0; j < NV; ++j)
-            if (j * 32 + lane == bi) v[j] = -INFINITY;
+            if (j * 32 + lane == bi) { wsc = sc[j]; key[j] = -INFINITY; }
+        wsc = __shfl_sync(0xffffffffu, wsc, bi & 31);
+        if (lane == k) { my_sc = wsc; my_i = bi; }
     }
-    const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
-    const float ex = (lane < K) ? expf(my_v - vmax) : 0.f;
-    float sum = ex;
+    // weights: the selected raw scores over their sum (for logits: exp(r - r_max) terms)
+    float num;
+    if (on_logits) {
+        const float vmax = __shfl_sync(0xffffffffu, my_sc, 0);
+        num = (lane < K) ? expf(my_sc - vmax) : 0.f;
+    } else {
+        num = (lane < K) ? my_sc : 0.f;
+    }
+    float sum = num;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
     if (lane < K) {
+        float w = num / sum;
+        if (bf16_weights) w = __bfloat162float(__float2bfloat16_rn(w));
         topk_idx[static_cast<size_t>(token) * K + lane] = my_i;
-        topk_w[static_cast<size_t>(token) * K + lane] = ex / sum;
+        topk_w[static_cast<size_t>(token) * K + lane] = w;
         atomicAdd(&counts[my_i], 1);
     }
 }
 
 // NV = logits per lane = ceil(E / 32), so the selection loops run exactly as far as E needs.
-__device__ __forceinline__ void select_topk_warp(const float* lg, const float* add_bias, int E,
-                                                 int K, int token, int lane, int32_t* topk_idx,
-                                                 float* topk_w, int32_t* counts) {
-    const int nv = (E + 31) / 32;
-    if (nv <= 1) select_topk_nv<1>(lg, add_bias, E, K, token, lane, topk_idx, topk_w, counts);
-    else if (nv <= 2) select_topk_nv<2>(lg, add_bias, E, K, token, lane, topk_idx, topk_w, counts);
-    else if (nv <= 4) select_topk_nv<4>(lg, add_bias, E, K, token, lane, topk_idx, topk_w, counts);
-    else if (nv <= 8) select_topk_nv<8>(lg, add_bias, E, K, token, lane, topk_idx, topk_w, counts);
-    else select_topk_nv<16>(lg, add_bias, E, K, token, lane, topk_idx, topk_w, counts);
+__device__ __forceinline__ void select_topk_warp(const float* lg, const float* add_bias,
+                                                 const RouterLaunch& a, int token, int lane) {
+    const int nv = (a.E + 31) / 32;
+#define MOE_SELECT(N)                                                                     \
+    select_topk_nv<N>(lg, add_bias, a.E, a.K, token, lane, a.topk_idx, a.topk_w, a.counts, \
+                      a.score_mode, a.select_bias, a.bf16_weights)
+    if (nv <= 1) MOE_SELECT(1);
+    else if (nv <= 2) MOE_SELECT(2);
+    else if (nv <= 4) MOE_SELECT(4);
+    else if (nv <= 8) MOE_SELECT(8);
+    else MOE_SELECT(16);
+#undef MOE_SELECT
 }
 
 __global__ void __launch_bounds__(kRouterThreads)
@@ -219,7 +272,7 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
     for (int t = warp; t < nt; t += kRouterThreads / 32) {
         const int token = t0 + t;
         const float* lg = a.logits + static_cast<size_t>(token) * (E + 1);
-        select_topk_warp(lg, nullptr, E, a.K, token, lane, a.topk_idx, a.topk_w, a.counts);
+        select_topk_warp(lg, nullptr, a, token, lane);
         if (a.w_shared_gate && lane == 0) {
             const float g = __ldcg(lg + E);
             a.shared_gate[token] = 1.f / (1.f + expf(-g));
@@ -244,8 +297,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_select_kernel(RouterLau
     }
     if (warp >= nt) return;
     const int token = t0 + warp;
-    select_topk_warp(a.logits + static_cast<size_t>(token) * a.E, a.logit_bias, a.E, a.K, token,
-                     lane, a.topk_idx, a.topk_w, a.counts);
+    select_topk_warp(a.logits + static_cast<size_t>(token) * a.E, a.logit_bias, a, token, lane);
     if (a.w_shared_gate) {
         const uint4* xv = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(token) * a.D);
         const uint4* wv = reinterpret_cast<const uint4*>(a.w_shared_gate);
