@@ -148,6 +148,9 @@ def test_permute_flags_inconsistent_counts(moe):
     ("uniform", 64, 2048, 256, 8, 512),        # 2 rows per expert (the pages' uniform case)
     ("concentrated", 64, 2048, 256, 8, 512),   # 64 rows on 8 experts
     ("one_hot_expert", 300, 256, 16, 4, 128),  # one expert with every token
+    # 200 rows on expert 0, ~29 on the others: fewer 128-row tiles than SMs, so the
+    # weights-on-M kernel narrows its tiles, with a tall and short tiles in one launch
+    ("one_hot_expert", 200, 256, 8, 2, 128),
     ("random", 1, 256, 8, 3, 256),
     ("random", 777, 512, 12, 3, 384),          # ragged groups, several row blocks
 ])

@@ -126,7 +126,8 @@ struct GroupedGemmLaunch {
     // gate_up only: when gather_tok != NULL, act is the token matrix x [T, D] and row r of
     // the expert-ordered problem is x[gather_tok[r]] (gathered inside the kernel)
     const int32_t* gather_tok;
-    int block_rows;   // rows per tile (16/32/64/128); 0 picks from the average group size
+    int block_rows;   // weights on M: largest rows per tile (16..128); 0: from max_group_rows
+    int max_group_rows;  // rows the largest group can have (T for routed experts); 0: rows
     int orientation;  // 0: auto; 1: weights on M; 2: tokens on M (one CTA); 3: CTA pairs
     // down with acc_out: when final_out and done are set, the kernel converts acc_out
     // [final_rows, D] to bf16 in final_out after all its CTAs finished (done = 0 at launch)

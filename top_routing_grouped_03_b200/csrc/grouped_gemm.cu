@@ -148,8 +148,17 @@ __device__ __forceinline__ bool epilogue_bar_and(bool v) {
 }
 
 struct Tile {
-    int g, i, row0, row_end;
+    int g, i, row0, row_end, bn;
 };
+
+// Rows per tile of a group of n rows under a cap (weights-on-M kernel): the next power of
+// two of n between 16 and the cap, so a hot expert is covered by few wide tiles and a
+// cold one by a single narrow tile.
+__device__ __forceinline__ int group_block_rows(int n, int cap) {
+    int b = 16;
+    while (b < n && b < cap) b <<= 1;
+    return b;
+}
 
 __device__ __forceinline__ Tile decode_tile(int tile, const int* g_tile, const int* g_off, int G,
                                             int BN) {
@@ -166,6 +175,28 @@ __device__ __forceinline__ Tile decode_tile(int tile, const int* g_tile, const i
     t.i = local / nb;
     const int j = local - t.i * nb;
     t.row0 = g_off[lo] + j * BN;
+    t.row_end = g_off[lo + 1];
+    t.bn = BN;
+    return t;
+}
+
+// decode_tile for per-group tile heights (group_block_rows under `cap`)
+__device__ __forceinline__ Tile decode_tile_adaptive(int tile, const int* g_tile, const int* g_off,
+                                                     int G, int cap) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (g_tile[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    Tile t;
+    t.g = lo;
+    const int n = g_off[lo + 1] - g_off[lo];
+    t.bn = group_block_rows(n, cap);
+    const int nb = (n + t.bn - 1) / t.bn;
+    const int local = tile - g_tile[lo];
+    t.i = local / nb;
+    const int j = local - t.i * nb;
+    t.row0 = g_off[lo] + j * t.bn;
     t.row_end = g_off[lo + 1];
     return t;
 }
@@ -204,6 +235,53 @@ __device__ __forceinline__ void build_tile_table(const Params& p, int rows_per_t
     }
 }
 
+// The group table with per-group tile heights: the cap starts at bn_max and is halved
+// while the groups would give fewer tiles than the grid has CTAs (so a few hot groups
+// still spread over the GPU); the cap chosen is stored in *cap_slot.
+__device__ __forceinline__ void build_tile_table_adaptive(const Params& p, int bn_max,
+                                                          int* g_off, int* g_tile, int* total_slot,
+                                                          int* cap_slot, int warp, int lane) {
+    for (int i = threadIdx.x; i <= p.G; i += blockDim.x)
+        g_off[i] = p.offsets ? p.offsets[i] : (i == 0 ? 0 : p.rows_total);
+    __syncthreads();
+    if (warp == 2) {
+        const int per = (p.G + 31) / 32;
+        const int gb = min(lane * per, p.G), ge = min(gb + per, p.G);
+        auto tiles_of = [&](int g, int cap) {
+            const int n = g_off[g + 1] - g_off[g];
+            const int b = group_block_rows(n, cap);
+            return ((n + b - 1) / b) * p.nf;
+        };
+        int cap = bn_max;
+        while (cap > 16) {
+            int local = 0;
+            for (int g = gb; g < ge; ++g) local += tiles_of(g, cap);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
+            if (local >= static_cast<int>(gridDim.x)) break;
+            cap >>= 1;
+        }
+        int local = 0;
+        for (int g = gb; g < ge; ++g) local += tiles_of(g, cap);
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - local;
+        for (int g = gb; g < ge; ++g) {
+            g_tile[g] = run;
+            run += tiles_of(g, cap);
+        }
+        if (lane == 31) {
+            g_tile[p.G] = incl;
+            *total_slot = incl;
+            *cap_slot = cap;
+        }
+    }
+}
+
 // Per-lane plan for gathering ROWS token rows of x into a 128-byte-swizzled operand tile
 // with cp.async: lane l owns 16-byte chunk c = l % 8 of tile rows l/8 + 4u; that chunk of
 // tile row r lands at r*128 + ((c ^ (r % 8)) * 16).
@@ -226,15 +304,18 @@ struct RowGather {
         }
     }
 
-    // copies columns [k0, k0 + 64) of the planned rows into the tile at smem_tile
-    __device__ __forceinline__ void issue(uint32_t smem_tile, const bf16* x, int k0,
-                                          int lane) const {
+    // copies columns [k0, k0 + 64) of the planned rows [0, nrows) into the tile at
+    // smem_tile (rows past the group or past nrows are zero-filled)
+    __device__ __forceinline__ void issue(uint32_t smem_tile, const bf16* x, int k0, int lane,
+                                          int nrows = ROWS) const {
         const int c = lane & 7;
 #pragma unroll
         for (int u = 0; u < kChunks; ++u) {
+            // branch-free: rows past the group or past nrows get a zero fill (no global read)
             const int r = (lane >> 3) + 4 * u;
+            const bool live = ((valid >> u) & 1u) && r < nrows;
             cp_async_16(smem_tile + r * 128 + ((c ^ (r & 7)) << 4), x + src_off[u] + k0,
-                        ((valid >> u) & 1u) ? 16u : 0u);
+                        live ? 16u : 0u);
         }
     }
 };
@@ -244,6 +325,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                     const __grid_constant__ CUtensorMap map_act, Params p) {
     using C = Cfg<BN, GATE_UP>;
+    // 16-row tiles are the narrowest: per-group heights only pay above them
+    constexpr bool kAdapt = BN > 16;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -255,8 +338,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* total_slot = reinterpret_cast<int*>(tmem_slot + 2);
+    int* cap_slot = reinterpret_cast<int*>(tmem_slot + 3);
     int* g_off = reinterpret_cast<int*>(tmem_slot + 4);
     int* g_tile = g_off + (p.G + 1);
+    int* stage_bn = g_tile + (p.G + 1);  // [kStages] rows of the tile each stage belongs to
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -288,19 +373,27 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
     // and the accumulator are produced by earlier kernels of the stream
     grid_dep_wait();
     grid_dep_launch();
-    build_tile_table(p, BN, g_off, g_tile, total_slot, warp, lane);
+    if constexpr (kAdapt)
+        build_tile_table_adaptive(p, BN, g_off, g_tile, total_slot, cap_slot, warp, lane);
+    else
+        build_tile_table(p, BN, g_off, g_tile, total_slot, warp, lane);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int total = *total_slot;
+    const int cap = kAdapt ? *cap_slot : BN;
+    auto tile_at = [&](int tile) {
+        if constexpr (kAdapt) return decode_tile_adaptive(tile, g_tile, g_off, p.G, cap);
+        else return decode_tile(tile, g_tile, g_off, p.G, BN);
+    };
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
-        // Weights (operand A) always by TMA from lane 0.  Activation rows (operand B): one
-        // TMA box when they are contiguous in expert order; otherwise (gather) each lane
-        // copies 16-byte chunks of x[gather_tok[row]] with cp.async into the swizzled tile
-        // (RowGather).
+        // Weights (operand A) always by TMA from lane 0.  Activation rows (operand B, the
+        // tile's bn rows): 16-row TMA boxes when they are contiguous in expert order;
+        // otherwise (gather) each lane copies 16-byte chunks of x[gather_tok[row]] with
+        // cp.async into the swizzled tile (RowGather).
         if (gather || lane == 0) {
             const uint64_t pol_w = policy_evict_first();  // weights stream through once
             const uint64_t pol_a = policy_evict_last();   // activations are re-read
@@ -309,8 +402,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
             uint32_t phase = 0, filled = 0, fill_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const Tile t = decode_tile(tile, g_tile, g_off, p.G, BN);
+                const Tile t = tile_at(tile);
                 const int wr0 = t.g * p.w_group_rows + t.i * kBM;
+                const uint32_t stage_bytes = a_bytes + t.bn * kBK * 2;
                 RowGather<BN> rg;
                 if (gather) rg.plan(p.gather_tok, t.row0, t.row_end, p.nk * kBK, lane);
                 for (int kk = 0; kk < p.nk; ++kk) {
@@ -324,17 +418,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                     }
                     uint8_t* st = smem + stage * C::kStageBytes;
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(&full[stage], gather ? a_bytes : C::kStageBytes);
+                        stage_bn[stage] = t.bn;  // published by the arrive below
+                        mbar_arrive_expect_tx(&full[stage], gather ? a_bytes : stage_bytes);
                         tma_load_2d(st, &map_w, &full[stage], kk * kBK, wr0, pol_w);
                         if (GATE_UP)
                             tma_load_2d(st + C::kABytes, &map_w, &full[stage], kk * kBK,
                                         wr0 + p.up_rows, pol_w);
                         if (!gather)
-                            tma_load_2d(st + a_bytes, &map_act, &full[stage], kk * kBK, t.row0,
-                                        pol_a);
+                            for (int b = 0; b < t.bn; b += 16)
+                                tma_load_2d(st + a_bytes + b * kBK * 2, &map_act, &full[stage],
+                                            kk * kBK, t.row0 + b, pol_a);
                     }
                     if (gather) {
-                        rg.issue(smem_u32(st + a_bytes), p.x, kk * kBK, lane);
+                        rg.issue(smem_u32(st + a_bytes), p.x, kk * kBK, lane, t.bn);
                         cp_async_mbar_arrive_noinc(&full[stage]);
                     }
                     filled |= 1u << stage;
@@ -353,7 +449,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
             int stage = 0;
             uint32_t phase = 0, abuf = 0, aphase = 0;
             bool ok = true, issued = false;
@@ -366,6 +461,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                 }
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + abuf * C::kAccCols;
+                uint32_t idesc = idesc_bf16_f32(kBM, BN);
                 for (int kk = 0; kk < p.nk; ++kk) {
                     if (!mbar_wait(&full[stage], phase, kWaitBudgetNs, abort_flag)) {
                         set_status(p.status, MOE_ERR_TIMEOUT);
@@ -375,6 +471,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                     }
                     tc_fence_after();
                     if (gather) fence_proxy_async_smem();
+                    if (kAdapt && kk == 0)
+                        idesc = idesc_bf16_f32(kBM, stage_bn[stage]);  // N = this tile's rows
                     const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
                     const uint32_t a1 = a0 + C::kABytes;
                     const uint32_t b0 = a0 + C::kNumA * C::kABytes;
@@ -406,7 +504,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
         const int feat_in_tile = q * 32 + lane;
         uint32_t abuf = 0, aphase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const Tile t = decode_tile(tile, g_tile, g_off, p.G, BN);
+            const Tile t = tile_at(tile);
             const bool ready = mbar_wait(&tfull[abuf], aphase, kWaitBudgetNs, abort_flag);
             if (!epilogue_bar_and(ready)) {
                 set_status(p.status, MOE_ERR_TIMEOUT);
@@ -418,7 +516,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                                    abuf * C::kAccCols;
             const int feat = t.i * kBM + feat_in_tile;
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 16) {
+            for (int c0 = 0; c0 < (kAdapt ? t.bn : BN); c0 += 16) {
                 uint32_t gv[16];
                 uint32_t uv[16];
                 tmem_ld16(tbase + c0, gv);
@@ -970,7 +1068,8 @@ cudaError_t launch_tpl(const CUtensorMap& mw, const CUtensorMap& ma, const Param
                        cudaStream_t s, bool pdl) {
     using C = Cfg<BN, GATE_UP>;
     const size_t smem = 1024 + static_cast<size_t>(C::kStages) * C::kStageBytes +
-                        (2 * C::kStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int);
+                        (2 * C::kStages + 5) * 8 + 16 +
+                        (2 * (p.G + 1) + C::kStages) * sizeof(int);
     auto kfn = grouped_gemm_kernel<BN, GATE_UP>;
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
@@ -1050,7 +1149,12 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
     const bool gathered = a.gate_up && a.gather_tok != nullptr;
     const bool pairs = tm && a.orientation != 2 && (!gathered || a.gather_buf != nullptr) &&
                        num_sms >= 2;
-    const int BN = tm ? kTmRows : (a.block_rows ? a.block_rows : pick_block_rows(a.rows, a.E));
+    // weights on M: tiles adapt per group up to BN, sized for groups up to 8x the average
+    // (skewed routing) but never past the largest possible group
+    const int max_rows = a.max_group_rows > 0 ? a.max_group_rows : a.rows;
+    const long long avg8 = 8ll * a.rows / (a.E > 0 ? a.E : 1);
+    const int bn_rows = static_cast<int>(std::min<long long>(max_rows, std::max(avg8, 16ll)));
+    const int BN = tm ? kTmRows : (a.block_rows ? a.block_rows : pick_block_rows(bn_rows, 1));
     if (BN != 16 && BN != 32 && BN != 64 && BN != 128) return cudaErrorInvalidValue;
     const int K = a.gate_up ? a.D : a.f;
     const uint64_t w_group_rows = a.gate_up ? 2ull * a.f : static_cast<uint64_t>(a.D);
@@ -1067,7 +1171,9 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
         act = a.gather_buf;
         gather = false;
     }
-    if ((err = make_map(&ma, act, gather ? 1 : a.rows, K, gather ? 1 : BN)) != cudaSuccess)
+    // activation boxes: 128 rows (tokens on M) or 16 rows (weights on M, bn/16 per stage)
+    if ((err = make_map(&ma, act, gather ? 1 : a.rows, K, gather ? 1 : (tm ? kTmRows : 16))) !=
+        cudaSuccess)
         return err;
     Params p{};
     p.offsets = a.offsets;
@@ -1090,7 +1196,8 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
     p.final_rows = a.final_rows;
     p.done = a.done;
     p.final_residual = a.final_residual;
-    const long long max_tiles = (static_cast<long long>(ceil_div(a.rows, BN)) + a.E) * p.nf;
+    const long long max_tiles =
+        (static_cast<long long>(ceil_div(a.rows, tm ? BN : 16)) + a.E) * p.nf;
     const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
     if (pairs) {
         const long long pair_tiles =

@@ -344,6 +344,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     up.gather_buf = at<bf16>(workspace, L.x_sorted);
     up.offsets = pm.offsets;
     up.rows = rows; up.E = E; up.D = D; up.f = f;
+    up.max_group_rows = T;
     up.h_out = at<bf16>(workspace, L.h);
     up.status = status;
     if (!mark(MOE_EV_GATE_UP) || launch_grouped_gemm(up, sms, s, true) != cudaSuccess)
@@ -357,6 +358,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     dn.sorted_token = pm.sorted_token;
     dn.sorted_w = det ? nullptr : pm.sorted_w;
     dn.rows = rows; dn.E = E; dn.D = D; dn.f = f;
+    dn.max_group_rows = T;
     dn.acc_out = det ? nullptr : out_acc;
     dn.y_out = det ? at<float>(workspace, L.y_sorted) : nullptr;
     dn.status = status;
