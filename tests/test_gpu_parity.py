@@ -113,7 +113,12 @@ def test_route_shapes(moe, oracle_mod, T, D, E, K):
 @pytest.mark.parametrize("kind,T,E,K", [("uniform", 64, 256, 8), ("concentrated", 64, 256, 8),
                                         ("one_hot_expert", 300, 16, 4), ("random", 1, 8, 3),
                                         ("random", 517, 128, 8), ("random", 4096, 512, 10),
-                                        ("random", 3000, 4, 4)])
+                                        ("random", 3000, 4, 4),
+                                        # several chunks: hot experts, 256 chunks of a length
+                                        # that is not a multiple of 1024
+                                        ("concentrated", 2048, 256, 8),
+                                        ("one_hot_expert", 9000, 64, 6),
+                                        ("random", 70001, 64, 4)])
 def test_permute_bitexact(moe, oracle_mod, kind, T, E, K):
     idx = (random_routing(T, E, K, seed=T) if kind == "random"
            else crafted_routing(T, E, K, kind)).numpy()
@@ -138,6 +143,19 @@ def test_permute_flags_inconsistent_counts(moe):
     ws = moe.alloc_workspace(2, 128, 4, 2, 128)
     ws.zero_()
     moe.permute(idx, None, bad_counts, 4, workspace=ws)
+    assert moe.read_device_status(ws) == -7  # MOE_ERR_DEVICE
+
+
+@pytest.mark.parametrize("delta", [-1, 1])
+def test_permute_flags_inconsistent_counts_chunked(moe, delta):
+    T, E, K = 3000, 8, 4   # 12000 entries: several chunks
+    idx = random_routing(T, E, K, seed=5)
+    counts = np.bincount(idx.numpy().reshape(-1), minlength=E).astype(np.int32)
+    counts[3] += delta
+    counts[5] -= delta        # the total stays right, two groups do not
+    ws = moe.alloc_workspace(T, 128, E, K, 128)
+    ws.zero_()
+    moe.permute(idx.cuda(), None, torch.as_tensor(counts).cuda(), E, workspace=ws)
     assert moe.read_device_status(ws) == -7  # MOE_ERR_DEVICE
 
 

@@ -126,7 +126,9 @@ def alloc_workspace(T, D, E, K, f, f_s=0, device=None) -> torch.Tensor:
     n = workspace_size(T, D, E, K, f, f_s)
     if n == 0:
         raise MoEError(-2, "moe_workspace_size")
-    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    ws = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    ws[:256].zero_()  # the device status word starts clear
+    return ws
 
 
 def route(x, w_router, K, logit_bias=None, w_shared_gate=None, workspace=None, stream=None,
@@ -180,6 +182,8 @@ def permute(topk_idx, topk_w, expert_counts, E, workspace=None, stream=None):
     st = torch.empty((T * K,), dtype=torch.int32, device=dev)
     sw = torch.empty((T * K,), dtype=torch.float32, device=dev) if topk_w is not None else None
     s2r = torch.empty((T * K,), dtype=torch.int32, device=dev)
+    if workspace is None and T > 0:
+        workspace = alloc_workspace(T, 128, E, K, 128, 0, dev)
     rc = lib().moe_permute(_p(topk_idx), _p(topk_w), _p(expert_counts), T, E, K, _p(off),
                            _p(st), _p(sw), _p(s2r), _p(workspace), _stream(stream))
     _check(rc, "moe_permute")

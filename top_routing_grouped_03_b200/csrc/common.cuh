@@ -107,7 +107,10 @@ struct PermuteLaunch {
     int32_t* slot_to_row;
     int32_t* dense_offsets;  // optional [2] = {0, T} for a dense (shared) expert group
     int* status;
+    int32_t* hist;           // [permute_chunks(T*K) * E] scratch, or NULL (one CTA)
 };
+// chunks the permutation cuts T*K entries into (1 at decode sizes, at most 256)
+int permute_chunks(long long entries);
 cudaError_t launch_permute(const PermuteLaunch& a, cudaStream_t s, bool pdl = false);
 
 

@@ -35,7 +35,7 @@ int num_sms_current() {
 
 // Workspace of the whole layer.  The status word is always at offset 0.
 struct Layout {
-    size_t status, counters, counts, logits, offsets, dense_offsets, topk_idx, topk_w, sgate,
+    size_t status, counters, counts, perm_hist, logits, offsets, dense_offsets, topk_idx, topk_w, sgate,
         sorted_token, sorted_w, slot_to_row, x_sorted, h, h_s, out_acc, y_sorted, total;
     size_t zero_end;  // [0, zero_end) is cleared at the start of a layer call
 };
@@ -52,6 +52,8 @@ Layout layout(long long T, long long D, long long E, long long K, long long f, l
     L.counters = take(sizeof(unsigned) * static_cast<size_t>((T + 7) / 8));
     L.counts = take(sizeof(int32_t) * E);
     L.zero_end = o;
+    // depends on T, E and K only, so any workspace sized for the same T, E, K has it here
+    L.perm_hist = take(sizeof(int32_t) * E * permute_chunks(T * K));
     L.logits = take(sizeof(float) * T * (E + 1));
     L.offsets = take(sizeof(int32_t) * (E + 1));
     L.dense_offsets = take(sizeof(int32_t) * 2);
@@ -184,6 +186,7 @@ int moe_permute(const int32_t* topk_idx, const float* topk_w, const int32_t* exp
     a.sorted_w = sorted_w;
     a.slot_to_row = slot_to_row;
     a.status = workspace ? at<int>(workspace, 0) : nullptr;
+    a.hist = workspace ? at<int32_t>(workspace, layout(T, 128, E, K, 128, 0).perm_hist) : nullptr;
     return launch_permute(a, as_stream(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -333,6 +336,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     pm.slot_to_row = at<int32_t>(workspace, L.slot_to_row);
     pm.dense_offsets = at<int32_t>(workspace, L.dense_offsets);
     pm.status = status;
+    pm.hist = at<int32_t>(workspace, L.perm_hist);
     if (!mark(MOE_EV_PERMUTE) || launch_permute(pm, s, true) != cudaSuccess) return MOE_ERR_CUDA;
 
     const int rows = T * K;

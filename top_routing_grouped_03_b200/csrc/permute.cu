@@ -5,11 +5,13 @@
 // "1.6 混合专家（MoE）", section 2: tokens are first grouped by route, computed per
 // expert, then merged back in their original order.
 //
-// permute_kernel: one CTA per expert e.
-//   offsets[e] = sum_{e' < e} counts[e']            (block reduction over <= 512 counts)
-//   a block-wide ballot scan walks the T*K routing entries in order and writes the
-//   entries equal to e to rows offsets[e] + rank  -> ascending token order (stable).
-// permute_small_kernel: the same result from one CTA when T*K <= 4096 (decode sizes).
+// The (token, slot) entries are cut into chunks of consecutive entries.  With one chunk a
+// single CTA does everything; otherwise permute_hist_kernel counts each chunk's entries per
+// expert and permute_scatter_kernel gives every entry its row:
+//   row = offsets[e] + (entries of e in earlier chunks) + (entries of e earlier in this
+//         chunk),
+// offsets being the exclusive scan of the counts -- ascending (token, slot) order inside
+// each group, i.e. a stable counting sort by expert.
 // The token rows themselves are never copied: the grouped GEMM gathers them from x.
 #include <algorithm>
 
@@ -18,109 +20,65 @@
 namespace moe {
 namespace {
 
-constexpr int kPermThreads = 512;
+constexpr int kPermThreads = 1024;
+constexpr int kPermWarps = kPermThreads / 32;
+constexpr int kSingleChunk = 4096;  // entries one CTA takes alone (decode sizes)
+constexpr int kMaxChunks = 256;
 
-__global__ void __launch_bounds__(kPermThreads) permute_kernel(PermuteLaunch a) {
-    __shared__ int warp_tot[kPermThreads / 32];
-    __shared__ int warp_pre[kPermThreads / 32];
-    __shared__ int s_off;
-    __shared__ int s_block_hits;
-    const int e = blockIdx.x;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int total = a.T * a.K;
-
-    grid_dep_wait();  // routing and counts come from the router
-    grid_dep_launch();
-
-    int v = 0;
-    for (int i = tid; i < e; i += kPermThreads) v += a.counts[i];
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    if (lane == 0) warp_tot[warp] = v;
-    __syncthreads();
-    if (tid == 0) {
-        int s = 0;
-        for (int w = 0; w < kPermThreads / 32; ++w) s += warp_tot[w];
-        s_off = s;
-    }
-    __syncthreads();
-    const int off = s_off;
-    const int n_e = a.counts[e];
-    if (tid == 0) {
-        a.offsets[e] = off;
-        if (e == a.E - 1) {
-            a.offsets[a.E] = off + n_e;
-            if (off + n_e != total) set_status(a.status, MOE_ERR_DEVICE);
-        }
-        if (e == 0 && a.dense_offsets) {
-            a.dense_offsets[0] = 0;
-            a.dense_offsets[1] = a.T;
-        }
-    }
-    if (n_e == 0) return;
-
-    const unsigned lt_mask = (1u << lane) - 1u;
-    int base = 0;
-    for (int j0 = 0; j0 < total; j0 += kPermThreads) {
-        const int j = j0 + tid;
-        const bool hit = (j < total) && (__ldg(a.topk_idx + j) == e);
-        const unsigned b = __ballot_sync(0xffffffffu, hit);
-        if (lane == 0) warp_tot[warp] = __popc(b);
-        __syncthreads();
-        if (warp == 0) {
-            const int c = (lane < kPermThreads / 32) ? warp_tot[lane] : 0;
-            int incl = c;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += n;
-            }
-            if (lane < kPermThreads / 32) warp_pre[lane] = incl - c;
-            if (lane == kPermThreads / 32 - 1) s_block_hits = incl;
-        }
-        __syncthreads();
-        if (hit) {
-            const int r = base + warp_pre[warp] + __popc(b & lt_mask);
-            if (r < n_e) {
-                const int row = off + r;
-                a.sorted_token[row] = j / a.K;
-                if (a.topk_w) a.sorted_w[row] = __ldg(a.topk_w + j);
-                a.slot_to_row[j] = row;
-            }
-        }
-        base += s_block_hits;
-        __syncthreads();
-    }
-    if (tid == 0 && base != n_e) set_status(a.status, MOE_ERR_DEVICE);
-
+// [c*chunk_len, min(total, (c+1)*chunk_len)): the entries of chunk c
+struct ChunkRange {
+    int begin, end;
+};
+__device__ __forceinline__ ChunkRange chunk_range(int c, int chunk_len, int total) {
+    const long long b = static_cast<long long>(c) * chunk_len;
+    const long long e = b + chunk_len;
+    return {static_cast<int>(b < total ? b : total), static_cast<int>(e < total ? e : total)};
 }
 
+// hist[c * E + e] = entries of chunk c routed to expert e
+__global__ void __launch_bounds__(kPermThreads) permute_hist_kernel(PermuteLaunch a,
+                                                                    int chunk_len) {
+    extern __shared__ int cnt[];  // [E]
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int E = a.E;
+    grid_dep_wait();  // routing comes from the router
+    grid_dep_launch();
+    for (int e = tid; e < E; e += kPermThreads) cnt[e] = 0;
+    __syncthreads();
+    const ChunkRange r = chunk_range(blockIdx.x, chunk_len, a.T * a.K);
+    for (int j0 = r.begin; j0 < r.end; j0 += kPermThreads) {
+        const int j = j0 + tid;
+        const int e = j < r.end ? __ldg(a.topk_idx + j) : -1;
+        const bool ok = e >= 0 && e < E;
+        const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
+        if (ok && (peers & ((1u << lane) - 1u)) == 0) atomicAdd(&cnt[e], __popc(peers));
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kPermThreads)
+        a.hist[static_cast<size_t>(blockIdx.x) * E + e] = cnt[e];
+}
 
-// Small problems (T*K <= kSmallEntries): one CTA of 1024 threads does the whole
-// permutation.  offsets = exclusive scan of the counts; then the entries are walked in
-// chunks of 1024 in order, and an entry's row is offsets[e] + (entries of e in earlier
-// chunks) + (entries of e in earlier warps of this chunk) + (its rank among the lanes of
-// its warp holding e, from __match_any_sync) -- ascending token order, as the
-// one-CTA-per-expert kernel gives.
-constexpr int kSmallEntries = 4096;
-constexpr int kSmallThreads = 1024;
-constexpr int kSmallWarps = kSmallThreads / 32;
-
-__global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(PermuteLaunch a) {
+// Rows of chunk blockIdx.x.  Inside a chunk, 1024 entries at a time: an entry's row is
+// offsets[e] + base[e] (entries of e before this step) + (entries of e in earlier warps of
+// this step) + (its rank among the lanes of its warp holding e, from __match_any_sync).
+__global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(PermuteLaunch a,
+                                                                       int chunk_len,
+                                                                       int chunks) {
     extern __shared__ int sm[];
-    int* warp_cnt = sm;                          // [kSmallWarps][E]
-    int* base = warp_cnt + kSmallWarps * a.E;    // [E] rows of e placed so far
+    int* warp_cnt = sm;                          // [kPermWarps][E]
+    int* base = warp_cnt + kPermWarps * a.E;     // [E] entries of e placed before this step
     int* off = base + a.E;                       // [E + 1]
-    __shared__ int warp_sums[kSmallWarps];
+    __shared__ int warp_sums[kPermWarps];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int E = a.E, total = a.T * a.K;
+    const int c = blockIdx.x;
 
-    grid_dep_wait();
+    grid_dep_wait();  // counts (router) and chunk histograms (previous kernel)
     grid_dep_launch();
 
-    // offsets: exclusive scan of counts (E <= 512 < kSmallThreads)
-    const int c = tid < E ? a.counts[tid] : 0;
-    int incl = c;
+    // offsets: exclusive scan of counts (E <= 512 < kPermThreads)
+    const int n = tid < E ? a.counts[tid] : 0;
+    int incl = n;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -129,35 +87,44 @@ __global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(PermuteLau
     if (lane == 31) warp_sums[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        const int s = warp_sums[lane];
-        int ws = s;
+        const int sw = warp_sums[lane];
+        int ws = sw;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int v = __shfl_up_sync(0xffffffffu, ws, o);
             if (lane >= o) ws += v;
         }
-        warp_sums[lane] = ws - s;  // exclusive prefix of the warps
+        warp_sums[lane] = ws - sw;  // exclusive prefix of the warps
     }
     __syncthreads();
     if (tid < E) {
-        off[tid] = warp_sums[warp] + incl - c;
+        off[tid] = warp_sums[warp] + incl - n;
         base[tid] = 0;
-        a.offsets[tid] = off[tid];
+        if (c == 0) a.offsets[tid] = off[tid];
     }
     if (tid == 0) {
         off[E] = total;
-        a.offsets[E] = total;
-        if (a.dense_offsets) {
-            a.dense_offsets[0] = 0;
-            a.dense_offsets[1] = a.T;
+        if (c == 0) {
+            a.offsets[E] = total;
+            if (a.dense_offsets) {
+                a.dense_offsets[0] = 0;
+                a.dense_offsets[1] = a.T;
+            }
         }
     }
+    __syncthreads();
+    // entries of each expert in the chunks before this one
+    for (int i = tid; i < c * E; i += kPermThreads) {
+        const int v = a.hist[i];
+        if (v) atomicAdd(&base[i % E], v);
+    }
+    const ChunkRange r = chunk_range(c, chunk_len, total);
     const unsigned lt = (1u << lane) - 1u;
-    for (int j0 = 0; j0 < total; j0 += kSmallThreads) {
-        for (int i = tid; i < kSmallWarps * E; i += kSmallThreads) warp_cnt[i] = 0;
+    for (int j0 = r.begin; j0 < r.end; j0 += kPermThreads) {
+        for (int i = tid; i < kPermWarps * E; i += kPermThreads) warp_cnt[i] = 0;
         __syncthreads();
         const int j = j0 + tid;
-        const bool live = j < total;
+        const bool live = j < r.end;
         const int e = live ? __ldg(a.topk_idx + j) : -1;
         const bool ok = live && e >= 0 && e < E;
         const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
@@ -165,9 +132,9 @@ __global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(PermuteLau
         if (ok && rank == 0) warp_cnt[warp * E + e] = __popc(peers);
         if (live && !ok) set_status(a.status, MOE_ERR_DEVICE);
         __syncthreads();
-        if (tid < E) {  // prefix over the warps of this chunk, per expert
+        if (tid < E) {  // prefix over the warps of this step, per expert
             int run = base[tid];
-            for (int w = 0; w < kSmallWarps; ++w) {
+            for (int w = 0; w < kPermWarps; ++w) {
                 const int v = warp_cnt[w * E + tid];
                 warp_cnt[w * E + tid] = run;
                 run += v;
@@ -177,7 +144,9 @@ __global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(PermuteLau
         __syncthreads();
         if (ok) {
             const int row = off[e] + warp_cnt[warp * E + e] + rank;
-            if (row < off[e + 1]) {
+            // counts that disagree with the entries can push a row out of its group, or
+            // (when they do not sum to T*K) out of the arrays: flag it, write nothing
+            if (row >= 0 && row < off[e + 1] && row < total) {
                 a.sorted_token[row] = j / a.K;
                 if (a.topk_w) a.sorted_w[row] = __ldg(a.topk_w + j);
                 a.slot_to_row[j] = row;
@@ -187,7 +156,9 @@ __global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(PermuteLau
         }
         __syncthreads();
     }
-    if (tid < E && base[tid] != off[tid + 1] - off[tid]) set_status(a.status, MOE_ERR_DEVICE);
+    // the last chunk has seen every entry: each group must be exactly full
+    if (c == chunks - 1 && tid < E && base[tid] != off[tid + 1] - off[tid])
+        set_status(a.status, MOE_ERR_DEVICE);
 }
 
 
@@ -210,18 +181,31 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const bf16* x, const i
 
 }  // namespace
 
+int permute_chunks(long long entries) {
+    if (entries <= kSingleChunk) return 1;
+    const long long want = std::min<long long>(kMaxChunks, (entries + kPermThreads - 1) / kPermThreads);
+    const long long len = (entries + want - 1) / want;
+    return static_cast<int>((entries + len - 1) / len);
+}
+
 cudaError_t launch_permute(const PermuteLaunch& a, cudaStream_t s, bool pdl) {
+    const long long entries = static_cast<long long>(a.T) * a.K;
+    // without a histogram buffer one CTA walks every entry
+    const int chunks = a.hist ? permute_chunks(entries) : 1;
+    const int chunk_len = static_cast<int>(chunks > 1 ? (entries + chunks - 1) / chunks : entries);
     cudaError_t err;
-    if (static_cast<long long>(a.T) * a.K <= kSmallEntries) {
-        const size_t smem = sizeof(int) * (static_cast<size_t>(kSmallWarps) * a.E + 2 * a.E + 1);
-        err = cudaFuncSetAttribute(permute_small_kernel,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   static_cast<int>(smem));
+    if (chunks > 1) {
+        err = launch_kernel(permute_hist_kernel, dim3(chunks), dim3(kPermThreads),
+                            sizeof(int) * static_cast<size_t>(a.E), s, pdl, a, chunk_len);
+        count_launches(1);
         if (err != cudaSuccess) return err;
-        err = launch_kernel(permute_small_kernel, dim3(1), dim3(kSmallThreads), smem, s, pdl, a);
-    } else {
-        err = launch_kernel(permute_kernel, dim3(a.E), dim3(kPermThreads), 0, s, pdl, a);
     }
+    const size_t smem = sizeof(int) * (static_cast<size_t>(kPermWarps) * a.E + 2 * a.E + 1);
+    err = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    err = launch_kernel(permute_scatter_kernel, dim3(chunks), dim3(kPermThreads), smem, s,
+                        pdl || chunks > 1, a, chunk_len, chunks);
     count_launches(1);
     return err;
 }
