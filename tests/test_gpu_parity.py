@@ -47,6 +47,9 @@ SMALL_LAYERS = {
     "dense_E1": LayerConfig("dense_E1", T=33, D=256, E=1, K=1, f=384, seed=5),
     "all_experts": LayerConfig("all_experts", T=50, D=256, E=8, K=8, f=128, seed=6),
     "hot_rows": LayerConfig("hot_rows", T=300, D=256, E=4, K=2, f=128, seed=7),
+    # at most 16 tokens: weights-on-M grouped GEMMs, routed and shared
+    "few_tokens_shared": LayerConfig("few_tokens_shared", T=12, D=256, E=32, K=4, f=256,
+                                     f_s=128, seed=9),
     # T >= 256 and E % 128 == 0: router logits on the tensor cores, shared gate in the
     # selection kernel
     "tc_router_shared": LayerConfig("tc_router_shared", T=300, D=384, E=128, K=6, f=128,
@@ -166,9 +169,10 @@ def test_permute_flags_inconsistent_counts_chunked(moe, delta):
     ("uniform", 64, 2048, 256, 8, 512),        # 2 rows per expert (the pages' uniform case)
     ("concentrated", 64, 2048, 256, 8, 512),   # 64 rows on 8 experts
     ("one_hot_expert", 300, 256, 16, 4, 128),  # one expert with every token
-    # 200 rows on expert 0, ~29 on the others: fewer 128-row tiles than SMs, so the
-    # weights-on-M kernel narrows its tiles, with a tall and short tiles in one launch
-    ("one_hot_expert", 200, 256, 8, 2, 128),
+    ("one_hot_expert", 200, 256, 8, 2, 128),   # one 200-row group, the rest ~29 rows
+    # at most 16 tokens: the weights-on-M orientation (narrow token tiles)
+    ("concentrated", 16, 2048, 256, 8, 512),   # 16 rows on each of 8 experts
+    ("random", 13, 512, 4, 2, 384),            # ragged groups of a few rows
     ("random", 1, 256, 8, 3, 256),
     ("random", 777, 512, 12, 3, 384),          # ragged groups, several row blocks
 ])

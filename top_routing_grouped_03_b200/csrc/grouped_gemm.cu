@@ -85,6 +85,11 @@ struct Params {
     const bf16* final_residual; //   + this bf16 [final_rows, out_cols] when not NULL
 };
 
+// tiles of a group of n rows cut into row blocks of `rows`
+__device__ __forceinline__ int group_tiles(const Params& p, int n, int rows) {
+    return ((n + rows - 1) / rows) * p.nf;
+}
+
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -148,17 +153,8 @@ __device__ __forceinline__ bool epilogue_bar_and(bool v) {
 }
 
 struct Tile {
-    int g, i, row0, row_end, bn;
+    int g, i, row0, row_end;
 };
-
-// Rows per tile of a group of n rows under a cap (weights-on-M kernel): the next power of
-// two of n between 16 and the cap, so a hot expert is covered by few wide tiles and a
-// cold one by a single narrow tile.
-__device__ __forceinline__ int group_block_rows(int n, int cap) {
-    int b = 16;
-    while (b < n && b < cap) b <<= 1;
-    return b;
-}
 
 __device__ __forceinline__ Tile decode_tile(int tile, const int* g_tile, const int* g_off, int G,
                                             int BN) {
@@ -175,28 +171,6 @@ __device__ __forceinline__ Tile decode_tile(int tile, const int* g_tile, const i
     t.i = local / nb;
     const int j = local - t.i * nb;
     t.row0 = g_off[lo] + j * BN;
-    t.row_end = g_off[lo + 1];
-    t.bn = BN;
-    return t;
-}
-
-// decode_tile for per-group tile heights (group_block_rows under `cap`)
-__device__ __forceinline__ Tile decode_tile_adaptive(int tile, const int* g_tile, const int* g_off,
-                                                     int G, int cap) {
-    int lo = 0, hi = G - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (g_tile[mid] <= tile) lo = mid; else hi = mid - 1;
-    }
-    Tile t;
-    t.g = lo;
-    const int n = g_off[lo + 1] - g_off[lo];
-    t.bn = group_block_rows(n, cap);
-    const int nb = (n + t.bn - 1) / t.bn;
-    const int local = tile - g_tile[lo];
-    t.i = local / nb;
-    const int j = local - t.i * nb;
-    t.row0 = g_off[lo] + j * t.bn;
     t.row_end = g_off[lo + 1];
     return t;
 }
@@ -215,8 +189,7 @@ __device__ __forceinline__ void build_tile_table(const Params& p, int rows_per_t
         const int per = (p.G + 31) / 32;
         const int gb = min(lane * per, p.G), ge = min(gb + per, p.G);
         int local = 0;
-        for (int g = gb; g < ge; ++g)
-            local += ((g_off[g + 1] - g_off[g] + rows_per_tile - 1) / rows_per_tile) * p.nf;
+        for (int g = gb; g < ge; ++g) local += group_tiles(p, g_off[g + 1] - g_off[g], rows_per_tile);
         int incl = local;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -226,58 +199,11 @@ __device__ __forceinline__ void build_tile_table(const Params& p, int rows_per_t
         int run = incl - local;
         for (int g = gb; g < ge; ++g) {
             g_tile[g] = run;
-            run += ((g_off[g + 1] - g_off[g] + rows_per_tile - 1) / rows_per_tile) * p.nf;
+            run += group_tiles(p, g_off[g + 1] - g_off[g], rows_per_tile);
         }
         if (lane == 31) {
             g_tile[p.G] = incl;
             *total_slot = incl;
-        }
-    }
-}
-
-// The group table with per-group tile heights: the cap starts at bn_max and is halved
-// while the groups would give fewer tiles than the grid has CTAs (so a few hot groups
-// still spread over the GPU); the cap chosen is stored in *cap_slot.
-__device__ __forceinline__ void build_tile_table_adaptive(const Params& p, int bn_max,
-                                                          int* g_off, int* g_tile, int* total_slot,
-                                                          int* cap_slot, int warp, int lane) {
-    for (int i = threadIdx.x; i <= p.G; i += blockDim.x)
-        g_off[i] = p.offsets ? p.offsets[i] : (i == 0 ? 0 : p.rows_total);
-    __syncthreads();
-    if (warp == 2) {
-        const int per = (p.G + 31) / 32;
-        const int gb = min(lane * per, p.G), ge = min(gb + per, p.G);
-        auto tiles_of = [&](int g, int cap) {
-            const int n = g_off[g + 1] - g_off[g];
-            const int b = group_block_rows(n, cap);
-            return ((n + b - 1) / b) * p.nf;
-        };
-        int cap = bn_max;
-        while (cap > 16) {
-            int local = 0;
-            for (int g = gb; g < ge; ++g) local += tiles_of(g, cap);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
-            if (local >= static_cast<int>(gridDim.x)) break;
-            cap >>= 1;
-        }
-        int local = 0;
-        for (int g = gb; g < ge; ++g) local += tiles_of(g, cap);
-        int incl = local;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        int run = incl - local;
-        for (int g = gb; g < ge; ++g) {
-            g_tile[g] = run;
-            run += tiles_of(g, cap);
-        }
-        if (lane == 31) {
-            g_tile[p.G] = incl;
-            *total_slot = incl;
-            *cap_slot = cap;
         }
     }
 }
@@ -304,16 +230,16 @@ struct RowGather {
         }
     }
 
-    // copies columns [k0, k0 + 64) of the planned rows [0, nrows) into the tile at
-    // smem_tile (rows past the group or past nrows are zero-filled)
-    __device__ __forceinline__ void issue(uint32_t smem_tile, const bf16* x, int k0, int lane,
-                                          int nrows = ROWS) const {
+    // copies columns [k0, k0 + 64) of the planned rows into the tile at smem_tile (rows
+    // past the group are zero-filled)
+    __device__ __forceinline__ void issue(uint32_t smem_tile, const bf16* x, int k0,
+                                          int lane) const {
         const int c = lane & 7;
 #pragma unroll
         for (int u = 0; u < kChunks; ++u) {
-            // branch-free: rows past the group or past nrows get a zero fill (no global read)
+            // branch-free: rows past the group get a zero fill (no global read)
             const int r = (lane >> 3) + 4 * u;
-            const bool live = ((valid >> u) & 1u) && r < nrows;
+            const bool live = (valid >> u) & 1u;
             cp_async_16(smem_tile + r * 128 + ((c ^ (r & 7)) << 4), x + src_off[u] + k0,
                         live ? 16u : 0u);
         }
@@ -325,8 +251,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                     const __grid_constant__ CUtensorMap map_act, Params p) {
     using C = Cfg<BN, GATE_UP>;
-    // 16-row tiles are the narrowest: per-group heights only pay above them
-    constexpr bool kAdapt = BN > 16;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -338,10 +262,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* total_slot = reinterpret_cast<int*>(tmem_slot + 2);
-    int* cap_slot = reinterpret_cast<int*>(tmem_slot + 3);
     int* g_off = reinterpret_cast<int*>(tmem_slot + 4);
     int* g_tile = g_off + (p.G + 1);
-    int* stage_bn = g_tile + (p.G + 1);  // [kStages] rows of the tile each stage belongs to
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -373,20 +295,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
     // and the accumulator are produced by earlier kernels of the stream
     grid_dep_wait();
     grid_dep_launch();
-    if constexpr (kAdapt)
-        build_tile_table_adaptive(p, BN, g_off, g_tile, total_slot, cap_slot, warp, lane);
-    else
-        build_tile_table(p, BN, g_off, g_tile, total_slot, warp, lane);
+    build_tile_table(p, BN, g_off, g_tile, total_slot, warp, lane);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int total = *total_slot;
-    const int cap = kAdapt ? *cap_slot : BN;
-    auto tile_at = [&](int tile) {
-        if constexpr (kAdapt) return decode_tile_adaptive(tile, g_tile, g_off, p.G, cap);
-        else return decode_tile(tile, g_tile, g_off, p.G, BN);
-    };
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
@@ -402,9 +316,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
             uint32_t phase = 0, filled = 0, fill_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const Tile t = tile_at(tile);
+                const Tile t = decode_tile(tile, g_tile, g_off, p.G, BN);
                 const int wr0 = t.g * p.w_group_rows + t.i * kBM;
-                const uint32_t stage_bytes = a_bytes + t.bn * kBK * 2;
                 RowGather<BN> rg;
                 if (gather) rg.plan(p.gather_tok, t.row0, t.row_end, p.nk * kBK, lane);
                 for (int kk = 0; kk < p.nk; ++kk) {
@@ -418,19 +331,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                     }
                     uint8_t* st = smem + stage * C::kStageBytes;
                     if (lane == 0) {
-                        stage_bn[stage] = t.bn;  // published by the arrive below
-                        mbar_arrive_expect_tx(&full[stage], gather ? a_bytes : stage_bytes);
+                        mbar_arrive_expect_tx(&full[stage], gather ? a_bytes : C::kStageBytes);
                         tma_load_2d(st, &map_w, &full[stage], kk * kBK, wr0, pol_w);
                         if (GATE_UP)
                             tma_load_2d(st + C::kABytes, &map_w, &full[stage], kk * kBK,
                                         wr0 + p.up_rows, pol_w);
                         if (!gather)
-                            for (int b = 0; b < t.bn; b += 16)
+                            for (int b = 0; b < BN; b += 16)
                                 tma_load_2d(st + a_bytes + b * kBK * 2, &map_act, &full[stage],
                                             kk * kBK, t.row0 + b, pol_a);
                     }
                     if (gather) {
-                        rg.issue(smem_u32(st + a_bytes), p.x, kk * kBK, lane, t.bn);
+                        rg.issue(smem_u32(st + a_bytes), p.x, kk * kBK, lane);
                         cp_async_mbar_arrive_noinc(&full[stage]);
                     }
                     filled |= 1u << stage;
@@ -461,7 +373,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                 }
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + abuf * C::kAccCols;
-                uint32_t idesc = idesc_bf16_f32(kBM, BN);
+                constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
                 for (int kk = 0; kk < p.nk; ++kk) {
                     if (!mbar_wait(&full[stage], phase, kWaitBudgetNs, abort_flag)) {
                         set_status(p.status, MOE_ERR_TIMEOUT);
@@ -471,8 +383,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                     }
                     tc_fence_after();
                     if (gather) fence_proxy_async_smem();
-                    if (kAdapt && kk == 0)
-                        idesc = idesc_bf16_f32(kBM, stage_bn[stage]);  // N = this tile's rows
                     const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
                     const uint32_t a1 = a0 + C::kABytes;
                     const uint32_t b0 = a0 + C::kNumA * C::kABytes;
@@ -504,7 +414,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
         const int feat_in_tile = q * 32 + lane;
         uint32_t abuf = 0, aphase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const Tile t = tile_at(tile);
+            const Tile t = decode_tile(tile, g_tile, g_off, p.G, BN);
             const bool ready = mbar_wait(&tfull[abuf], aphase, kWaitBudgetNs, abort_flag);
             if (!epilogue_bar_and(ready)) {
                 set_status(p.status, MOE_ERR_TIMEOUT);
@@ -516,7 +426,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                                    abuf * C::kAccCols;
             const int feat = t.i * kBM + feat_in_tile;
 #pragma unroll 1
-            for (int c0 = 0; c0 < (kAdapt ? t.bn : BN); c0 += 16) {
+            for (int c0 = 0; c0 < BN; c0 += 16) {
                 uint32_t gv[16];
                 uint32_t uv[16];
                 tmem_ld16(tbase + c0, gv);
@@ -566,6 +476,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
 // one row, so h is written with 16-byte stores and the down epilogue reduces 16-byte
 // vectors (red.global.add.v4.f32) into the token's output row.
 constexpr int kTmRows = 128;  // token rows per tile (MMA M)
+// auto orientation: weights on M only while no group can exceed this many rows
+constexpr int kSwapMaxRows = 16;
 constexpr int kTmN = 256;     // weight rows per tile (MMA N)
 // 2 warps (producer, MMA) + 8 epilogue warps: two warps per tensor-memory lane quarter,
 // each draining half of the accumulator's columns
@@ -1069,7 +981,7 @@ cudaError_t launch_tpl(const CUtensorMap& mw, const CUtensorMap& ma, const Param
     using C = Cfg<BN, GATE_UP>;
     const size_t smem = 1024 + static_cast<size_t>(C::kStages) * C::kStageBytes +
                         (2 * C::kStages + 5) * 8 + 16 +
-                        (2 * (p.G + 1) + C::kStages) * sizeof(int);
+                        2 * (p.G + 1) * sizeof(int);
     auto kfn = grouped_gemm_kernel<BN, GATE_UP>;
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
@@ -1133,38 +1045,25 @@ int pick_block_rows(int rows, int groups) {
     return 128;
 }
 
-cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s,
-                                bool pdl) {
-    if (a.rows == 0 || a.E == 0) return cudaSuccess;
-    if (a.E > kMaxGroups) return cudaErrorInvalidValue;
-    cudaError_t err = get_encoder();
-    if (err != cudaSuccess) return err;
-    // orientation: tokens on the MMA's M side once the groups average a full 128-row tile
-    // (and the output width splits into 256-wide blocks for down); weights on M otherwise
-    const bool tm_ok = a.gate_up ? (a.f % 128 == 0) : (a.D % 256 == 0);
-    const bool tm = tm_ok && (a.orientation >= 2 ||
-                              (a.orientation == 0 && a.block_rows == 0 && a.rows / a.E >= 128));
-    // tokens on M: CTA pairs when A's rows are contiguous (always for down; for gate_up once
-    // x is gathered into expert order), unless a single CTA is asked for
-    const bool gathered = a.gate_up && a.gather_tok != nullptr;
-    const bool pairs = tm && a.orientation != 2 && (!gathered || a.gather_buf != nullptr) &&
-                       num_sms >= 2;
-    // weights on M: tiles adapt per group up to BN, sized for groups up to 8x the average
-    // (skewed routing) but never past the largest possible group
-    const int max_rows = a.max_group_rows > 0 ? a.max_group_rows : a.rows;
-    const long long avg8 = 8ll * a.rows / (a.E > 0 ? a.E : 1);
-    const int bn_rows = static_cast<int>(std::min<long long>(max_rows, std::max(avg8, 16ll)));
-    const int BN = tm ? kTmRows : (a.block_rows ? a.block_rows : pick_block_rows(bn_rows, 1));
-    if (BN != 16 && BN != 32 && BN != 64 && BN != 128) return cudaErrorInvalidValue;
+namespace {
+
+enum class Kind { kSwap, kTm, kPair };
+
+// One launch of one kernel kind over every group.  BN: largest rows per tile of the
+// weights-on-M kernel.
+cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_sms,
+                        cudaStream_t s, bool pdl) {
+    const bool tm = kind != Kind::kSwap;
     const int K = a.gate_up ? a.D : a.f;
     const uint64_t w_group_rows = a.gate_up ? 2ull * a.f : static_cast<uint64_t>(a.D);
     CUtensorMap mw, ma;
+    cudaError_t err;
     if ((err = make_map(&mw, a.w, w_group_rows * a.E, K, kBM)) != cudaSuccess) return err;  // 128-row boxes
     // the activation map is only read when the rows are contiguous (no gather); with a
     // gather it still has to be a valid descriptor, so it covers the first row of x
     const void* act = a.act;
-    bool gather = gathered;
-    if (pairs && gathered) {
+    bool gather = a.gate_up && a.gather_tok != nullptr;
+    if (kind == Kind::kPair && gather) {
         err = launch_gather_rows(reinterpret_cast<const bf16*>(a.act), a.gather_tok, a.rows, a.D,
                                  a.gather_buf, num_sms, s, pdl);
         if (err != cudaSuccess) return err;
@@ -1196,16 +1095,16 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
     p.final_rows = a.final_rows;
     p.done = a.done;
     p.final_residual = a.final_residual;
+    // persistent grids: one CTA (or pair) per SM, fewer when the tiles cannot fill them
+    const int rows_per_tile = kind == Kind::kPair ? CfgPair::kPairRows : (tm ? kTmRows : 16);
     const long long max_tiles =
-        (static_cast<long long>(ceil_div(a.rows, tm ? BN : 16)) + a.E) * p.nf;
-    const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
-    if (pairs) {
-        const long long pair_tiles =
-            (static_cast<long long>(ceil_div(a.rows, CfgPair::kPairRows)) + a.E) * p.nf;
-        const int npairs = static_cast<int>(std::min<long long>(pair_tiles, num_sms / 2));
+        (static_cast<long long>(ceil_div(a.rows, rows_per_tile)) + a.E) * p.nf;
+    if (kind == Kind::kPair) {
+        const int npairs = static_cast<int>(std::min<long long>(max_tiles, num_sms / 2));
         return a.gate_up ? launch_pair<true>(mw, ma, p, npairs, s, true)
                          : launch_pair<false>(mw, ma, p, npairs, s, true);
     }
+    const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
     if (tm) return a.gate_up ? launch_tm<true>(mw, ma, p, grid, s, pdl)
                              : launch_tm<false>(mw, ma, p, grid, s, pdl);
     switch (BN) {
@@ -1214,6 +1113,46 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
         case 64: return a.gate_up ? launch_tpl<64, true>(mw, ma, p, grid, s, pdl) : launch_tpl<64, false>(mw, ma, p, grid, s, pdl);
         default: return a.gate_up ? launch_tpl<128, true>(mw, ma, p, grid, s, pdl) : launch_tpl<128, false>(mw, ma, p, grid, s, pdl);
     }
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s,
+                                bool pdl) {
+    if (a.rows == 0 || a.E == 0) return cudaSuccess;
+    if (a.E > kMaxGroups) return cudaErrorInvalidValue;
+    cudaError_t err = get_encoder();
+    if (err != cudaSuccess) return err;
+    // tokens on M needs f (gate_up) or D (down) in 128- or 256-wide blocks
+    const bool tm_ok = a.gate_up ? (a.f % 128 == 0) : (a.D % 256 == 0);
+    const bool gathered = a.gate_up && a.gather_tok != nullptr;
+    const bool pair_ok = tm_ok && (!gathered || a.gather_buf != nullptr) && num_sms >= 2;
+    // weights on M: tiles adapt per group up to BN, sized for groups up to 8x the average
+    // (skewed routing) but never past the largest possible group
+    const int max_rows = a.max_group_rows > 0 ? a.max_group_rows : a.rows;
+    const long long avg8 = 8ll * a.rows / a.E;
+    const int bn_rows = static_cast<int>(std::min<long long>(max_rows, std::max(avg8, 16ll)));
+    const int BN = a.block_rows ? a.block_rows : pick_block_rows(bn_rows, 1);
+    if (BN != 16 && BN != 32 && BN != 64 && BN != 128) return cudaErrorInvalidValue;
+
+    // Orientation.  Weights on M (token tiles of 16..128 rows) when asked for, or while no
+    // group can hold more than kSwapMaxRows rows (a handful of tokens: the weight-read-bound
+    // regime, where a 128-row token tile would be nearly empty).  Otherwise tokens on M:
+    // both orientations stream each weight tile once per row block and are within a few
+    // percent of each other on 2-row groups, but tokens on M keeps features along the
+    // accumulator's columns (16-byte stores and vector reductions in the epilogue) and wins
+    // clearly once groups hold tens of rows.  CTA pairs once the groups average a full
+    // 256-row pair tile's half (their rows must be contiguous: x is gathered first).
+    Kind kind;
+    if (a.orientation == 1 || a.block_rows || !tm_ok)
+        kind = Kind::kSwap;
+    else if (a.orientation == 2)
+        kind = Kind::kTm;
+    else if (a.orientation == 3 || a.rows / a.E >= 128)
+        kind = pair_ok ? Kind::kPair : Kind::kTm;
+    else
+        kind = max_rows <= kSwapMaxRows ? Kind::kSwap : Kind::kTm;
+    return launch_kind(a, kind, BN, num_sms, s, pdl);
 }
 
 }  // namespace moe
