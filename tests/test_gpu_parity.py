@@ -110,6 +110,19 @@ def test_route_shapes(moe, oracle_mod, T, D, E, K):
     check_route(orc, _np(idx), _np(w), _np(counts))
 
 
+@pytest.mark.parametrize("T,D,E,K", [(1000, 2048, 256, 8), (4099, 4096, 128, 8)])
+def test_route_repeatable(moe, T, D, E, K):
+    """The tensor-core router's split reduction adds its partial planes in a fixed order:
+    two calls give the same bits."""
+    cfg = LayerConfig("r", T=T, D=D, E=E, K=K, f=128, seed=1)
+    inp = make_inputs(cfg).to("cuda")
+    a = moe.route(inp.x, inp.w_router, K)
+    b = moe.route(inp.x, inp.w_router, K)
+    torch.cuda.synchronize()
+    for u, v in zip(a[:3], b[:3]):
+        assert torch.equal(u, v)
+
+
 # ------------------------------------------------------------------ permutation
 
 

@@ -77,7 +77,8 @@ struct RouterLaunch {
     unsigned* counters;   // [ceil(T/8)] workspace, zeroed before the launch
     int32_t* topk_idx;
     float* topk_w;
-    int32_t* counts;      // zeroed before the launch
+    int32_t* counts;      // zeroed before the launch; NULL: not counted (the
+                          // permutation derives them, tensor-core path)
     float* shared_gate;
     int* status;
     // optional: rows [T, zero_cols] of zero_acc are cleared by the router kernel (the
@@ -87,19 +88,24 @@ struct RouterLaunch {
     int score_mode;           // 0: softmax over the experts; 1: per-expert sigmoid
     const float* select_bias; // [E] added to the scores for the selection only, or NULL
     int bf16_weights;         // round the renormalised weights to bf16
+    int logit_planes;         // tensor-core path: partial-sum planes of [T, E] in logits
 };
 cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bool pdl = false);
 
 // Router for many tokens: the logits x W_r^T [T, E] (fp32) on the tensor cores through the
-// grouped GEMM (one dense group), then a selection kernel.  Needs E % 128 == 0 and
-// a.logits with room for T*E floats.
+// grouped GEMM (one dense group, the reduction over D split into up to
+// router_tc_max_planes(T) slices, each writing a partial [T, E] plane), then a selection
+// kernel that adds the planes in slice order.  Needs E % 128 == 0 and a.logits with room
+// for router_tc_max_planes(T) * T * E floats.
 bool router_uses_tensor_cores(int T, int E);
+int router_tc_max_planes(int T);
 cudaError_t launch_router_tc(const RouterLaunch& a, int num_sms, cudaStream_t s, bool pdl = false);
 
 struct PermuteLaunch {
     const int32_t* topk_idx;
     const float* topk_w;
-    const int32_t* counts;
+    const int32_t* counts;   // [E] from the router, or NULL: counted here from topk_idx
+    int32_t* counts_out;     // with counts NULL: where the counts are written, or NULL
     int T, E, K;
     int32_t* offsets;
     int32_t* sorted_token;
@@ -141,6 +147,13 @@ struct GroupedGemmLaunch {
     // gate_up with gather_tok: room for the rows in expert order [rows, D]; when given, the
     // CTA-pair kernel may be used (rows gathered by a copy kernel first)
     bf16* gather_buf;
+    // down with y_out only (weights on M): split the reduction over f into ksplit equal
+    // slices; slice s writes y_out + s * rows * D (0 or 1: no split)
+    int ksplit;
+    // gate_up: clear zero_acc[0, zero_floats) (a multiple of 4, 16-byte aligned) in the
+    // kernel, before the down projection adds into it; NULL: nothing to clear
+    float* zero_acc;
+    long long zero_floats;
 };
 cudaError_t launch_gather_rows(const bf16* x, const int32_t* tok, int rows, int D, bf16* out,
                                int num_sms, cudaStream_t s, bool pdl);

@@ -83,7 +83,25 @@ struct Params {
     int final_rows;             //   bf16 here once every CTA of the grid has added its tiles
     unsigned* done;             //   (grid barrier counter, zero at launch)
     const bf16* final_residual; //   + this bf16 [final_rows, out_cols] when not NULL
+    // weights-on-M kernel, y_out only: the K steps are cut into ksplit equal slices, one
+    // tile per slice, and slice s writes its partial sums to y_out + s * split_stride
+    int ksplit;
+    long long split_stride;
+    // gate_up: the epilogue warps clear zero_acc[0, zero_n4) (float4s, the layer's fp32
+    // accumulator) before their first tile -- they would otherwise wait for it idle
+    float* zero_acc;
+    long long zero_n4;
 };
+
+// Epilogue threads of every CTA clear their grid-strided share of p.zero_acc.
+__device__ __forceinline__ void clear_accumulator(const Params& p, int epi_tid, int epi_threads) {
+    if (p.zero_acc == nullptr) return;
+    float4* dst = reinterpret_cast<float4*>(p.zero_acc);
+    const long long step = static_cast<long long>(gridDim.x) * epi_threads;
+    for (long long i = static_cast<long long>(blockIdx.x) * epi_threads + epi_tid; i < p.zero_n4;
+         i += step)
+        __stcs(dst + i, make_float4(0.f, 0.f, 0.f, 0.f));
+}
 
 // tiles of a group of n rows cut into row blocks of `rows`
 __device__ __forceinline__ int group_tiles(const Params& p, int n, int rows) {
@@ -300,7 +318,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int total = *total_slot;
+    // tiles: (group tile, K slice) with the slice varying fastest, so that CTAs working at
+    // the same time read different K ranges of the weights
+    const int nsplit = p.ksplit;
+    const int total = *total_slot * nsplit;
+    const int nks = p.nk / nsplit;  // K steps per slice
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
@@ -316,11 +338,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
             uint32_t phase = 0, filled = 0, fill_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const Tile t = decode_tile(tile, g_tile, g_off, p.G, BN);
+                const Tile t = decode_tile(tile / nsplit, g_tile, g_off, p.G, BN);
+                const int kb = (tile % nsplit) * nks;
                 const int wr0 = t.g * p.w_group_rows + t.i * kBM;
                 RowGather<BN> rg;
                 if (gather) rg.plan(p.gather_tok, t.row0, t.row_end, p.nk * kBK, lane);
-                for (int kk = 0; kk < p.nk; ++kk) {
+                for (int kk = kb; kk < kb + nks; ++kk) {
                     bool got = mbar_wait(&empty[stage], phase ^ 1u, kWaitBudgetNs, abort_flag);
                     if (gather) got = __all_sync(0xffffffffu, got);
                     if (!got) {
@@ -374,7 +397,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + abuf * C::kAccCols;
                 constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
-                for (int kk = 0; kk < p.nk; ++kk) {
+                for (int kk = 0; kk < nks; ++kk) {
                     if (!mbar_wait(&full[stage], phase, kWaitBudgetNs, abort_flag)) {
                         set_status(p.status, MOE_ERR_TIMEOUT);
                         *abort_flag = 1;
@@ -412,9 +435,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
         // ---------------------------------------------------------------- epilogue
         const int q = warp & 3;  // tensor-memory lane quarter this warp may read
         const int feat_in_tile = q * 32 + lane;
+        if (GATE_UP) clear_accumulator(p, threadIdx.x - 64, kEpiThreads);
         uint32_t abuf = 0, aphase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const Tile t = decode_tile(tile, g_tile, g_off, p.G, BN);
+            const Tile t = decode_tile(tile / nsplit, g_tile, g_off, p.G, BN);
+            float* y_slice = p.y_out ? p.y_out + (tile % nsplit) * p.split_stride : nullptr;
             const bool ready = mbar_wait(&tfull[abuf], aphase, kWaitBudgetNs, abort_flag);
             if (!epilogue_bar_and(ready)) {
                 set_status(p.status, MOE_ERR_TIMEOUT);
@@ -448,7 +473,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                             const int tok = p.sorted_token ? __ldg(p.sorted_token + row) : row;
                             red_add_f32(p.acc_out + static_cast<size_t>(tok) * p.out_cols + feat, v);
                         }
-                        if (p.y_out) p.y_out[static_cast<size_t>(row) * p.out_cols + feat] = v;
+                        if (y_slice) y_slice[static_cast<size_t>(row) * p.out_cols + feat] = v;
                     }
                 }
             }
@@ -719,6 +744,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
     } else {
         // ---------------------------------------------------------------- epilogue
         const int q = warp & 3;
+        if (GATE_UP) clear_accumulator(p, threadIdx.x - 64, kTmEpiThreads);
         uint32_t abuf = 0, aphase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             const Tile t = decode_tile(tile, g_tile, g_off, p.G, kTmRows);
@@ -912,6 +938,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_w,
     } else {
         // ---------------------------------------------------------------- epilogue (both)
         const int q = warp & 3;
+        if (GATE_UP) clear_accumulator(p, threadIdx.x - 64, kTmEpiThreads);
         const uint32_t leader_tempty0 = map_to_rank(smem_u32(&tempty[0]), 0);
         uint32_t abuf = 0, aphase = 0;
         for (int tile = pair; tile < total; tile += npairs) {
@@ -1095,10 +1122,14 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
     p.final_rows = a.final_rows;
     p.done = a.done;
     p.final_residual = a.final_residual;
+    p.ksplit = kind == Kind::kSwap && a.ksplit > 1 ? a.ksplit : 1;
+    p.zero_acc = a.gate_up ? a.zero_acc : nullptr;
+    p.zero_n4 = a.zero_floats / 4;
+    p.split_stride = static_cast<long long>(a.rows) * p.out_cols;
     // persistent grids: one CTA (or pair) per SM, fewer when the tiles cannot fill them
     const int rows_per_tile = kind == Kind::kPair ? CfgPair::kPairRows : (tm ? kTmRows : 16);
     const long long max_tiles =
-        (static_cast<long long>(ceil_div(a.rows, rows_per_tile)) + a.E) * p.nf;
+        (static_cast<long long>(ceil_div(a.rows, rows_per_tile)) + a.E) * p.nf * p.ksplit;
     if (kind == Kind::kPair) {
         const int npairs = static_cast<int>(std::min<long long>(max_tiles, num_sms / 2));
         return a.gate_up ? launch_pair<true>(mw, ma, p, npairs, s, true)
@@ -1143,8 +1174,11 @@ cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStr
     // accumulator's columns (16-byte stores and vector reductions in the epilogue) and wins
     // clearly once groups hold tens of rows.  CTA pairs once the groups average a full
     // 256-row pair tile's half (their rows must be contiguous: x is gathered first).
+    if (a.ksplit > 1 && (a.gate_up || !a.y_out || a.acc_out || a.final_out ||
+                         (a.f / kBK) % a.ksplit != 0))
+        return cudaErrorInvalidValue;
     Kind kind;
-    if (a.orientation == 1 || a.block_rows || !tm_ok)
+    if (a.orientation == 1 || a.block_rows || !tm_ok || a.ksplit > 1)
         kind = Kind::kSwap;
     else if (a.orientation == 2)
         kind = Kind::kTm;

@@ -1,5 +1,6 @@
 // moe_api.cu -- the extern "C" entry points of libmoe_b200.so: argument checks on the
 // host, workspace layout, and the launch sequence of the layer.  See include/moe_api.h.
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -54,7 +55,11 @@ Layout layout(long long T, long long D, long long E, long long K, long long f, l
     L.zero_end = o;
     // depends on T, E and K only, so any workspace sized for the same T, E, K has it here
     L.perm_hist = take(sizeof(int32_t) * E * permute_chunks(T * K));
-    L.logits = take(sizeof(float) * T * (E + 1));
+    // router logits: [T, E+1] (CUDA-core router) or partial-sum planes of [T, E]
+    L.logits = take(sizeof(float) * T *
+                    std::max<long long>(E + 1, router_uses_tensor_cores(static_cast<int>(T), static_cast<int>(E))
+                                                   ? router_tc_max_planes(static_cast<int>(T)) * E
+                                                   : 0));
     L.offsets = take(sizeof(int32_t) * (E + 1));
     L.dense_offsets = take(sizeof(int32_t) * 2);
     L.topk_idx = take(sizeof(int32_t) * T * K);
@@ -141,7 +146,7 @@ int moe_route_ex(const moe_bf16* x, const moe_bf16* w_router, const float* logit
         return MOE_ERR_ALIGN;
     const Layout L = layout(T, D, E, K, 128, 0);
     if (!workspace) return MOE_ERR_WORKSPACE;
-    if (ws_bytes < L.logits + sizeof(float) * static_cast<size_t>(T) * (E + 1)) return MOE_ERR_WORKSPACE;
+    if (ws_bytes < L.offsets) return MOE_ERR_WORKSPACE;  // through the logits region
     cudaStream_t s = as_stream(stream);
     if (cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * E, s) != cudaSuccess) return MOE_ERR_CUDA;
     if (T == 0) return MOE_OK;
@@ -295,13 +300,15 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     float* out_acc = at<float>(workspace, L.out_acc);
 
     if (!mark(MOE_EV_START)) return MOE_ERR_CUDA;
-    // the only clear: status word, router tickets, expert counts (a few KB); the router
-    // kernel clears the fp32 accumulator itself
+    // the only clear: status word, router tickets, expert counts (a few KB); the fp32
+    // accumulator is cleared by the CUDA-core router kernel, or (tensor-core router, many
+    // tokens) by the gate_up kernel's epilogue warps while its first tiles accumulate
     if (cudaMemsetAsync(workspace, 0, L.zero_end, s) != cudaSuccess) return MOE_ERR_CUDA;
     if (p->expert_counts_out && cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     const bool use_acc = !det || shared;
 
+    const bool tc_router = router_uses_tensor_cores(T, E);
     RouterLaunch r{};
     r.x = reinterpret_cast<const bf16*>(p->x);
     r.w_router = reinterpret_cast<const bf16*>(p->w_router);
@@ -312,23 +319,25 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     r.counters = at<unsigned>(workspace, L.counters);
     r.topk_idx = idx;
     r.topk_w = tw;
-    r.counts = counts;
+    // tensor-core router (many tokens): no per-entry count atomics in the selection; the
+    // permutation counts from its chunk histograms
+    r.counts = tc_router ? nullptr : counts;
     r.shared_gate = sgate;
     r.status = status;
-    r.zero_acc = use_acc ? out_acc : nullptr;
+    r.zero_acc = use_acc && !tc_router ? out_acc : nullptr;
     r.zero_cols = D;
     r.score_mode = p->score_mode;
     r.select_bias = p->select_bias;
     r.bf16_weights = (p->flags & MOE_FLAG_BF16_WEIGHTS) ? 1 : 0;
     if (!mark(MOE_EV_ROUTER)) return MOE_ERR_CUDA;
-    if ((router_uses_tensor_cores(T, E) ? launch_router_tc(r, sms, s) : launch_router(r, sms, s)) !=
-        cudaSuccess)
+    if ((tc_router ? launch_router_tc(r, sms, s) : launch_router(r, sms, s)) != cudaSuccess)
         return MOE_ERR_CUDA;
 
     PermuteLaunch pm{};
     pm.topk_idx = idx;
     pm.topk_w = tw;
-    pm.counts = counts;
+    pm.counts = tc_router ? nullptr : counts;
+    pm.counts_out = tc_router ? p->expert_counts_out : nullptr;
     pm.T = T; pm.E = E; pm.K = K;
     pm.offsets = at<int32_t>(workspace, L.offsets);
     pm.sorted_token = at<int32_t>(workspace, L.sorted_token);
@@ -351,6 +360,8 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     up.max_group_rows = T;
     up.h_out = at<bf16>(workspace, L.h);
     up.status = status;
+    up.zero_acc = use_acc && tc_router ? out_acc : nullptr;
+    up.zero_floats = static_cast<long long>(T) * D;
     if (!mark(MOE_EV_GATE_UP) || launch_grouped_gemm(up, sms, s, true) != cudaSuccess)
         return MOE_ERR_CUDA;
 

@@ -72,12 +72,40 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(PermuteLa
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int E = a.E, total = a.T * a.K;
     const int c = blockIdx.x;
+    const unsigned lt = (1u << lane) - 1u;
 
     grid_dep_wait();  // counts (router) and chunk histograms (previous kernel)
     grid_dep_launch();
 
-    // offsets: exclusive scan of counts (E <= 512 < kPermThreads)
-    const int n = tid < E ? a.counts[tid] : 0;
+    // counts: from the router, or counted here -- from every chunk's histogram, or (one
+    // chunk) by a first pass over the entries
+    int n = 0;
+    if (a.counts) {
+        n = tid < E ? a.counts[tid] : 0;
+    } else {
+        int* tot = warp_cnt;  // scratch until the walk below clears it
+        for (int e = tid; e < E; e += kPermThreads) tot[e] = 0;
+        __syncthreads();
+        if (chunks > 1) {
+            for (int i = tid; i < chunks * E; i += kPermThreads) {
+                const int v = a.hist[i];
+                if (v) atomicAdd(&tot[i % E], v);
+            }
+        } else {
+            for (int j0 = 0; j0 < total; j0 += kPermThreads) {
+                const int j = j0 + tid;
+                const int e = j < total ? __ldg(a.topk_idx + j) : -1;
+                const bool ok = e >= 0 && e < E;
+                const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
+                if (ok && (peers & lt) == 0) atomicAdd(&tot[e], __popc(peers));
+            }
+        }
+        __syncthreads();
+        n = tid < E ? tot[tid] : 0;
+        if (c == 0 && a.counts_out && tid < E) a.counts_out[tid] = n;
+        __syncthreads();
+    }
+    // offsets: exclusive scan of the counts (E <= 512 < kPermThreads)
     int incl = n;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -119,7 +147,6 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(PermuteLa
         if (v) atomicAdd(&base[i % E], v);
     }
     const ChunkRange r = chunk_range(c, chunk_len, total);
-    const unsigned lt = (1u << lane) - 1u;
     for (int j0 = r.begin; j0 < r.end; j0 += kPermThreads) {
         for (int i = tid; i < kPermWarps * E; i += kPermThreads) warp_cnt[i] = 0;
         __syncthreads();

@@ -22,6 +22,7 @@
 // For many tokens (T >= 256, E a multiple of 128) the logits instead come from the
 // tcgen05 grouped GEMM as one dense [T, E] product, and router_select_kernel runs the
 // same selection with one warp per token.
+#include <algorithm>
 #include <cfloat>
 
 #include "common.cuh"
@@ -35,10 +36,12 @@ constexpr int kRouterThreads = 256;
 constexpr int kExpertsPerWarp = 2;
 
 // TopK of one token's logits by one warp, in registers, then the renormalised weights.
-// lg: the token's E logits (bias already added when add_bias is NULL).  Writes idx/w of
-// the token and adds its K experts to the counts.
+// lg: the token's E logits (bias already added when add_bias is NULL), or `planes` partial
+// sums of them `plane_stride` floats apart, added in plane order.  Writes idx/w of the
+// token and adds its K experts to the counts.
 template <int NV>
-__device__ __forceinline__ void select_topk_nv(const float* lg, const float* add_bias, int E,
+__device__ __forceinline__ void select_topk_nv(const float* lg, int planes, size_t plane_stride,
+                                               const float* add_bias, int E,
                                                int K, int token, int lane, int32_t* topk_idx,
                                                float* topk_w, int32_t* counts, int score_mode,
                                                const float* select_bias, int bf16_weights) {
@@ -46,7 +49,10 @@ __device__ __forceinline__ void select_topk_nv(const float* lg, const float* add
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
         const int e = j * 32 + lane;
-        v[j] = (e < E) ? __ldcg(lg + e) + (add_bias ? __ldg(add_bias + e) : 0.f) : -FLT_MAX;
+        float r = 0.f;
+        if (e < E)
+            for (int q = 0; q < planes; ++q) r += __ldcg(lg + q * plane_stride + e);
+        v[j] = (e < E) ? r + (add_bias ? __ldg(add_bias + e) : 0.f) : -FLT_MAX;
     }
     // scores and selection keys.  Softmax without selection bias: the key is the logit
     // itself (softmax is increasing) and only the K selected terms are exponentiated.
@@ -123,17 +129,18 @@ __device__ __forceinline__ void select_topk_nv(const float* lg, const float* add
         if (bf16_weights) w = __bfloat162float(__float2bfloat16_rn(w));
         topk_idx[static_cast<size_t>(token) * K + lane] = my_i;
         topk_w[static_cast<size_t>(token) * K + lane] = w;
-        atomicAdd(&counts[my_i], 1);
+        if (counts) atomicAdd(&counts[my_i], 1);
     }
 }
 
 // NV = logits per lane = ceil(E / 32), so the selection loops run exactly as far as E needs.
-__device__ __forceinline__ void select_topk_warp(const float* lg, const float* add_bias,
+__device__ __forceinline__ void select_topk_warp(const float* lg, int planes,
+                                                 size_t plane_stride, const float* add_bias,
                                                  const RouterLaunch& a, int token, int lane) {
     const int nv = (a.E + 31) / 32;
-#define MOE_SELECT(N)                                                                     \
-    select_topk_nv<N>(lg, add_bias, a.E, a.K, token, lane, a.topk_idx, a.topk_w, a.counts, \
-                      a.score_mode, a.select_bias, a.bf16_weights)
+#define MOE_SELECT(N)                                                                      \
+    select_topk_nv<N>(lg, planes, plane_stride, add_bias, a.E, a.K, token, lane, a.topk_idx, \
+                      a.topk_w, a.counts, a.score_mode, a.select_bias, a.bf16_weights)
     if (nv <= 1) MOE_SELECT(1);
     else if (nv <= 2) MOE_SELECT(2);
     else if (nv <= 4) MOE_SELECT(4);
@@ -272,7 +279,7 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
     for (int t = warp; t < nt; t += kRouterThreads / 32) {
         const int token = t0 + t;
         const float* lg = a.logits + static_cast<size_t>(token) * (E + 1);
-        select_topk_warp(lg, nullptr, a, token, lane);
+        select_topk_warp(lg, 1, 0, nullptr, a, token, lane);
         if (a.w_shared_gate && lane == 0) {
             const float g = __ldcg(lg + E);
             a.shared_gate[token] = 1.f / (1.f + expf(-g));
@@ -297,7 +304,8 @@ __global__ void __launch_bounds__(kRouterThreads) router_select_kernel(RouterLau
     }
     if (warp >= nt) return;
     const int token = t0 + warp;
-    select_topk_warp(a.logits + static_cast<size_t>(token) * a.E, a.logit_bias, a, token, lane);
+    select_topk_warp(a.logits + static_cast<size_t>(token) * a.E, a.logit_planes,
+                     static_cast<size_t>(a.T) * a.E, a.logit_bias, a, token, lane);
     if (a.w_shared_gate) {
         const uint4* xv = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(token) * a.D);
         const uint4* wv = reinterpret_cast<const uint4*>(a.w_shared_gate);
@@ -344,10 +352,25 @@ cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bo
 
 bool router_uses_tensor_cores(int T, int E) { return T >= 256 && E % 128 == 0; }
 
+int router_tc_max_planes(int T) { return std::min(16, std::max(1, 512 / ceil_div(T, 128))); }
+
 cudaError_t launch_router_tc(const RouterLaunch& a, int num_sms, cudaStream_t s, bool pdl) {
     if (a.T == 0) return cudaSuccess;
-    // logits = x W_r^T: W_r's E rows on the MMA's M side, tokens on N, one dense group;
-    // the tile height is chosen so that the (E/128) x (T/rows) tiles cover the GPU
+    // logits = x W_r^T: W_r's E rows on the MMA's M side, 128 tokens on N, one dense group.
+    // Few tiles with a long reduction (D) would leave most SMs idle, so the D steps are cut
+    // into S slices (partial planes).  S minimises waves x (steps per slice + a tile's fixed
+    // cost, about 8 steps of 64: pipeline fill, drain and epilogue), ties to fewer planes,
+    // with at least 4 steps per slice.
+    constexpr int kTileCostSteps = 8;
+    const int nk = a.D / 64;
+    const int base = (a.E / 128) * ceil_div(a.T, 128);
+    int S = 1;
+    long long best = static_cast<long long>(ceil_div(base, num_sms)) * (nk + kTileCostSteps);
+    for (int c = 2; c <= router_tc_max_planes(a.T) && nk % c == 0 && nk / c >= 4; c *= 2) {
+        const long long cost =
+            static_cast<long long>(ceil_div(base * c, num_sms)) * (nk / c + kTileCostSteps);
+        if (cost < best) { best = cost; S = c; }
+    }
     GroupedGemmLaunch g{};
     g.gate_up = false;
     g.w = a.w_router;
@@ -359,13 +382,14 @@ cudaError_t launch_router_tc(const RouterLaunch& a, int num_sms, cudaStream_t s,
     g.f = a.D;  // reduction length
     g.y_out = a.logits;
     g.status = a.status;
-    g.block_rows = 16;
-    for (int bn = 128; bn >= 16; bn /= 2)
-        if ((a.E / 128) * ceil_div(a.T, bn) >= num_sms) { g.block_rows = bn; break; }
+    g.block_rows = 128;
+    g.ksplit = S;
     cudaError_t err = launch_grouped_gemm(g, num_sms, s, pdl);
     if (err != cudaSuccess) return err;
+    RouterLaunch sel = a;
+    sel.logit_planes = S;
     err = launch_kernel(router_select_kernel, dim3(ceil_div(a.T, kRouterThreads / 32)),
-                        dim3(kRouterThreads), 0, s, true, a);
+                        dim3(kRouterThreads), 0, s, true, sel);
     count_launches(1);
     return err;
 }
