@@ -50,6 +50,10 @@ def _load():
         lib.oracle_experts.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P, I, P]
         lib.oracle_dense_masked.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P]
         lib.oracle_permute.argtypes = [P, I, I, I, P, P, P, P, P]
+        lib.oracle_expert_capacity.argtypes = [I, I, I, ctypes.c_double, I]
+        lib.oracle_expert_capacity.restype = ctypes.c_longlong
+        lib.oracle_capacity_keep.argtypes = [P, I, I, I, ctypes.c_longlong, P]
+        lib.oracle_capacity_keep.restype = ctypes.c_int
         for fn in (lib.oracle_route, lib.oracle_experts, lib.oracle_dense_masked,
                    lib.oracle_permute):
             fn.restype = ctypes.c_int
@@ -172,14 +176,40 @@ def permute(idx, E: int):
                 sorted_slot=sorted_slot, slot_to_row=slot_to_row)
 
 
+def expert_capacity(T: int, K: int, E: int, capacity_factor: float, min_capacity: int = 0) -> int:
+    """Assignments an expert may take: max(min_capacity, ceil(capacity_factor*T*K/E))
+    ("1.6 混合专家（MoE）", expert capacity and token dropping)."""
+    c = _load().oracle_expert_capacity(T, K, E, float(capacity_factor), int(min_capacity))
+    if c < 0:
+        raise ValueError("oracle_expert_capacity: bad arguments")
+    return int(c)
+
+
+def capacity_keep(idx, E: int, C: int) -> np.ndarray:
+    """bool [T, K]: the assignment is among the first C of its expert in token order."""
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    T, K = idx.shape
+    keep = np.zeros((T * K,), np.uint8)
+    rc = _load().oracle_capacity_keep(_ptr(idx), T, K, E, int(C), _ptr(keep))
+    if rc != 0:
+        raise ValueError(f"oracle_capacity_keep failed ({rc})")
+    return keep.reshape(T, K).astype(bool)
+
+
 def layer(inp, tokens=None, score: str = "softmax", select_bias=None, bf16_weights=False,
-          residual=None):
+          residual=None, capacity=None):
     """Whole layer for a ``workloads.LayerInputs``: route every token, then the sparse
     expert sum for ``tokens`` (all when None), plus the residual h (bf16 [T, D]) when given
-    ("MoE", section 4: h_out = h + y).  Returns (route dict, y [ntok, D])."""
+    ("MoE", section 4: h_out = h + y).  With ``capacity`` = C, each expert keeps only its
+    first C assignments in token order and the dropped ones contribute nothing.
+    Returns (route dict, y [ntok, D])."""
     r = route(inp.x, inp.w_router, inp.cfg.K, inp.logit_bias, inp.w_shared_gate, score,
               select_bias, bf16_weights)
-    y = experts(inp.x, r["idx"], r["alpha"], inp.w_gate_up, inp.w_down, tokens,
+    alpha = r["alpha"]
+    if capacity is not None:
+        r["keep"] = capacity_keep(r["idx"], inp.cfg.E, capacity)
+        alpha = np.where(r["keep"], alpha, 0.0)
+    y = experts(inp.x, r["idx"], alpha, inp.w_gate_up, inp.w_down, tokens,
                 inp.w_shared_gate_up, inp.w_shared_down, r["shared_gate"])
     if residual is not None:
         h = bf16_to_f64(residual)

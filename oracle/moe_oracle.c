@@ -259,3 +259,41 @@ int oracle_permute(const int32_t* idx, int T, int E, int K, int32_t* counts, int
     offsets[E] = row;
     return row == T * K ? 0 : -1;
 }
+
+/*
+ * Expert capacity and token dropping ("1.6 混合专家（MoE）", section "专家容量与 token
+ * 丢弃"; the zskr.cn training configuration's capacity_factor / min_capacity keys): every
+ * expert processes at most C of the (token, expert) assignments routed to it; the ones
+ * past capacity are dropped -- they skip the expert, so the token keeps only its other
+ * experts' terms (nothing at all when every assignment is dropped: the layer's output is
+ * then zero and the token passes on through the residual).
+ *   C = max(min_capacity, ceil(capacity_factor * T * K / E))
+ * Readings: the capacity counts assignments (T*K of them spread over E experts; counting
+ * tokens alone, T/E, would drop most assignments at K = 8); an expert keeps its first C
+ * assignments in ascending token order; the surviving weights are not renormalised again.
+ */
+long long oracle_expert_capacity(int T, int K, int E, double capacity_factor, int min_capacity) {
+    if (T < 0 || K <= 0 || E <= 0 || capacity_factor <= 0.0) return -1;
+    const double c = ceil(capacity_factor * (double)T * (double)K / (double)E);
+    long long cap = (long long)c;
+    if (cap < min_capacity) cap = min_capacity;
+    return cap;
+}
+
+/* keep[t*K+k] = 1 when assignment (t, k) is among the first C of its expert in ascending
+ * token order, else 0.  Walks the tokens in order with one running count per expert. */
+int oracle_capacity_keep(const int32_t* idx, int T, int K, int E, long long C, uint8_t* keep) {
+    if (T < 0 || K <= 0 || E <= 0 || C < 0) return -1;
+    long long* seen = (long long*)calloc((size_t)E, sizeof(long long));
+    if (!seen) return -1;
+    int bad = 0;
+    for (int t = 0; t < T; ++t)
+        for (int k = 0; k < K; ++k) {
+            const int e = idx[(size_t)t * K + k];
+            if (e < 0 || e >= E) { bad = 1; keep[(size_t)t * K + k] = 0; continue; }
+            keep[(size_t)t * K + k] = seen[e] < C ? 1 : 0;
+            ++seen[e];
+        }
+    free(seen);
+    return bad ? -1 : 0;
+}

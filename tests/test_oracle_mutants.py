@@ -32,6 +32,15 @@ MUTANTS = {
                            ";"),
     "unstable_permutation": ("sorted_token[row] = t;", "sorted_token[row] = T - 1 - t;"),
     "softmax_without_exp": ("p[e] = exp(p[e] - m);", "p[e] = 1.0 + (p[e] - m);"),
+    "capacity_keeps_one_more": ("keep[(size_t)t * K + k] = seen[e] < C ? 1 : 0;",
+                                "keep[(size_t)t * K + k] = seen[e] <= C ? 1 : 0;"),
+    "capacity_floor_not_ceil": ("const double c = ceil(capacity_factor * (double)T * (double)K / (double)E);",
+                                "const double c = floor(capacity_factor * (double)T * (double)K / (double)E);"),
+    "capacity_counts_tokens": ("const double c = ceil(capacity_factor * (double)T * (double)K / (double)E);",
+                               "const double c = ceil(capacity_factor * (double)T / (double)E);"),
+    "capacity_ignores_minimum": ("if (cap < min_capacity) cap = min_capacity;", ";"),
+    "capacity_keeps_latest": ("keep[(size_t)t * K + k] = seen[e] < C ? 1 : 0;",
+                              "keep[(size_t)t * K + k] = seen[e] >= C ? 1 : 0;"),
 }
 
 

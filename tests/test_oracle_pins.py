@@ -360,3 +360,92 @@ def test_shared_expert_flops_formula(oracle_mod):
     counts = [3, 0, 5, 8]
     F = acc.layer_flops(counts, m=8, d=64, f=32, f_s=16)
     assert F == 2 * 8 * 3 * 64 * 16 + 2 * 16 * 3 * 64 * 32
+
+
+# ---------------------------------------------------------------- expert capacity
+
+
+def _pairs(text):
+    return np.array([[int(v) for v in p.split()] for p in text.split(",")], dtype=np.int32)
+
+
+def test_capacity_values(oracle_mod):
+    """C = max(min_capacity, ceil(cf * T * K / E)) against hand-worked values for the
+    configuration the pages print (capacity_factor 1.25, min_capacity 4)."""
+    g = golden("capacity.txt")
+    cf, mn = float(g["capacity_factor"]), int(g["min_capacity"])
+    n = 0
+    for key, val in g.items():
+        if key.startswith("cap "):
+            T, K, E = map(int, key.split()[1:])
+            assert oracle_mod.expert_capacity(T, K, E, cf, mn) == int(val), key
+            n += 1
+        elif key.startswith("cap0 "):
+            T, K, E = map(int, key.split()[1:])
+            assert oracle_mod.expert_capacity(T, K, E, 1.0, 0) == int(val), key
+    assert n == 5
+
+
+def test_capacity_keep_worked_example(oracle_mod):
+    g = golden("capacity.txt")
+    idx, keep = _pairs(g["route"]), _pairs(g["keep"]).astype(bool)
+    np.testing.assert_array_equal(oracle_mod.capacity_keep(idx, 3, 2), keep)
+
+
+@pytest.mark.parametrize("T,E,K,C", [(50, 8, 3, 4), (200, 16, 4, 30), (64, 256, 8, 2), (7, 4, 4, 0)])
+def test_capacity_keep_is_first_c_in_token_order(oracle_mod, T, E, K, C):
+    """Brute force: for every expert, the kept assignments are exactly the first C tokens
+    (ascending) that chose it."""
+    idx = random_routing(T, E, K, seed=T + C).numpy()
+    keep = oracle_mod.capacity_keep(idx, E, C)
+    for e in range(E):
+        toks = [t for t in range(T) if e in idx[t]]
+        kept = [t for t in range(T) for k in range(K) if idx[t, k] == e and keep[t, k]]
+        assert kept == toks[:C], e
+
+
+def test_capacity_drops_whole_tokens_to_zero(oracle_mod):
+    """Every token picks experts 0..K-1: with C = 3 only tokens 0, 1, 2 keep anything.  The
+    later tokens get y = 0 exactly (they pass through the residual alone); the first three
+    are unchanged from the dropless layer."""
+    cfg = LayerConfig("cap", T=9, D=64, E=8, K=2, f=32)
+    inp = make_inputs(cfg)
+    big = torch.zeros(8)
+    big[:2] = 30.0   # every token routes to experts 0 and 1
+    inp.logit_bias = big
+    r0, y0 = oracle_mod.layer(inp)
+    r, y = oracle_mod.layer(inp, capacity=3)
+    assert np.all(np.sort(r["idx"], axis=1) == [0, 1])
+    assert np.all(y[3:] == 0.0)
+    np.testing.assert_array_equal(y[:3], y0[:3])
+
+
+def test_capacity_keeps_weights_unrenormalised(oracle_mod):
+    """A token that loses one of its two experts keeps alpha_kept * E_kept(x) -- the surviving
+    weight is not renormalised (torch float64 SwiGLU)."""
+    cfg = LayerConfig("cap", T=5, D=64, E=16, K=2, f=48)
+    inp = make_inputs(cfg)
+    bias = torch.zeros(16)
+    bias[0] = 30.0   # expert 0 is every token's first choice; C = 1 leaves it to token 0
+    inp.logit_bias = bias
+    r, y = oracle_mod.layer(inp, capacity=1)
+    checked = 0
+    for t in range(1, cfg.T):
+        k0 = int(np.where(r["idx"][t] == 0)[0][0])
+        assert not r["keep"][t, k0]
+        if not r["keep"][t, 1 - k0]:
+            continue  # its second expert was already taken by an earlier token
+        e2 = int(r["idx"][t, 1 - k0])
+        ref = r["alpha"][t, 1 - k0] * _torch_swiglu(inp.x[t:t + 1], inp.w_gate_up[e2],
+                                                    inp.w_down[e2]).numpy()[0]
+        np.testing.assert_allclose(y[t], ref, rtol=1e-10, atol=1e-12)
+        checked += 1
+    assert checked >= 2
+
+
+def test_capacity_at_or_above_every_group_is_dropless(oracle_mod):
+    cfg = LayerConfig("cap", T=40, D=64, E=8, K=3, f=32, f_s=32, seed=4)
+    inp = make_inputs(cfg)
+    _, y0 = oracle_mod.layer(inp)
+    _, y = oracle_mod.layer(inp, capacity=cfg.T)
+    np.testing.assert_array_equal(y, y0)
