@@ -157,12 +157,32 @@ MOE_API int moe_route_noalloc(const moe_bf16* x, const moe_bf16* w_router,
  *   sorted_token   [T*K] int32 token of each row
  *   sorted_w       [T*K] fp32 routing weight of each row (ignored if topk_w is NULL)
  *   slot_to_row    [T*K] int32 row of pair t*K+k (the inverse map)
+ * workspace: NULL, or at least moe_workspace_size(T, 128, E, K, 128, 0) bytes (any layer
+ * workspace for the same T, E, K qualifies) with its first 256 bytes zero before the
+ * first call: it holds the device status word and the per-chunk expert histograms that
+ * let many CTAs place T*K > 4096 entries; with NULL one CTA walks every entry.
  * Counts that disagree with topk_idx set MOE_ERR_DEVICE in the device status word of
- * `workspace` when it is not NULL.
+ * `workspace` when it is not NULL; rows they would push out of the arrays are not written.
  */
 MOE_API int moe_permute(const int32_t* topk_idx, const float* topk_w, const int32_t* expert_counts,
                 int T, int E, int K, int32_t* expert_offsets, int32_t* sorted_token,
                 float* sorted_w, int32_t* slot_to_row, void* workspace, void* stream);
+
+/*
+ * moe_permute with an expert capacity ("1.6 混合专家（MoE）", section 三, expert capacity and
+ * token dropping): capacity >= 0 keeps only the first `capacity` entries of each expert in
+ * ascending token order (see moe_expert_capacity); capacity < 0 is moe_permute.  Then
+ *   expert_offsets[e+1] - expert_offsets[e] = min(counts[e], capacity),
+ *   expert_offsets[E] = the kept total (<= T*K);
+ *   slot_to_row[t*K+k] = -1 for a dropped pair;
+ *   sorted_token / sorted_w rows from expert_offsets[E] to T*K are filled with token 0 and
+ *   weight 0 (they belong to no group).
+ * Other arguments, outputs and errors as moe_permute (expert_counts stay the full counts).
+ */
+MOE_API int moe_permute_ex(const int32_t* topk_idx, const float* topk_w,
+                           const int32_t* expert_counts, int T, int E, int K, long long capacity,
+                           int32_t* expert_offsets, int32_t* sorted_token, float* sorted_w,
+                           int32_t* slot_to_row, void* workspace, void* stream);
 
 /*
  * Grouped SwiGLU experts ("MoE", section 3 expert equation and section 3.2 expert loop):
@@ -199,7 +219,8 @@ MOE_API int moe_grouped_swiglu(const moe_bf16* x, const int32_t* sorted_token,
  *                     + shared_gate[t] * shared_out[t, :] )
  * Every term is optional: out_acc (fp32 [T, D]) NULL -> acc = 0; y_sorted (fp32 [T*K, D])
  * NULL -> no routed sum; topk_w NULL -> w = 1 (y_sorted already weighted); shared_out
- * (bf16 [T, D]) NULL -> no shared term.  The k-sum runs in slot order (deterministic).
+ * (bf16 [T, D]) NULL -> no shared term.  The k-sum runs in slot order (deterministic);
+ * a pair with slot_to_row = -1 (dropped by an expert capacity, moe_permute_ex) adds nothing.
  */
 MOE_API int moe_combine(const float* out_acc, const float* y_sorted, const int32_t* slot_to_row,
                 const float* topk_w, const moe_bf16* shared_out, const float* shared_gate,
@@ -224,7 +245,25 @@ typedef struct moe_layer_params {
     int score_mode;                   /* MOE_SCORE_SOFTMAX (0) or MOE_SCORE_SIGMOID */
     const float* select_bias;         /* [E] selection-only bias, or NULL (see moe_route_ex) */
     const moe_bf16* residual;         /* [T, D] decoder residual h: out = h + y, or NULL */
+    /* Expert capacity ("1.6 混合专家（MoE）", section 三, expert capacity and token
+     * dropping): capacity_factor > 0 limits every expert to
+     * C = moe_expert_capacity(T, K, E, capacity_factor, min_capacity) of its assignments,
+     * the first C in ascending token order; the others are dropped and add nothing (the
+     * kept weights are not renormalised; a token whose every assignment is dropped gets
+     * y = 0, i.e. out = residual).  0: no capacity (dropless, the default). */
+    float capacity_factor;
+    int min_capacity;                 /* lower bound on C (0: none) */
 } moe_layer_params;
+
+/*
+ * The expert capacity the layer applies: max(min_capacity, ceil(capacity_factor * T * K / E))
+ * assignments per expert -- the batch's T*K (token, expert) assignments spread over E
+ * experts, times the capacity factor (for top-1 routing this is the pages' tokens / experts
+ * x capacity_factor).  Computed in double precision.  Returns -1 for capacity_factor <= 0
+ * (no capacity) or bad sizes.
+ */
+MOE_API long long moe_expert_capacity(int T, int K, int E, float capacity_factor,
+                                      int min_capacity);
 
 /*
  * Step boundaries at which moe_layer_forward records p->step_events[i] on its stream when

@@ -20,6 +20,16 @@ def oracle_mod():
     return oracle
 
 
+@pytest.fixture(scope="session")
+def moe():
+    """The CUDA library's binding, for GPU tests (fails when there is no device)."""
+    import torch
+    import top_routing_grouped_03_b200 as m
+    m.lib()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return m
+
+
 def golden(name: str) -> dict:
     """Parse a ``key = value  # comment`` fixture from tests/golden/."""
     out = {}

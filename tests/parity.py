@@ -105,9 +105,11 @@ def oracle_outputs(orc_mod, inp, idx, alpha, tokens, shared_gate=None):
 
 
 def check_layer(orc_mod, inp, y_gpu, gpu_idx, gpu_w, tokens=None, orc=None, score="softmax",
-                select_bias=None, bf16_weights=False, residual=None):
+                select_bias=None, bf16_weights=False, residual=None, capacity=None):
     """Route on the oracle (all tokens), compare routing, then compare y (+ residual) on
-    `tokens` (all when None).  Returns a dict of measured errors."""
+    `tokens` (all when None); with an expert capacity C the oracle drops every assignment
+    past the first C of its expert (token order) of that routing.  Returns a dict of
+    measured errors."""
     cfg = inp.cfg
     if orc is None:
         orc = orc_mod.route(inp.x, inp.w_router, cfg.K, inp.logit_bias, inp.w_shared_gate,
@@ -124,6 +126,11 @@ def check_layer(orc_mod, inp, y_gpu, gpu_idx, gpu_w, tokens=None, orc=None, scor
         alpha[t] = p / p.sum()
         if bf16_weights:
             alpha[t] = torch.tensor(alpha[t]).float().bfloat16().double().numpy()
+    dropped = 0
+    if capacity is not None:
+        keep = orc_mod.capacity_keep(idx, cfg.E, capacity)
+        alpha = np.where(keep, alpha, 0.0)
+        dropped = int((~keep).sum())
     y_ref = oracle_outputs(orc_mod, inp, idx, alpha, toks, orc["shared_gate"])
     if residual is not None:
         y_ref = y_ref + residual[torch.as_tensor(toks, device=residual.device)].cpu().double().numpy()
@@ -133,4 +140,4 @@ def check_layer(orc_mod, inp, y_gpu, gpu_idx, gpu_w, tokens=None, orc=None, scor
     assert used <= 1.0, (f"output error {err:.3e} exceeds {Y_TOL} x RMS {rms:.3e} + half a bf16 "
                          f"ulp ({used:.2f} of the bound)")
     return dict(near_tie=rep.near_tie, differing=len(rep.differing_sets), w_err=rep.max_w_err,
-                y_err=err, y_rms=rms, y_rel=err / rms, bound_used=used)
+                y_err=err, y_rms=rms, y_rel=err / rms, bound_used=used, dropped=dropped)

@@ -104,6 +104,15 @@ def test_host_validation_returns_before_launch(lib):
     assert L.moe_layer_forward(ctypes.byref(p), _fake(A), ws, 1 << 40, None) == ARG
     p.f_s, p.D = 0, 2000
     assert L.moe_layer_forward(ctypes.byref(p), _fake(A), ws, 1 << 40, None) == UNSUP
+    p.D = 2048
+    for bad in (-1.0, float("nan"), float("inf")):  # capacity factor
+        p.capacity_factor = bad
+        assert L.moe_layer_forward(ctypes.byref(p), _fake(A), ws, 1 << 40, None) == ARG
+    p.capacity_factor, p.min_capacity = 1.25, -1
+    assert L.moe_layer_forward(ctypes.byref(p), _fake(A), ws, 1 << 40, None) == ARG
+    # moe_permute_ex: same checks as moe_permute
+    assert L.moe_permute_ex(_fake(A), None, None, 4, 16, 4, 3, _fake(A), _fake(A), None,
+                            _fake(A), None, None) == ARG
     assert L.moe_read_device_status(None, None) == WS
 
 
@@ -118,3 +127,19 @@ def test_python_binding_needs_cuda_tensors(lib):
     import torch
     with pytest.raises(ValueError):
         moe._p(torch.zeros(4))
+
+
+def test_expert_capacity_matches_oracle(lib, oracle_mod):
+    """The layer's capacity C (host arithmetic of the library) equals the oracle's for the
+    same float capacity factor, over sizes, factors and minimums."""
+    import numpy as np
+    for T, K, E in [(64, 8, 256), (8192, 8, 128), (4096, 10, 512), (1, 8, 128), (1000, 2, 3),
+                    (7, 1, 7), (300, 6, 128), (0, 4, 16)]:
+        for cf in (0.5, 0.75, 1.0, 1.1, 1.25, 2.0, 3.3):
+            cf32 = float(np.float32(cf))
+            for mn in (0, 4, 1000):
+                assert moe.expert_capacity(T, K, E, cf, mn) == \
+                    oracle_mod.expert_capacity(T, K, E, cf32, mn), (T, K, E, cf, mn)
+    assert moe.expert_capacity(64, 8, 256, 0.0) == -1
+    assert moe.expert_capacity(64, 8, 256, -1.0) == -1
+    assert moe.expert_capacity(64, 8, 0, 1.25) == -1

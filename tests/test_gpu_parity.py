@@ -13,14 +13,6 @@ from workloads import CONFIGS, LayerConfig, crafted_routing, make_inputs, random
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(scope="module")
-def moe():
-    import top_routing_grouped_03_b200 as m
-    m.lib()
-    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
-    return m
-
-
 def _np(t):
     return t.detach().cpu().numpy()
 

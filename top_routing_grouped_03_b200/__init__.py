@@ -43,6 +43,7 @@ class LayerParams(ctypes.Structure):
         ("expert_counts_out", ctypes.c_void_p), ("step_events", ctypes.c_void_p),
         ("score_mode", ctypes.c_int), ("select_bias", ctypes.c_void_p),
         ("residual", ctypes.c_void_p),
+        ("capacity_factor", ctypes.c_float), ("min_capacity", ctypes.c_int),
     ]
 
 
@@ -74,6 +75,10 @@ def lib() -> ctypes.CDLL:
         L.moe_route_ex.restype = I
         L.moe_permute.argtypes = [P, P, P, I, I, I, P, P, P, P, P, P]
         L.moe_permute.restype = I
+        L.moe_permute_ex.argtypes = [P, P, P, I, I, I, ctypes.c_longlong, P, P, P, P, P, P]
+        L.moe_permute_ex.restype = I
+        L.moe_expert_capacity.argtypes = [I, I, I, ctypes.c_float, I]
+        L.moe_expert_capacity.restype = ctypes.c_longlong
         L.moe_grouped_swiglu.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P, P, Z, P]
         L.moe_grouped_swiglu.restype = I
         L.moe_combine.argtypes = [P, P, P, P, P, P, I, I, I, P, P]
@@ -174,8 +179,14 @@ def route_noalloc(x, w_router, K, logit_bias=None, w_shared_gate=None, stream=No
     return idx, w, counts, sg
 
 
-def permute(topk_idx, topk_w, expert_counts, E, workspace=None, stream=None):
-    """Permutation step.  Returns dict(offsets [E+1], sorted_token, sorted_w, slot_to_row)."""
+def expert_capacity(T, K, E, capacity_factor, min_capacity=0) -> int:
+    """Assignments per expert the layer keeps (moe_expert_capacity); -1: no capacity."""
+    return int(lib().moe_expert_capacity(T, K, E, float(capacity_factor), int(min_capacity)))
+
+
+def permute(topk_idx, topk_w, expert_counts, E, workspace=None, stream=None, capacity=None):
+    """Permutation step.  Returns dict(offsets [E+1], sorted_token, sorted_w, slot_to_row).
+    ``capacity``: keep each expert's first ``capacity`` entries (moe_permute_ex)."""
     T, K = topk_idx.shape
     dev = topk_idx.device
     off = torch.empty((E + 1,), dtype=torch.int32, device=dev)
@@ -184,9 +195,10 @@ def permute(topk_idx, topk_w, expert_counts, E, workspace=None, stream=None):
     s2r = torch.empty((T * K,), dtype=torch.int32, device=dev)
     if workspace is None and T > 0:
         workspace = alloc_workspace(T, 128, E, K, 128, 0, dev)
-    rc = lib().moe_permute(_p(topk_idx), _p(topk_w), _p(expert_counts), T, E, K, _p(off),
-                           _p(st), _p(sw), _p(s2r), _p(workspace), _stream(stream))
-    _check(rc, "moe_permute")
+    cap = -1 if capacity is None else int(capacity)
+    rc = lib().moe_permute_ex(_p(topk_idx), _p(topk_w), _p(expert_counts), T, E, K, cap,
+                              _p(off), _p(st), _p(sw), _p(s2r), _p(workspace), _stream(stream))
+    _check(rc, "moe_permute_ex")
     return dict(offsets=off, sorted_token=st, sorted_w=sw, slot_to_row=s2r)
 
 
@@ -247,7 +259,8 @@ class MoELayer:
 
     def __init__(self, w_router, w_gate_up, w_down, K, logit_bias=None, w_shared_gate=None,
                  w_shared_gate_up=None, w_shared_down=None, deterministic=False,
-                 score="softmax", select_bias=None, bf16_weights=False):
+                 score="softmax", select_bias=None, bf16_weights=False, capacity_factor=0.0,
+                 min_capacity=0):
         self.w_router, self.w_gate_up, self.w_down = w_router, w_gate_up, w_down
         self.logit_bias = logit_bias
         self.w_shared_gate, self.w_shared_gate_up = w_shared_gate, w_shared_gate_up
@@ -260,6 +273,8 @@ class MoELayer:
             (MOE_FLAG_BF16_WEIGHTS if bf16_weights else 0)
         self.score_mode = SCORES[score]
         self.select_bias = select_bias
+        self.capacity_factor = float(capacity_factor)
+        self.min_capacity = int(min_capacity)
         self._ws = None
         self._ws_T = -1
 
@@ -284,7 +299,8 @@ class MoELayer:
                            _p(self.w_down), _p(self.w_shared_gate), _p(self.w_shared_gate_up),
                            _p(self.w_shared_down), T, self.D, self.E, self.K, self.f, self.f_s,
                            self.flags, _p(topk_idx), _p(topk_w), _p(counts), ev,
-                           self.score_mode, _p(self.select_bias), _p(residual))
+                           self.score_mode, _p(self.select_bias), _p(residual),
+                           self.capacity_factor, self.min_capacity)
 
     def __call__(self, x, out=None, topk_idx=None, topk_w=None, counts=None, stream=None,
                  step_events=None, residual=None):

@@ -4,8 +4,9 @@
 // + sigma(w_s^T x_t) E_s(x_t); section 3.2: the expert outputs are index-added back to
 // their tokens.  One thread owns 8 consecutive features of one token (16-byte loads and
 // stores) and sums, in this fixed order: the fp32 accumulator row (if any), the K routed
-// rows in slot order, the gated shared-expert row, then the decoder residual h (section 4:
-// h_out = h + y); the result is rounded once to bf16 (round to nearest even).
+// rows in slot order (skipping pairs dropped by an expert capacity, slot_to_row = -1), the
+// gated shared-expert row, then the decoder residual h (section 4: h_out = h + y); the
+// result is rounded once to bf16 (round to nearest even).
 #include <algorithm>
 
 #include "common.cuh"
@@ -47,6 +48,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineLaunch a) {
             for (int k = 0; k < a.K; ++k) {
                 const int slot = t * a.K + k;
                 const int row = __ldg(a.slot_to_row + slot);
+                if (row < 0) continue;  // dropped past its expert's capacity
                 const float w = a.topk_w ? __ldg(a.topk_w + slot) : 1.f;
                 const size_t o = 2 * (static_cast<size_t>(row) * vec + c);
                 const float4 lo = __ldg(ys + o), hi = __ldg(ys + o + 1);

@@ -114,6 +114,7 @@ struct PermuteLaunch {
     int32_t* dense_offsets;  // optional [2] = {0, T} for a dense (shared) expert group
     int* status;
     int32_t* hist;           // [permute_chunks(T*K) * E] scratch, or NULL (one CTA)
+    long long capacity;      // >= 0: each expert keeps its first `capacity` entries; < 0: all
 };
 // chunks the permutation cuts T*K entries into (1 at decode sizes, at most 256)
 int permute_chunks(long long entries);

@@ -1,6 +1,7 @@
 // moe_api.cu -- the extern "C" entry points of libmoe_b200.so: argument checks on the
 // host, workspace layout, and the launch sequence of the layer.  See include/moe_api.h.
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -176,6 +177,24 @@ int moe_route_ex(const moe_bf16* x, const moe_bf16* w_router, const float* logit
 int moe_permute(const int32_t* topk_idx, const float* topk_w, const int32_t* expert_counts, int T,
                 int E, int K, int32_t* expert_offsets, int32_t* sorted_token, float* sorted_w,
                 int32_t* slot_to_row, void* workspace, void* stream) {
+    return moe_permute_ex(topk_idx, topk_w, expert_counts, T, E, K, -1, expert_offsets,
+                          sorted_token, sorted_w, slot_to_row, workspace, stream);
+}
+
+long long moe_expert_capacity(int T, int K, int E, float capacity_factor, int min_capacity) {
+    if (T < 0 || K <= 0 || E <= 0 || min_capacity < 0 || !(capacity_factor > 0.f) ||
+        !std::isfinite(capacity_factor))
+        return -1;
+    const double c = std::ceil(static_cast<double>(capacity_factor) * static_cast<double>(T) *
+                               static_cast<double>(K) / static_cast<double>(E));
+    const long long cap = c > 9.0e18 ? static_cast<long long>(9.0e18) : static_cast<long long>(c);
+    return cap < min_capacity ? min_capacity : cap;
+}
+
+int moe_permute_ex(const int32_t* topk_idx, const float* topk_w, const int32_t* expert_counts,
+                   int T, int E, int K, long long capacity, int32_t* expert_offsets,
+                   int32_t* sorted_token, float* sorted_w, int32_t* slot_to_row,
+                   void* workspace, void* stream) {
     int rc = check_shape(T, 128, E, K, 128, 0);
     if (rc) return rc;
     if (!expert_counts || !expert_offsets) return MOE_ERR_ARG;
@@ -192,6 +211,7 @@ int moe_permute(const int32_t* topk_idx, const float* topk_w, const int32_t* exp
     a.slot_to_row = slot_to_row;
     a.status = workspace ? at<int>(workspace, 0) : nullptr;
     a.hist = workspace ? at<int32_t>(workspace, layout(T, 128, E, K, 128, 0).perm_hist) : nullptr;
+    a.capacity = capacity < 0 ? -1 : capacity;
     return launch_permute(a, as_stream(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -274,6 +294,12 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     if (shared && (!p->w_shared_gate || !p->w_shared_gate_up || !p->w_shared_down)) return MOE_ERR_ARG;
     if (!shared && (p->w_shared_gate || p->w_shared_gate_up || p->w_shared_down)) return MOE_ERR_ARG;
     if (p->score_mode != MOE_SCORE_SOFTMAX && p->score_mode != MOE_SCORE_SIGMOID) return MOE_ERR_ARG;
+    if (!(p->capacity_factor >= 0.f) || !std::isfinite(p->capacity_factor) || p->min_capacity < 0)
+        return MOE_ERR_ARG;
+    // expert capacity (assignments per expert), or -1: dropless
+    const long long capacity = p->capacity_factor > 0.f
+                                   ? moe_expert_capacity(T, K, E, p->capacity_factor, p->min_capacity)
+                                   : -1;
     if (!aligned16(p->x) || !aligned16(p->w_router) || !aligned16(p->w_gate_up) ||
         !aligned16(p->w_down) || !aligned16(out) || !aligned16(p->residual) ||
         (shared && (!aligned16(p->w_shared_gate) || !aligned16(p->w_shared_gate_up) ||
@@ -346,6 +372,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     pm.dense_offsets = at<int32_t>(workspace, L.dense_offsets);
     pm.status = status;
     pm.hist = at<int32_t>(workspace, L.perm_hist);
+    pm.capacity = capacity;
     if (!mark(MOE_EV_PERMUTE) || launch_permute(pm, s, true) != cudaSuccess) return MOE_ERR_CUDA;
 
     const int rows = T * K;
@@ -357,7 +384,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     up.gather_buf = at<bf16>(workspace, L.x_sorted);
     up.offsets = pm.offsets;
     up.rows = rows; up.E = E; up.D = D; up.f = f;
-    up.max_group_rows = T;
+    up.max_group_rows = capacity >= 0 && capacity < T ? static_cast<int>(capacity) : T;
     up.h_out = at<bf16>(workspace, L.h);
     up.status = status;
     up.zero_acc = use_acc && tc_router ? out_acc : nullptr;
@@ -373,7 +400,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     dn.sorted_token = pm.sorted_token;
     dn.sorted_w = det ? nullptr : pm.sorted_w;
     dn.rows = rows; dn.E = E; dn.D = D; dn.f = f;
-    dn.max_group_rows = T;
+    dn.max_group_rows = up.max_group_rows;
     dn.acc_out = det ? nullptr : out_acc;
     dn.y_out = det ? at<float>(workspace, L.y_sorted) : nullptr;
     dn.status = status;

@@ -11,7 +11,10 @@
 //   row = offsets[e] + (entries of e in earlier chunks) + (entries of e earlier in this
 //         chunk),
 // offsets being the exclusive scan of the counts -- ascending (token, slot) order inside
-// each group, i.e. a stable counting sort by expert.
+// each group, i.e. a stable counting sort by expert.  With an expert capacity C
+// ("1.6 混合专家（MoE）", section 三, expert capacity and token dropping) an entry whose
+// place in its group is C or more is dropped (slot_to_row = -1) and the groups are the
+// kept prefixes, min(count, C) rows each.
 // The token rows themselves are never copied: the grouped GEMM gathers them from x.
 #include <algorithm>
 
@@ -67,7 +70,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(PermuteLa
     extern __shared__ int sm[];
     int* warp_cnt = sm;                          // [kPermWarps][E]
     int* base = warp_cnt + kPermWarps * a.E;     // [E] entries of e placed before this step
-    int* off = base + a.E;                       // [E + 1]
+    int* off = base + a.E;                       // [E + 1] first row of each (kept) group
+    int* raw = off + a.E + 1;                    // [E] entries of each expert
     __shared__ int warp_sums[kPermWarps];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int E = a.E, total = a.T * a.K;
@@ -105,8 +109,10 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(PermuteLa
         if (c == 0 && a.counts_out && tid < E) a.counts_out[tid] = n;
         __syncthreads();
     }
-    // offsets: exclusive scan of the counts (E <= 512 < kPermThreads)
-    int incl = n;
+    // rows each group keeps: all its entries, or the first `capacity` of them
+    const int kept = (a.capacity >= 0 && n > a.capacity) ? static_cast<int>(a.capacity) : n;
+    // offsets: exclusive scan of the kept counts (E <= 512 < kPermThreads)
+    int incl = kept;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -126,14 +132,17 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(PermuteLa
     }
     __syncthreads();
     if (tid < E) {
-        off[tid] = warp_sums[warp] + incl - n;
+        off[tid] = warp_sums[warp] + incl - kept;
+        raw[tid] = n;
         base[tid] = 0;
         if (c == 0) a.offsets[tid] = off[tid];
+        if (tid == E - 1) {
+            off[E] = warp_sums[warp] + incl;  // rows kept in all (T*K without a capacity)
+            if (c == 0) a.offsets[E] = off[E];
+        }
     }
     if (tid == 0) {
-        off[E] = total;
         if (c == 0) {
-            a.offsets[E] = total;
             if (a.dense_offsets) {
                 a.dense_offsets[0] = 0;
                 a.dense_offsets[1] = a.T;
@@ -141,6 +150,13 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(PermuteLa
         }
     }
     __syncthreads();
+    // with a capacity, rows [kept total, T*K) belong to no group: token 0, weight 0
+    if (c == 0 && a.capacity >= 0) {
+        for (int row = off[E] + tid; row < total; row += kPermThreads) {
+            a.sorted_token[row] = 0;
+            if (a.topk_w) a.sorted_w[row] = 0.f;
+        }
+    }
     // entries of each expert in the chunks before this one
     for (int i = tid; i < c * E; i += kPermThreads) {
         const int v = a.hist[i];
@@ -170,22 +186,26 @@ __global__ void __launch_bounds__(kPermThreads) permute_scatter_kernel(PermuteLa
         }
         __syncthreads();
         if (ok) {
-            const int row = off[e] + warp_cnt[warp * E + e] + rank;
-            // counts that disagree with the entries can push a row out of its group, or
-            // (when they do not sum to T*K) out of the arrays: flag it, write nothing
-            if (row >= 0 && row < off[e + 1] && row < total) {
-                a.sorted_token[row] = j / a.K;
-                if (a.topk_w) a.sorted_w[row] = __ldg(a.topk_w + j);
-                a.slot_to_row[j] = row;
+            const int in_group = warp_cnt[warp * E + e] + rank;  // entries of e before it
+            if (a.capacity >= 0 && in_group >= a.capacity) {
+                a.slot_to_row[j] = -1;  // past the expert's capacity: dropped
             } else {
-                set_status(a.status, MOE_ERR_DEVICE);
+                const int row = off[e] + in_group;
+                // counts that disagree with the entries can push a row out of its group,
+                // or (when they do not sum to T*K) out of the arrays: flag it, write nothing
+                if (row >= 0 && row < off[e + 1] && row < total) {
+                    a.sorted_token[row] = j / a.K;
+                    if (a.topk_w) a.sorted_w[row] = __ldg(a.topk_w + j);
+                    a.slot_to_row[j] = row;
+                } else {
+                    set_status(a.status, MOE_ERR_DEVICE);
+                }
             }
         }
         __syncthreads();
     }
-    // the last chunk has seen every entry: each group must be exactly full
-    if (c == chunks - 1 && tid < E && base[tid] != off[tid + 1] - off[tid])
-        set_status(a.status, MOE_ERR_DEVICE);
+    // the last chunk has seen every entry: each expert's entries must match its count
+    if (c == chunks - 1 && tid < E && base[tid] != raw[tid]) set_status(a.status, MOE_ERR_DEVICE);
 }
 
 
@@ -227,7 +247,7 @@ cudaError_t launch_permute(const PermuteLaunch& a, cudaStream_t s, bool pdl) {
         count_launches(1);
         if (err != cudaSuccess) return err;
     }
-    const size_t smem = sizeof(int) * (static_cast<size_t>(kPermWarps) * a.E + 2 * a.E + 1);
+    const size_t smem = sizeof(int) * (static_cast<size_t>(kPermWarps) * a.E + 3 * a.E + 1);
     err = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
