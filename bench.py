@@ -20,6 +20,7 @@ import argparse
 import datetime
 import hashlib
 import json
+import re
 import os
 import statistics
 import subprocess
@@ -80,11 +81,20 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without comments and with whitespace collapsed: an edit to a comment
+    does not change the kernel the profiler measured."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash() -> str:
+    """Identifies the grouped GEMM kernels' source (code only) that a profile was taken on."""
     h = hashlib.sha256()
     for f in ("grouped_gemm.cu", "ptx.cuh", "common.cuh"):
-        with open(os.path.join(ROOT, "top_routing_grouped_03_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "top_routing_grouped_03_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode("utf-8"))
     return h.hexdigest()[:16]
 
 

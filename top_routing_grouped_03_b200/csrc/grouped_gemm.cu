@@ -6,24 +6,31 @@
 // token.  "MoE 到底省了什么" (clxhxhhr.top), section 3: with few rows per expert the
 // layer is bound by reading the expert weights, with many rows it is bound by compute.
 //
-// Both projections run through one persistent, warp-specialised kernel template:
-//   * operand A = 128 weight rows x 64 K (TMA, 128-byte swizzle) -- the MMA's M side,
-//     so an expert with only a couple of rows still fills the 128-lane tensor-core tile
-//     ("swap-AB": weights on M, tokens on N);
-//   * operand B = BN rows of activations in expert order x 64 K (TMA);
-//   * D = fp32 accumulator in tensor memory, 128 lanes (features) x BN columns (rows);
-//     the gate_up kernel keeps the gate block in columns [0, BN) and the up block in
-//     [BN, 2BN) so one thread holds gate and up of the same feature;
-//   * two accumulator buffers so the epilogue of one tile overlaps the MMAs of the next.
-// Warp 0 issues TMA loads into a STAGES-deep ring, warp 1 issues tcgen05.mma (one
-// thread) and owns the TMEM allocation, warps 2-5 drain TMEM (tcgen05.ld) and run the
-// epilogue: h = SiLU(g) * u -> bf16 for gate_up; w * v -> fp32 red.add into the token's
-// output row (and/or fp32 y_sorted) for down.  When the gate_up rows are tokens of x in
-// expert order, the producer warp gathers them itself with cp.async (16-byte chunks
-// written in the 128-byte swizzle the MMA descriptor expects), so no permuted copy of x is
-// ever materialised.
-// The work list (group, feature block, row block) is derived on the device from the
-// group offsets, so no host synchronisation is needed.  Every wait is bounded.
+// Three persistent, warp-specialised kernels share one structure: warp 0 fills a ring of
+// shared-memory stages (TMA, 128-byte swizzle, 64-deep K steps), warp 1 owns the tensor
+// memory and one of its threads issues tcgen05.mma (bf16 in, fp32 accumulate), and the
+// epilogue warps drain a double-buffered TMEM accumulator with tcgen05.ld while the next
+// tile accumulates.  Epilogues: h = SiLU(g) * u -> bf16 for gate_up; w * v -> fp32
+// reductions into the token's output row (and/or fp32 y_sorted) for down.  The work list
+// (group, feature block, row block) is derived on the device from the group offsets, so no
+// host synchronisation is needed, and every wait is bounded.
+//   * grouped_gemm_kernel<BN, GATE_UP>, weights on M: 128 weight rows x BN token rows
+//     (16..128), for groups of a handful of rows -- an expert with two rows still fills
+//     the 128-lane tile.  gate_up keeps the gate block in accumulator columns [0, BN) and
+//     the up block in [BN, 2BN) so one thread holds both halves of a feature.  Also the
+//     router's logits GEMM (one dense group, the reduction split into partial planes).
+//   * grouped_gemm_tm_kernel<GATE_UP>, tokens on M: 128 token rows x 256 weight rows (128
+//     gate + 128 up features, or 256 output features), 8 epilogue warps; features lie
+//     along the accumulator's columns, so h leaves as 16-byte stores and the down results
+//     as 4-wide vector reductions.
+//   * grouped_gemm_pair_kernel<GATE_UP>, CTA pairs: clusters of two with
+//     tcgen05.mma.cta_group::2 over 256 token rows x 256 weight rows, each CTA loading its
+//     own token rows and half of the weights (.cta_group::2 TMA, no multicast), commits
+//     multicast to both CTAs' barriers; its token rows must be contiguous, so gate_up
+//     reads an expert-ordered copy of x.
+// The other two kernels gather gate_up's token rows themselves: the producer warp's lanes
+// copy 16-byte chunks of x[token] with cp.async into the 128-byte swizzle the MMA
+// descriptor expects, zero-filling rows past the group.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
