@@ -39,6 +39,18 @@ SMALL_LAYERS = {
     "dense_E1": LayerConfig("dense_E1", T=33, D=256, E=1, K=1, f=384, seed=5),
     "all_experts": LayerConfig("all_experts", T=50, D=256, E=8, K=8, f=128, seed=6),
     "hot_rows": LayerConfig("hot_rows", T=300, D=256, E=4, K=2, f=128, seed=7),
+    # few tiles with deep reductions (D = 1024 for gate_up, f = 1024 for down), routed and
+    # shared
+    "deep_gate_up": LayerConfig("deep_gate_up", T=40, D=1024, E=8, K=2, f=256, seed=10),
+    "deep_down": LayerConfig("deep_down", T=48, D=512, E=4, K=2, f=1024, seed=11),
+    "deep_shared": LayerConfig("deep_shared", T=40, D=1024, E=8, K=2, f=256, f_s=512,
+                               seed=12),
+    # the largest sizes the library takes: K = 16 of E = 512 experts (16 logits per lane
+    # in the selection, 512 groups), D = 8192 (128 KiB of staged tokens in the router,
+    # 128 K steps), f = 8192 (64 feature blocks, 128 K steps in down)
+    "max_k_e": LayerConfig("max_k_e", T=70, D=256, E=512, K=16, f=128, seed=13),
+    "max_d": LayerConfig("max_d", T=24, D=8192, E=8, K=2, f=128, seed=14),
+    "max_f": LayerConfig("max_f", T=24, D=256, E=4, K=2, f=8192, seed=15),
     # at most 16 tokens: weights-on-M grouped GEMMs, routed and shared
     "few_tokens_shared": LayerConfig("few_tokens_shared", T=12, D=256, E=32, K=4, f=256,
                                      f_s=128, seed=9),
@@ -232,7 +244,8 @@ def test_layer_matches_oracle(moe, oracle_mod, name):
     print(name, rep)
 
 
-@pytest.mark.parametrize("name", ["tiny", "decode", "shared_small", "ragged_T"])
+@pytest.mark.parametrize("name", ["tiny", "decode", "shared_small", "ragged_T", "deep_gate_up",
+                                  "deep_down", "deep_shared"])
 def test_layer_deterministic_mode(moe, oracle_mod, name):
     inp = make_inputs(SMALL_LAYERS[name]).to("cuda")
     layer, y1, idx, w, _ = _run_layer(moe, inp, deterministic=True)
