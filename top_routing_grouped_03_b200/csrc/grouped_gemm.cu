@@ -528,7 +528,7 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 // columns [128 half, 128 half + 128) of its 256).  The warp's 32 lanes are 32 rows.
 template <bool GATE_UP>
 __device__ __forceinline__ void tm_epilogue(const Params& p, uint32_t tbase, int row, bool valid,
-                                            int tile_i, int half) {
+                                            int tile_i, int half, float* stage) {
     if (GATE_UP) {
         bf16* hrow = p.h_out + static_cast<size_t>(row) * p.out_cols + tile_i * kBM + half * 64;
 #pragma unroll 1
@@ -557,31 +557,66 @@ __device__ __forceinline__ void tm_epilogue(const Params& p, uint32_t tbase, int
         const float w = (valid && p.sorted_w) ? __ldg(p.sorted_w + row) : 1.f;
         const int tok = valid ? (p.sorted_token ? __ldg(p.sorted_token + row) : row) : 0;
         const int col0 = tile_i * kTmN + half * 128;
+        const int lane = threadIdx.x & 31;
+        if (p.acc_out) {
+            // Reductions into the token rows, 16 columns at a time.  A thread holds one
+            // row; a 4-wide reduction per thread and row would touch 32 rows' lines with 16
+            // bytes each.  So the warp's 32 rows x 16 columns go through shared memory
+            // (`stage`, 2 KB, 16-byte chunks XOR-swizzled so that both the row-wise writes
+            // and the transposed reads are free of bank conflicts) and each reduction
+            // instruction then covers 8 rows x 64 contiguous bytes: whole 32-byte sectors.
+            const int rr0 = lane >> 2, kq = lane & 3;  // read side: row (of 8), chunk
 #pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 32) {
+            for (int c0 = 0; c0 < 128; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld16(tbase + half * 128 + c0, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    *reinterpret_cast<float4*>(stage + lane * 16 + ((k ^ ((lane >> 1) & 3)) << 2)) =
+                        make_float4(w * __uint_as_float(v[4 * k]), w * __uint_as_float(v[4 * k + 1]),
+                                    w * __uint_as_float(v[4 * k + 2]), w * __uint_as_float(v[4 * k + 3]));
+                __syncwarp();
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {
+                    const int rr = it * 8 + rr0;
+                    const float4 val = *reinterpret_cast<const float4*>(
+                        stage + rr * 16 + ((kq ^ ((rr >> 1) & 3)) << 2));
+                    const int tok_r = __shfl_sync(0xffffffffu, tok, rr);
+                    const bool valid_r = __shfl_sync(0xffffffffu, valid ? 1 : 0, rr) != 0;
+                    if (valid_r)
+                        red_add_v4(p.acc_out + static_cast<size_t>(tok_r) * p.out_cols + col0 + c0 +
+                                       4 * kq,
+                                   val.x, val.y, val.z, val.w);
+                }
+                __syncwarp();
+            }
+        }
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128 && p.y_out; c0 += 32) {
             uint32_t v[32];
             tmem_ld32(tbase + half * 128 + c0, v);
             tmem_ld_wait();
             if (valid) {
-                if (p.acc_out) {
-                    float* dst = p.acc_out + static_cast<size_t>(tok) * p.out_cols + col0 + c0;
+                float4* dst = reinterpret_cast<float4*>(
+                    p.y_out + static_cast<size_t>(row) * p.out_cols + col0 + c0);
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        red_add_v4(dst + j, w * __uint_as_float(v[j]), w * __uint_as_float(v[j + 1]),
-                                   w * __uint_as_float(v[j + 2]), w * __uint_as_float(v[j + 3]));
-                }
-                if (p.y_out) {
-                    float4* dst = reinterpret_cast<float4*>(
-                        p.y_out + static_cast<size_t>(row) * p.out_cols + col0 + c0);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        dst[j] = make_float4(w * __uint_as_float(v[4 * j]), w * __uint_as_float(v[4 * j + 1]),
-                                             w * __uint_as_float(v[4 * j + 2]),
-                                             w * __uint_as_float(v[4 * j + 3]));
-                }
+                for (int j = 0; j < 8; ++j)
+                    dst[j] = make_float4(w * __uint_as_float(v[4 * j]), w * __uint_as_float(v[4 * j + 1]),
+                                         w * __uint_as_float(v[4 * j + 2]),
+                                         w * __uint_as_float(v[4 * j + 3]));
             }
         }
     }
+}
+
+// down epilogue staging of the tokens-on-M kernels: 2 KB per epilogue warp, after the
+// group table
+constexpr int kStageFloatsPerWarp = 32 * 16;
+constexpr size_t kEpiStageBytes = 16 + (kTmEpiThreads / 32) * kStageFloatsPerWarp * sizeof(float);
+__device__ __forceinline__ float* epi_stage(int* table_end, int warp) {
+    const uintptr_t a = (reinterpret_cast<uintptr_t>(table_end) + 15) & ~static_cast<uintptr_t>(15);
+    return reinterpret_cast<float*>(a) + (warp - 2) * kStageFloatsPerWarp;
 }
 
 template <bool GATE_UP>
@@ -765,7 +800,8 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    abuf * C::kAccCols;
             const int row = t.row0 + q * 32 + lane;
-            tm_epilogue<GATE_UP>(p, tbase, row, row < t.row_end, t.i, (warp - 2) >> 2);
+            tm_epilogue<GATE_UP>(p, tbase, row, row < t.row_end, t.i, (warp - 2) >> 2,
+                                 GATE_UP ? nullptr : epi_stage(g_tile + p.G + 1, warp));
             tc_fence_before();
             mbar_arrive(&tempty[abuf]);
             abuf ^= 1u;
@@ -960,7 +996,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_w,
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    abuf * C::kAccCols;
             const int row = t.row0 + static_cast<int>(rank) * kTmRows + q * 32 + lane;
-            tm_epilogue<GATE_UP>(p, tbase, row, row < t.row_end, t.i, (warp - 2) >> 2);
+            tm_epilogue<GATE_UP>(p, tbase, row, row < t.row_end, t.i, (warp - 2) >> 2,
+                                 GATE_UP ? nullptr : epi_stage(g_tile + p.G + 1, warp));
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_tempty0 + abuf * 8);
@@ -1030,7 +1067,8 @@ cudaError_t launch_tm(const CUtensorMap& mw, const CUtensorMap& ma, const Params
                       cudaStream_t s, bool pdl) {
     using C = CfgTm<GATE_UP>;
     const size_t smem = 1024 + static_cast<size_t>(C::kStages) * C::kStageBytes +
-                        (2 * C::kStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int);
+                        (2 * C::kStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int) +
+                        (GATE_UP ? 0 : kEpiStageBytes);
     auto kfn = grouped_gemm_tm_kernel<GATE_UP>;
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
@@ -1045,7 +1083,8 @@ cudaError_t launch_pair(const CUtensorMap& mw, const CUtensorMap& ma, const Para
                         int npairs, cudaStream_t s, bool pdl) {
     using C = CfgPair;
     const size_t smem = 1024 + static_cast<size_t>(C::kStages) * C::kStageBytes +
-                        (2 * C::kStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int);
+                        (2 * C::kStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int) +
+                        (GATE_UP ? 0 : kEpiStageBytes);
     auto kfn = grouped_gemm_pair_kernel<GATE_UP>;
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
