@@ -558,7 +558,24 @@ __device__ __forceinline__ void tm_epilogue(const Params& p, uint32_t tbase, int
         const int tok = valid ? (p.sorted_token ? __ldg(p.sorted_token + row) : row) : 0;
         const int col0 = tile_i * kTmN + half * 128;
         const int lane = threadIdx.x & 31;
-        if (p.acc_out) {
+        // a warp with a handful of rows (a few tokens per expert) reduces row by row: the
+        // transpose below would move 32 rows through shared memory for 2 or 3 of them
+        const bool sparse = __popc(__ballot_sync(0xffffffffu, valid)) <= 4;
+        if (p.acc_out && sparse) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < 128; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(tbase + half * 128 + c0, v);
+                tmem_ld_wait();
+                if (valid) {
+                    float* dst = p.acc_out + static_cast<size_t>(tok) * p.out_cols + col0 + c0;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        red_add_v4(dst + j, w * __uint_as_float(v[j]), w * __uint_as_float(v[j + 1]),
+                                   w * __uint_as_float(v[j + 2]), w * __uint_as_float(v[j + 3]));
+                }
+            }
+        } else if (p.acc_out) {
             // Reductions into the token rows, 16 columns at a time.  A thread holds one
             // row; a 4-wide reduction per thread and row would touch 32 rows' lines with 16
             // bytes each.  So the warp's 32 rows x 16 columns go through shared memory
