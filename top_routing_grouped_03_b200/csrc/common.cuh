@@ -81,8 +81,8 @@ struct RouterLaunch {
                           // permutation derives them, tensor-core path)
     float* shared_gate;
     int* status;
-    // optional: rows [T, zero_cols] of zero_acc are cleared by the router kernel (the
-    // layer's fp32 accumulator)
+    // optional: rows [T, zero_cols] of zero_acc are cleared by the CUDA-core router kernel
+    // (the layer's fp32 accumulator); the tensor-core path leaves it to the gate_up kernel
     float* zero_acc;
     int zero_cols;
     int score_mode;           // 0: softmax over the experts; 1: per-expert sigmoid

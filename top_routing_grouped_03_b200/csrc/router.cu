@@ -288,20 +288,16 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
 }
 
 
-// Selection after the tensor-core logits: one warp per token over logits [T, E] (no bias
-// yet), the bias added on load; the shared gate's dot product w_s . x_t is done here by
-// the same warp; the block also clears its tokens' rows of the layer accumulator.
+// Selection after the tensor-core logits: one warp per token over the partial logit
+// planes (no bias yet), the planes added in order and the bias on load; the shared gate's
+// dot product w_s . x_t is done here by the same warp.  (The layer's accumulator is
+// cleared by the gate_up kernel on this path.)
 __global__ void __launch_bounds__(kRouterThreads) router_select_kernel(RouterLaunch a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = blockIdx.x * (kRouterThreads / 32);
     const int nt = min(kRouterThreads / 32, a.T - t0);
     grid_dep_wait();  // logits come from the GEMM
     grid_dep_launch();
-    if (a.zero_acc) {
-        float4* dst = reinterpret_cast<float4*>(a.zero_acc + static_cast<size_t>(t0) * a.zero_cols);
-        for (int i = threadIdx.x; i < nt * a.zero_cols / 4; i += kRouterThreads)
-            dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
     if (warp >= nt) return;
     const int token = t0 + warp;
     select_topk_warp(a.logits + static_cast<size_t>(token) * a.E, a.logit_planes,
