@@ -129,6 +129,19 @@ def test_python_binding_needs_cuda_tensors(lib):
         moe._p(torch.zeros(4))
 
 
+def test_python_binding_checks_element_types(lib):
+    """A tensor of another element type than the C ABI reads at that pointer is refused
+    (checked before anything touches the device)."""
+    import torch
+    with pytest.raises(TypeError):
+        moe._p(torch.zeros(4), moe.BF16)
+    with pytest.raises(TypeError):
+        moe._p(torch.zeros(4, dtype=torch.int64), moe.I32)
+    with pytest.raises(TypeError):
+        moe.combine(2, 128, 1, out=torch.empty((2, 128), dtype=torch.bfloat16),
+                    out_acc=torch.zeros((2, 128), dtype=torch.float64))
+
+
 def test_expert_capacity_matches_oracle(lib, oracle_mod):
     """The layer's capacity C (host arithmetic of the library) equals the oracle's for the
     same float capacity factor, over sizes, factors and minimums."""

@@ -108,9 +108,16 @@ def _check(rc: int, what: str):
         raise MoEError(rc, what)
 
 
-def _p(t: Optional[torch.Tensor]):
+BF16, F32, I32, U8 = torch.bfloat16, torch.float32, torch.int32, torch.uint8
+
+
+def _p(t: Optional[torch.Tensor], dtype: Optional[torch.dtype] = None):
+    """Device pointer of a contiguous CUDA tensor (None -> NULL), of the element type the
+    C ABI reads there when ``dtype`` is given."""
     if t is None:
         return None
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"expected a {dtype} tensor, got {t.dtype}")
     if not t.is_cuda:
         raise ValueError("expected a CUDA tensor")
     if not t.is_contiguous():
@@ -150,14 +157,15 @@ def route(x, w_router, K, logit_bias=None, w_shared_gate=None, workspace=None, s
     counts = torch.empty((E,), dtype=torch.int32, device=dev)
     sg = torch.empty((T,), dtype=torch.float32, device=dev) if w_shared_gate is not None else None
     if score == "softmax" and select_bias is None and not bf16_weights:
-        rc = lib().moe_route(_p(x), _p(w_router), _p(logit_bias), _p(w_shared_gate), T, D, E, K,
-                             _p(idx), _p(w), _p(counts), _p(sg), _p(ws), ws.numel(),
-                             _stream(stream))
+        rc = lib().moe_route(_p(x, BF16), _p(w_router, BF16), _p(logit_bias, F32),
+                             _p(w_shared_gate, BF16), T, D, E, K, _p(idx), _p(w), _p(counts),
+                             _p(sg), _p(ws, U8), ws.numel(), _stream(stream))
     else:
-        rc = lib().moe_route_ex(_p(x), _p(w_router), _p(logit_bias), _p(w_shared_gate), T, D, E,
-                                K, SCORES[score], _p(select_bias),
+        rc = lib().moe_route_ex(_p(x, BF16), _p(w_router, BF16), _p(logit_bias, F32),
+                                _p(w_shared_gate, BF16), T, D, E, K, SCORES[score],
+                                _p(select_bias, F32),
                                 MOE_FLAG_BF16_WEIGHTS if bf16_weights else 0, _p(idx), _p(w),
-                                _p(counts), _p(sg), _p(ws), ws.numel(), _stream(stream))
+                                _p(counts), _p(sg), _p(ws, U8), ws.numel(), _stream(stream))
     _check(rc, "moe_route")
     return idx, w, counts, sg
 
@@ -173,8 +181,9 @@ def route_noalloc(x, w_router, K, logit_bias=None, w_shared_gate=None, stream=No
     w = torch.empty((T, K), dtype=torch.float32, device=dev)
     counts = torch.empty((E,), dtype=torch.int32, device=dev)
     sg = torch.empty((T,), dtype=torch.float32, device=dev) if w_shared_gate is not None else None
-    rc = lib().moe_route_noalloc(_p(x), _p(w_router), _p(logit_bias), _p(w_shared_gate), T, D,
-                                 E, K, _p(idx), _p(w), _p(counts), _p(sg), _stream(stream))
+    rc = lib().moe_route_noalloc(_p(x, BF16), _p(w_router, BF16), _p(logit_bias, F32),
+                                 _p(w_shared_gate, BF16), T, D, E, K, _p(idx), _p(w),
+                                 _p(counts), _p(sg), _stream(stream))
     _check(rc, "moe_route_noalloc")
     return idx, w, counts, sg
 
@@ -196,8 +205,9 @@ def permute(topk_idx, topk_w, expert_counts, E, workspace=None, stream=None, cap
     if workspace is None and T > 0:
         workspace = alloc_workspace(T, 128, E, K, 128, 0, dev)
     cap = -1 if capacity is None else int(capacity)
-    rc = lib().moe_permute_ex(_p(topk_idx), _p(topk_w), _p(expert_counts), T, E, K, cap,
-                              _p(off), _p(st), _p(sw), _p(s2r), _p(workspace), _stream(stream))
+    rc = lib().moe_permute_ex(_p(topk_idx, I32), _p(topk_w, F32), _p(expert_counts, I32), T, E,
+                              K, cap, _p(off), _p(st), _p(sw), _p(s2r), _p(workspace, U8),
+                              _stream(stream))
     _check(rc, "moe_permute_ex")
     return dict(offsets=off, sorted_token=st, sorted_w=sw, slot_to_row=s2r)
 
@@ -211,9 +221,10 @@ def grouped_swiglu(x, sorted_token, offsets, sorted_w, w_gate_up, w_down, rows,
     if workspace is None:
         Kr = max(1, -(-rows // max(T, 1)))
         workspace = alloc_workspace(max(T, 1), D, E, min(Kr, E, 16), f, 0, x.device)
-    rc = lib().moe_grouped_swiglu(_p(x), _p(sorted_token), _p(offsets), _p(sorted_w),
-                                  _p(w_gate_up), _p(w_down), T, rows, D, E, f, _p(y_sorted),
-                                  _p(out_acc), _p(workspace), workspace.numel(), _stream(stream))
+    rc = lib().moe_grouped_swiglu(_p(x, BF16), _p(sorted_token, I32), _p(offsets, I32),
+                                  _p(sorted_w, F32), _p(w_gate_up, BF16), _p(w_down, BF16), T,
+                                  rows, D, E, f, _p(y_sorted, F32), _p(out_acc, F32),
+                                  _p(workspace, U8), workspace.numel(), _stream(stream))
     _check(rc, "moe_grouped_swiglu")
 
 
@@ -221,8 +232,9 @@ def combine(T, D, K, out=None, out_acc=None, y_sorted=None, slot_to_row=None, to
             shared_out=None, shared_gate=None, device=None, stream=None):
     dev = device or "cuda"
     out = out if out is not None else torch.empty((T, D), dtype=torch.bfloat16, device=dev)
-    rc = lib().moe_combine(_p(out_acc), _p(y_sorted), _p(slot_to_row), _p(topk_w),
-                           _p(shared_out), _p(shared_gate), T, D, K, _p(out), _stream(stream))
+    rc = lib().moe_combine(_p(out_acc, F32), _p(y_sorted, F32), _p(slot_to_row, I32),
+                           _p(topk_w, F32), _p(shared_out, BF16), _p(shared_gate, F32), T, D, K,
+                           _p(out, BF16), _stream(stream))
     _check(rc, "moe_combine")
     return out
 
@@ -295,12 +307,13 @@ class MoELayer:
                residual=None) -> LayerParams:
         T = x.shape[0]
         ev = None if events is None else ctypes.cast(events, ctypes.c_void_p)
-        return LayerParams(_p(x), _p(self.w_router), _p(self.logit_bias), _p(self.w_gate_up),
-                           _p(self.w_down), _p(self.w_shared_gate), _p(self.w_shared_gate_up),
-                           _p(self.w_shared_down), T, self.D, self.E, self.K, self.f, self.f_s,
-                           self.flags, _p(topk_idx), _p(topk_w), _p(counts), ev,
-                           self.score_mode, _p(self.select_bias), _p(residual),
-                           self.capacity_factor, self.min_capacity)
+        return LayerParams(_p(x, BF16), _p(self.w_router, BF16), _p(self.logit_bias, F32),
+                           _p(self.w_gate_up, BF16), _p(self.w_down, BF16),
+                           _p(self.w_shared_gate, BF16), _p(self.w_shared_gate_up, BF16),
+                           _p(self.w_shared_down, BF16), T, self.D, self.E, self.K, self.f,
+                           self.f_s, self.flags, _p(topk_idx, I32), _p(topk_w, F32),
+                           _p(counts, I32), ev, self.score_mode, _p(self.select_bias, F32),
+                           _p(residual, BF16), self.capacity_factor, self.min_capacity)
 
     def __call__(self, x, out=None, topk_idx=None, topk_w=None, counts=None, stream=None,
                  step_events=None, residual=None):
@@ -313,7 +326,7 @@ class MoELayer:
                                                       device=x.device)
         ws = self.workspace(T)
         prm = self.params(x, topk_idx, topk_w, counts, step_events, residual)
-        rc = lib().moe_layer_forward(ctypes.byref(prm), _p(out), _p(ws), ws.numel(),
+        rc = lib().moe_layer_forward(ctypes.byref(prm), _p(out, BF16), _p(ws, U8), ws.numel(),
                                      _stream(stream))
         _check(rc, "moe_layer_forward")
         return out
