@@ -287,10 +287,14 @@ enum {
 /*
  * The whole layer: route, permute, grouped SwiGLU (routed experts and, when present, the
  * shared expert scaled by sigma(w_s . x)), combine to out [T, D] bf16 -- plus the residual
- * h when p->residual is set ("MoE", section 4: h_out = h + y_MoE).  No host
- * synchronisation; every step reads its sizes from the device, so the call can be
- * captured in a CUDA graph.  workspace: at least moe_workspace_size(T, D, E, K, f, f_s)
- * bytes, 256-byte aligned.
+ * h when p->residual is set ("MoE", section 4: h_out = h + y_MoE), with the router
+ * variants of p->score_mode / p->select_bias / MOE_FLAG_BF16_WEIGHTS and the expert
+ * capacity of p->capacity_factor when it is > 0.  No host synchronisation; every step
+ * reads its sizes from the device, so the call can be captured in a CUDA graph.
+ * workspace: at least moe_workspace_size(T, D, E, K, f, f_s) bytes, 256-byte aligned.
+ * Errors: MOE_ERR_ARG / _UNSUPPORTED / _ALIGN / _WORKSPACE from the host checks before
+ * anything is enqueued; MOE_ERR_CUDA when a launch fails; device-side problems are left
+ * in the workspace's status word (moe_read_device_status).
  */
 MOE_API int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
                       size_t ws_bytes, void* stream);
