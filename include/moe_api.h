@@ -295,6 +295,10 @@ enum {
  * Errors: MOE_ERR_ARG / _UNSUPPORTED / _ALIGN / _WORKSPACE from the host checks before
  * anything is enqueued; MOE_ERR_CUDA when a launch fails; device-side problems are left
  * in the workspace's status word (moe_read_device_status).
+ * Concurrency: the kernels are persistent (one CTA, or CTA pair, per SM) and the last one
+ * converts the output after a grid-wide step that needs all of its CTAs resident; work
+ * that holds SMs for seconds on other streams can make that step give up after its 2 s
+ * bound, leaving MOE_ERR_TIMEOUT in the status word instead of hanging.
  */
 MOE_API int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
                       size_t ws_bytes, void* stream);
