@@ -9,8 +9,8 @@
  *   alpha_te = p_te / sum_{j in I_t} p_tj              renormalised routing weights
  *   E_e(x)   = W_down^e (SiLU(W_gate^e x) (.) W_up^e x)
  *   y_t      = sum_{e in I_t} alpha_te E_e(x_t) + sigma(w_s^T x_t) E_s(x_t)
- * The shared expert term is optional.  The residual add h + y of the decoder layer is
- * not part of this library.
+ * The shared expert term is optional.  moe_layer_forward can also add the decoder
+ * layer's residual h (h_out = h + y, "MoE", section 4) before its single bf16 rounding.
  *
  * Conventions that hold for every entry point:
  *   - Every pointer argument is a DEVICE pointer unless stated otherwise.  The caller
@@ -122,11 +122,16 @@ MOE_API int moe_route_ex(const moe_bf16* x, const moe_bf16* w_router, const floa
                          float* shared_gate, void* workspace, size_t ws_bytes, void* stream);
 
 /*
- * moe_route_noalloc: the router of moe_route (same kernel, same outputs, same argument
- * rules) for callers that cannot allocate device memory: code hosted by a framework that
- * owns every device allocation and hands its plugins no allocator, or latency-critical
- * code that cannot afford the device-wide synchronisation of cudaMalloc/cudaFree.  The
- * source pages have no counterpart to this entry point; it exists only for such callers.
+ * moe_route_noalloc: the router step of moe_route (same outputs, same argument rules)
+ * for callers that cannot allocate device memory: code hosted by a framework that owns
+ * every device allocation and hands its plugins no allocator, or latency-critical code
+ * that cannot afford the device-wide synchronisation of cudaMalloc/cudaFree.  The source
+ * pages have no counterpart to this entry point; it exists only for such callers.
+ *   - It always runs the CUDA-core router kernel.  moe_route runs that same kernel except
+ *     for T >= 256 with E a multiple of 128, where it takes the logits from the tensor
+ *     cores; there the two sum the logits in different orders, so they agree within the
+ *     router's parity tolerances (identical experts except on near-tie tokens, weights
+ *     within 1e-3), not bit for bit.
  *   - No workspace argument.  The router's scratch (fp32 logits [T, E+1] and one ticket
  *     per 8 tokens) lives in a 1 MiB array that the library declares in device memory;
  *     every GPU that loads the library holds that 1 MiB until the process exits.
@@ -134,7 +139,11 @@ MOE_API int moe_route_ex(const moe_bf16* x, const moe_bf16* w_router, const floa
  *     (for example T <= 1019 at E = 256, T <= 2030 at E = 128); larger calls return
  *     MOE_ERR_UNSUPPORTED before anything is enqueued.
  *   - The first call on a device looks up the array's device address (once per device,
- *     with that device current); make that first call before any stream capture.
+ *     with that device current) and keeps it for the life of the process; make that first
+ *     call before any stream capture.  Calls after a cudaDeviceReset of that device are
+ *     not supported (the array may then live at another address).
+ *   - There is no workspace, hence no device status word: nothing is recorded for
+ *     moe_read_device_status (the router kernel has no device-side error to report).
  *   - Every call on a device shares the one array and it keeps the last call's contents:
  *     the call clears the tickets itself, but calls whose work overlaps on the GPU (other
  *     streams, other host threads) race on the array and must be serialised by the caller.
@@ -305,6 +314,20 @@ MOE_API int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* wo
 
 /* Kernels this library has launched in this process so far (all devices, all calls). */
 MOE_API unsigned long long moe_launch_count(void);
+
+/*
+ * Bound of the layer's grid-wide wait, in nanoseconds (failure detection; no counterpart on
+ * the source pages).  The last kernel of moe_layer_forward converts the output only after
+ * every CTA of its grid has added its tiles: each CTA takes a ticket and waits for the
+ * others for at most this long, and a CTA that gives up records MOE_ERR_TIMEOUT in the
+ * workspace's status word and returns without converting its share of the output.
+ * Applies to the layer calls enqueued after it, on every device (a CUDA graph keeps the
+ * value it was captured with); returns the previous bound.  Default 2000000000 (2 s).
+ * 0 makes every CTA but the last to arrive give up at its first look: a way to drive the
+ * timeout path, and its report, without a hung or faulted GPU.  The waits inside the
+ * kernels' copy/MMA pipelines keep their own fixed 2 s bound.
+ */
+MOE_API unsigned long long moe_set_grid_wait_budget_ns(unsigned long long ns);
 
 /*
  * Synchronously reads (and clears) the device status word of a workspace after the

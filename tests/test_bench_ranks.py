@@ -56,7 +56,8 @@ def test_single_process_is_identity():
 def test_reference_arm_other_ranks_exit_without_work():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--steps", "3", "--warmup", "3"], env=env, capture_output=True,
+                        "--gpus", "2", "--steps", "3", "--warmup", "3"], env=env,
+                       capture_output=True,
                        text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == ""
 
@@ -81,3 +82,30 @@ def test_reference_arm_prints_the_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 2
     assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["config"]["workload"].startswith("tiny")
+
+
+def test_gpus_flag_spawns_that_many_ranks():
+    """`bench.py --gpus 2` without a launcher starts 2 ranks itself (torchrun on 127.0.0.1);
+    in the CPU check mode they join a gloo group and rank 0 prints one line for the job,
+    built from the slowest rank's time (rank r reports steps * (1 + r/2) ms)."""
+    import json
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                        "--dry-run", "--steps", "3", "--warmup", "3"], env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["dry_run"] is True
+    assert d["ms_per_step"] == pytest.approx(1.5)
+    assert d["value"] == pytest.approx(2 * 64 * 3 / 4.5e-3)
+
+
+def test_gpus_flag_must_match_the_launcher():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                        "--dry-run", "--steps", "3", "--warmup", "3"], env=env,
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode != 0 and "disagrees with WORLD_SIZE" in r.stderr

@@ -309,13 +309,27 @@ def test_rejects_bad_arguments(moe):
 # ------------------------------------------------------------------ full-size layers
 
 
-def _sample_tokens(T, idx, n_random=24, seed=0):
+def _sample_tokens(T, idx, n_random=24, seed=0, tile_rows=128):
+    """Tokens to check element by element on a multi-GB layer: for every expert hit, the
+    tokens of its first and last row (rows are in ascending token order within a group);
+    in the hottest group, the tokens on both sides of every tile_rows boundary (the
+    tokens-on-M tile height; the CTA pairs' 256-row tiles fall on every other one); the
+    first and last 6 tokens; 24 random ones."""
     rng = np.random.default_rng(seed)
-    hot = int(np.bincount(idx.reshape(-1)).argmax())
-    hot_tok = np.nonzero((idx == hot).any(1))[0]
-    pick = set(range(min(T, 6))) | set(range(max(0, T - 6), T))
+    K = idx.shape[1]
+    flat = idx.reshape(-1)
+    tok = np.repeat(np.arange(T), K)
+    order = np.argsort(flat, kind="stable")
+    se, st = flat[order], tok[order]
+    starts = np.r_[0, np.nonzero(np.diff(se))[0] + 1]
+    ends = np.r_[starts[1:], len(se)] - 1
+    pick = set(st[starts].tolist()) | set(st[ends].tolist())
+    hot = int(np.bincount(flat).argmax())
+    hot_rows = st[se == hot]
+    for b in range(tile_rows, len(hot_rows), tile_rows):
+        pick |= {int(hot_rows[b - 1]), int(hot_rows[b])}
+    pick |= set(range(min(T, 6))) | set(range(max(0, T - 6), T))
     pick |= set(rng.choice(T, size=min(T, n_random), replace=False).tolist())
-    pick |= set(hot_tok[:4].tolist()) | set(hot_tok[-4:].tolist())
     return np.array(sorted(pick), dtype=np.int64)
 
 
@@ -330,7 +344,13 @@ def test_full_size_layer(moe, oracle_mod, name):
     toks = _sample_tokens(cfg.T, gi)
     rep = check_layer(oracle_mod, inp, y, gi, _np(w), tokens=toks)
     np.testing.assert_array_equal(_np(counts), np.bincount(gi.reshape(-1), minlength=cfg.E))
-    print(name, rep, "U =", int((_np(counts) > 0).sum()))
+    hit = np.unique(gi)
+    covered = np.unique(gi[toks])
+    # every expert hit has at least its first and last row checked element by element
+    assert np.array_equal(covered, hit)
+    print(f"{name}: {len(toks)} tokens checked, {len(hit)} groups, bound used "
+          f"{rep['bound_used']:.3f}, near ties {rep['near_tie']}, differing sets "
+          f"{rep['differing']}, max|dy| {rep['y_err']:.3e} ({rep['y_rel']:.2e} x RMS)")
 
 
 # ------------------------------------------------------------------ router variants, residual

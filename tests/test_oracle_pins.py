@@ -355,11 +355,22 @@ def test_granularity_invariant(oracle_mod):
 
 
 def test_shared_expert_flops_formula(oracle_mod):
-    """Section 4: F = 2 m N_s + 2 sum t_e N_e -- the shared term scales with all m tokens."""
+    """Section 4: F = 2 m N_s + 2 sum t_e N_e.  Pinned through expert_flops (itself pinned
+    to the printed 3.22 GFLOPs): a shared expert is one more group that receives all m
+    tokens, and -- an expert's FLOPs being linear in its width -- a shared expert of width
+    2f is two such groups of width f.  Counts come from the oracle's permutation of a real
+    routing; without a shared expert the layer is its routed experts alone."""
     acc = oracle_mod.accounting
-    counts = [3, 0, 5, 8]
-    F = acc.layer_flops(counts, m=8, d=64, f=32, f_s=16)
-    assert F == 2 * 8 * 3 * 64 * 16 + 2 * 16 * 3 * 64 * 32
+    m, E, K, d, f = 24, 16, 4, 64, 32
+    counts = oracle_mod.permute(random_routing(m, E, K, seed=5).numpy(), E)["counts"]
+    routed = [int(c) for c in counts]
+    assert acc.layer_flops(routed, m=m, d=d, f=f, f_s=0) == acc.expert_flops(routed, d, f)
+    assert acc.layer_flops(routed, m=m, d=d, f=f, f_s=f) == acc.expert_flops(routed + [m], d, f)
+    assert acc.layer_flops(routed, m=m, d=d, f=f, f_s=2 * f) == \
+        acc.expert_flops(routed + [m, m], d, f)
+    # the shared term grows with every token, the routed one with the routed rows only
+    assert acc.layer_flops(routed, m=2 * m, d=d, f=f, f_s=f) - \
+        acc.layer_flops(routed, m=m, d=d, f=f, f_s=f) == acc.expert_flops([m], d, f)
 
 
 # ---------------------------------------------------------------- expert capacity

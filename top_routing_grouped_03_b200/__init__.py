@@ -91,6 +91,8 @@ def lib() -> ctypes.CDLL:
         L.moe_route_noalloc.restype = I
         L.moe_launch_count.argtypes = []
         L.moe_launch_count.restype = ctypes.c_ulonglong
+        L.moe_set_grid_wait_budget_ns.argtypes = [ctypes.c_ulonglong]
+        L.moe_set_grid_wait_budget_ns.restype = ctypes.c_ulonglong
         _lib = L
     return _lib
 
@@ -242,6 +244,12 @@ def combine(T, D, K, out=None, out_acc=None, y_sorted=None, slot_to_row=None, to
 def launch_count() -> int:
     """Kernels launched by the library in this process so far."""
     return int(lib().moe_launch_count())
+
+
+def set_grid_wait_budget_ns(ns: int) -> int:
+    """Bound of the layer's grid-wide wait for later calls (moe_set_grid_wait_budget_ns);
+    returns the previous bound."""
+    return int(lib().moe_set_grid_wait_budget_ns(int(ns)))
 
 
 def event_array(events):

@@ -64,6 +64,9 @@ cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
 // Host-side count of kernel launches issued by the library (read by moe_launch_count).
 void count_launches(unsigned n);
 
+// Bound, in nanoseconds, of the layer's grid-wide wait (moe_set_grid_wait_budget_ns).
+unsigned long long grid_wait_budget_ns();
+
 // ---------------------------------------------------------------- kernel launchers
 // (defined in the .cu files, called by the C entry points in moe_api.cu)
 
@@ -145,6 +148,7 @@ struct GroupedGemmLaunch {
     int final_rows;
     unsigned* done;
     const bf16* final_residual;  // [final_rows, D] added in the conversion, or NULL
+    unsigned long long barrier_budget_ns;  // bound of that grid-wide wait per CTA
     // gate_up with gather_tok: room for the rows in expert order [rows, D]; when given, the
     // CTA-pair kernel may be used (rows gathered by a copy kernel first)
     bf16* gather_buf;

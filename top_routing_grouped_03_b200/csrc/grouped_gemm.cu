@@ -90,6 +90,7 @@ struct Params {
     int final_rows;             //   bf16 here once every CTA of the grid has added its tiles
     unsigned* done;             //   (grid barrier counter, zero at launch)
     const bf16* final_residual; //   + this bf16 [final_rows, out_cols] when not NULL
+    unsigned long long barrier_budget_ns;  // how long a CTA waits at that grid barrier
     // weights-on-M kernel, y_out only: the K steps are cut into ksplit equal slices, one
     // tile per slice, and slice s writes its partial sums to y_out + s * split_stride
     int ksplit;
@@ -134,7 +135,8 @@ __device__ __noinline__ void finalize_output(const Params& p) {
         int ok = 1;
         const uint64_t t0 = global_timer_ns();
         while (ld_acquire_gpu(p.done) < gridDim.x) {
-            if (global_timer_ns() - t0 > kWaitBudgetNs) {
+            // (a budget of 0 gives up at the first look that finds the grid incomplete)
+            if (global_timer_ns() - t0 >= p.barrier_budget_ns) {
                 set_status(p.status, MOE_ERR_TIMEOUT);
                 ok = 0;
                 break;
@@ -1185,6 +1187,7 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
     p.final_rows = a.final_rows;
     p.done = a.done;
     p.final_residual = a.final_residual;
+    p.barrier_budget_ns = a.barrier_budget_ns;
     p.ksplit = kind == Kind::kSwap && a.ksplit > 1 ? a.ksplit : 1;
     p.zero_acc = a.gate_up ? a.zero_acc : nullptr;
     p.zero_n4 = a.zero_floats / 4;

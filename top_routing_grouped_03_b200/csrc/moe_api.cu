@@ -13,6 +13,10 @@ namespace moe {
 std::atomic<unsigned long long> g_launches{0};
 void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
+constexpr unsigned long long kDefaultGridWaitNs = 2000000000ull;  // 2 s
+std::atomic<unsigned long long> g_grid_wait_ns{kDefaultGridWaitNs};
+unsigned long long grid_wait_budget_ns() { return g_grid_wait_ns.load(std::memory_order_relaxed); }
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -118,6 +122,10 @@ const char* moe_status_string(int status) {
 int moe_version(void) { return 100; }
 
 unsigned long long moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+unsigned long long moe_set_grid_wait_budget_ns(unsigned long long ns) {
+    return g_grid_wait_ns.exchange(ns, std::memory_order_relaxed);
+}
 
 size_t moe_workspace_size(int T, int D, int E, int K, int f, int f_s) {
     if (check_shape(T, D, E, K, f, f_s) != MOE_OK) return 0;
@@ -412,6 +420,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
         dn.final_rows = T;
         dn.done = done;
         dn.final_residual = residual;
+        dn.barrier_budget_ns = grid_wait_budget_ns();
     }
     if (!mark(MOE_EV_DOWN) || launch_grouped_gemm(dn, sms, s, true) != cudaSuccess)
         return MOE_ERR_CUDA;
@@ -442,6 +451,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
             sd.final_rows = T;
             sd.done = done;
             sd.final_residual = residual;
+            sd.barrier_budget_ns = grid_wait_budget_ns();
         }
         if (launch_grouped_gemm(sd, sms, s, true) != cudaSuccess) return MOE_ERR_CUDA;
     }
