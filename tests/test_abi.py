@@ -156,3 +156,37 @@ def test_expert_capacity_matches_oracle(lib, oracle_mod):
     assert moe.expert_capacity(64, 8, 256, 0.0) == -1
     assert moe.expert_capacity(64, 8, 256, -1.0) == -1
     assert moe.expert_capacity(64, 8, 0, 1.25) == -1
+
+
+def _plan(L, T, D, E, K, f, f_s=0, flags=0):
+    A = 0x10000
+    p = moe.LayerParams()
+    p.x, p.w_router, p.w_gate_up, p.w_down = A, A, A, A
+    if f_s:
+        p.w_shared_gate, p.w_shared_gate_up, p.w_shared_down = A, A, A
+    p.T, p.D, p.E, p.K, p.f, p.f_s, p.flags = T, D, E, K, f, f_s, flags
+    mask, n = ctypes.c_uint(0), ctypes.c_int(0)
+    assert L.moe_layer_plan(ctypes.byref(p), ctypes.byref(mask), ctypes.byref(n)) == MOE_OK
+    steps = {name for i, name in enumerate(moe.STEP_EVENT_NAMES) if mask.value >> i & 1}
+    return steps, n.value
+
+
+def test_layer_plan_names_the_launched_steps(lib):
+    """moe_layer_plan (host only): which steps launch kernels and how many, per regime."""
+    # decode: the permutation runs in the router's last CTA
+    assert _plan(lib, 64, 2048, 256, 8, 512) == ({"router", "gate_up", "down"}, 3)
+    # fixed-order combine: one more kernel
+    assert _plan(lib, 64, 2048, 256, 8, 512, flags=1) == (
+        {"router", "gate_up", "down", "combine"}, 4)
+    # fine-grained + shared: tensor-core router (logits GEMM + selection), chunked
+    # permutation (histograms + scatter), the shared expert inside the routed launches
+    assert _plan(lib, 4096, 4096, 512, 10, 1024, 1024) == (
+        {"router", "permute", "gate_up", "down"}, 6)
+    # a shared expert of another width keeps its two launches
+    assert _plan(lib, 4096, 4096, 512, 10, 1024, 512) == (
+        {"router", "permute", "gate_up", "down", "shared"}, 8)
+    # prefill: CTA pairs, whose gate_up first copies the token rows into expert order
+    assert _plan(lib, 8192, 4096, 128, 8, 1536) == ({"router", "permute", "gate_up", "down"}, 7)
+    # E > 256 with few tokens: the permutation is a launch of its own
+    assert _plan(lib, 70, 256, 512, 16, 128) == ({"router", "permute", "gate_up", "down"}, 4)
+    assert _plan(lib, 0, 256, 16, 4, 128) == (set(), 0)

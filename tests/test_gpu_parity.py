@@ -54,6 +54,13 @@ SMALL_LAYERS = {
     # at most 16 tokens: weights-on-M grouped GEMMs, routed and shared
     "few_tokens_shared": LayerConfig("few_tokens_shared", T=12, D=256, E=32, K=4, f=256,
                                      f_s=128, seed=9),
+    # shared expert as wide as the routed ones: it runs as an extra, interleaved group of
+    # the routed launches (routed groups of a few to ~50 rows; then many small groups with
+    # the tensor-core router and several shared row blocks)
+    "shared_fused": LayerConfig("shared_fused", T=100, D=256, E=16, K=4, f=256, f_s=256,
+                                seed=16),
+    "shared_fused_tc": LayerConfig("shared_fused_tc", T=520, D=512, E=128, K=8, f=256,
+                                   f_s=256, seed=18),
     # T >= 256 and E % 128 == 0: router logits on the tensor cores, shared gate in the
     # selection kernel
     "tc_router_shared": LayerConfig("tc_router_shared", T=300, D=384, E=128, K=6, f=128,
@@ -245,7 +252,7 @@ def test_layer_matches_oracle(moe, oracle_mod, name):
 
 
 @pytest.mark.parametrize("name", ["tiny", "decode", "shared_small", "ragged_T", "deep_gate_up",
-                                  "deep_down", "deep_shared"])
+                                  "deep_down", "deep_shared", "shared_fused"])
 def test_layer_deterministic_mode(moe, oracle_mod, name):
     inp = make_inputs(SMALL_LAYERS[name]).to("cuda")
     layer, y1, idx, w, _ = _run_layer(moe, inp, deterministic=True)
@@ -411,7 +418,7 @@ def test_route_sigmoid_worked_example(moe):
 
 @pytest.mark.parametrize("det", [False, True])
 @pytest.mark.parametrize("vi", [0, 2, 4])
-@pytest.mark.parametrize("name", ["tiny", "tc_router_shared"])
+@pytest.mark.parametrize("name", ["tiny", "tc_router_shared", "shared_fused"])
 def test_layer_variants_with_residual(moe, oracle_mod, name, vi, det):
     cfg = SMALL_LAYERS[name]
     inp = make_inputs(cfg).to("cuda")

@@ -91,6 +91,8 @@ def lib() -> ctypes.CDLL:
         L.moe_route_noalloc.restype = I
         L.moe_launch_count.argtypes = []
         L.moe_launch_count.restype = ctypes.c_ulonglong
+        L.moe_layer_plan.argtypes = [ctypes.POINTER(LayerParams), P, P]
+        L.moe_layer_plan.restype = I
         L.moe_set_grid_wait_budget_ns.argtypes = [ctypes.c_ulonglong]
         L.moe_set_grid_wait_budget_ns.restype = ctypes.c_ulonglong
         _lib = L
@@ -338,6 +340,18 @@ class MoELayer:
                                      _stream(stream))
         _check(rc, "moe_layer_forward")
         return out
+
+    def plan(self, T: int):
+        """(steps that launch kernels, kernels per call) for T tokens, from moe_layer_plan:
+        the step names of STEP_EVENT_NAMES whose interval holds work of their own."""
+        x = torch.empty((0, self.D), dtype=BF16, device=self.w_router.device)
+        prm = self.params(x)
+        prm.T = T
+        mask, n = ctypes.c_uint(0), ctypes.c_int(0)
+        _check(lib().moe_layer_plan(ctypes.byref(prm), ctypes.byref(mask), ctypes.byref(n)),
+               "moe_layer_plan")
+        steps = [name for i, name in enumerate(STEP_EVENT_NAMES) if mask.value >> i & 1]
+        return steps, n.value
 
     def forward_host(self, x_host, y_host, x_dev, y_dev, stream=None):
         """End to end from host memory: copy x (pinned host) in, run the layer, copy y

@@ -70,6 +70,25 @@ unsigned long long grid_wait_budget_ns();
 // ---------------------------------------------------------------- kernel launchers
 // (defined in the .cu files, called by the C entry points in moe_api.cu)
 
+struct PermuteLaunch {
+    const int32_t* topk_idx;
+    const float* topk_w;
+    const int32_t* counts;   // [E] from the router, or NULL: counted here from topk_idx
+    int32_t* counts_out;     // where the counts (given or derived) are copied, or NULL
+    int T, E, K;
+    int32_t* offsets;
+    int32_t* sorted_token;
+    float* sorted_w;
+    int32_t* slot_to_row;
+    int32_t* dense_offsets;  // optional [2] = {0, T} for a dense (shared) expert group
+    int* status;
+    int32_t* hist;           // [permute_chunks(T*K) * E] scratch, or NULL (one CTA)
+    long long capacity;      // >= 0: each expert keeps its first `capacity` entries; < 0: all
+};
+// chunks the permutation cuts T*K entries into (1 at decode sizes, at most 256)
+int permute_chunks(long long entries);
+cudaError_t launch_permute(const PermuteLaunch& a, cudaStream_t s, bool pdl = false);
+
 struct RouterLaunch {
     const bf16* x;
     const bf16* w_router;
@@ -92,7 +111,14 @@ struct RouterLaunch {
     const float* select_bias; // [E] added to the scores for the selection only, or NULL
     int bf16_weights;         // round the renormalised weights to bf16
     int logit_planes;         // tensor-core path: partial-sum planes of [T, E] in logits
+    // CUDA-core router only: the last CTA to finish its selection also runs the
+    // permutation `perm` (one chunk: T*K <= 4096 entries, E <= 256; perm.counts = counts),
+    // taking the ticket counters[ceil(T/8)]
+    int fuse_perm;
+    PermuteLaunch perm;
 };
+// the router kernel can run the permutation of this many (token, slot) entries, E experts
+bool router_can_fuse_permute(int T, int E, int K);
 cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bool pdl = false);
 
 // Router for many tokens: the logits x W_r^T [T, E] (fp32) on the tensor cores through the
@@ -104,24 +130,7 @@ bool router_uses_tensor_cores(int T, int E);
 int router_tc_max_planes(int T);
 cudaError_t launch_router_tc(const RouterLaunch& a, int num_sms, cudaStream_t s, bool pdl = false);
 
-struct PermuteLaunch {
-    const int32_t* topk_idx;
-    const float* topk_w;
-    const int32_t* counts;   // [E] from the router, or NULL: counted here from topk_idx
-    int32_t* counts_out;     // with counts NULL: where the counts are written, or NULL
-    int T, E, K;
-    int32_t* offsets;
-    int32_t* sorted_token;
-    float* sorted_w;
-    int32_t* slot_to_row;
-    int32_t* dense_offsets;  // optional [2] = {0, T} for a dense (shared) expert group
-    int* status;
-    int32_t* hist;           // [permute_chunks(T*K) * E] scratch, or NULL (one CTA)
-    long long capacity;      // >= 0: each expert keeps its first `capacity` entries; < 0: all
-};
-// chunks the permutation cuts T*K entries into (1 at decode sizes, at most 256)
-int permute_chunks(long long entries);
-cudaError_t launch_permute(const PermuteLaunch& a, cudaStream_t s, bool pdl = false);
+
 
 
 struct GroupedGemmLaunch {
@@ -159,7 +168,21 @@ struct GroupedGemmLaunch {
     // kernel, before the down projection adds into it; NULL: nothing to clear
     float* zero_acc;
     long long zero_floats;
+    // one extra dense group after the E routed ones (the shared expert), run inside the same
+    // launch with its tiles interleaved: weights xg_w ([2f, D] gate_up or [D, f] down, the
+    // routed experts' f), rows [offsets[E], offsets[E] + xg_rows) of the sorted problem,
+    // row r being token r - offsets[E]; down scales row r by xg_weight[token].  `rows`
+    // then counts these rows too.  Only the one-CTA tokens-on-M kernel takes it
+    // (grouped_gemm_takes_extra_group); NULL: none
+    const void* xg_w;
+    int xg_rows;
+    const float* xg_weight;
 };
+// true when launch_grouped_gemm would run `a` on the one-CTA tokens-on-M kernel (the one
+// that can carry an extra dense group)
+bool grouped_gemm_takes_extra_group(const GroupedGemmLaunch& a, int num_sms);
+// kernels launch_grouped_gemm launches for `a` (0 when it has nothing to do)
+int grouped_gemm_launches(const GroupedGemmLaunch& a, int num_sms);
 cudaError_t launch_gather_rows(const bf16* x, const int32_t* tok, int rows, int D, bf16* out,
                                int num_sms, cudaStream_t s, bool pdl);
 cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s,

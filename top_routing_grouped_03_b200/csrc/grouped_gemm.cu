@@ -99,6 +99,15 @@ struct Params {
     // accumulator) before their first tile -- they would otherwise wait for it idle
     float* zero_acc;
     long long zero_n4;
+    // one-CTA tokens-on-M kernel: choose the tile width on the device (else 256 rows)
+    int tm_adaptive;
+    // one-CTA tokens-on-M kernel: group G-1 is an extra dense group (the shared expert):
+    // its xg_rows rows follow the routed ones, [offsets[G-1], offsets[G-1] + xg_rows), row
+    // r is token r - offsets[G-1], its weights come from the second weight map, and (down)
+    // row r is scaled by xg_weight[token]; its tiles are interleaved with the routed ones
+    int xg;
+    int xg_rows;
+    const float* xg_weight;
 };
 
 // Epilogue threads of every CTA clear their grid-strided share of p.zero_acc.
@@ -244,14 +253,15 @@ struct RowGather {
     uint32_t src_off[kChunks];  // element offset of the chunk's row in x (< 2^31)
     uint32_t valid;
 
+    // id_base >= 0: row r is token r - id_base (a dense group), tok is not read
     __device__ __forceinline__ void plan(const int32_t* tok, int row0, int row_end, int row_len,
-                                         int lane) {
+                                         int lane, int id_base = -1) {
         valid = 0;
 #pragma unroll
         for (int u = 0; u < kChunks; ++u) {
             const int row = row0 + (lane >> 3) + 4 * u;
             const bool ok = row < row_end;
-            const int t = ok ? __ldg(tok + row) : 0;
+            const int t = ok ? (id_base >= 0 ? row - id_base : __ldg(tok + row)) : 0;
             src_off[u] = static_cast<uint32_t>(t) * row_len + (lane & 7) * 8;
             valid |= (ok ? 1u : 0u) << u;
         }
@@ -503,16 +513,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
 }
 
 // ---------------------------------------------------------------- tokens-on-M variant
-// For groups with many rows: the MMA's M side holds 128 token rows and its N side 256
-// weight rows (gate_up: the gate and up rows of the same 128 features; down: 256 output
-// features), one tcgen05.mma of 128 x 256 x 16 per 16 of K.  Per tile: 128 rows x 128 h
-// features (gate_up) or 128 rows x 256 output features (down).  Each epilogue thread owns
-// one row, so h is written with 16-byte stores and the down epilogue reduces 16-byte
-// vectors (red.global.add.v4.f32) into the token's output row.
+// For groups with more than a handful of rows: the MMA's M side holds 128 token rows and
+// its N side wn weight rows (gate_up: the gate and up rows of the same wn/2 features;
+// down: wn output features), one tcgen05.mma of 128 x wn x 16 per 16 of K.  Each
+// epilogue thread owns one row, so h is written with 16-byte stores and the down epilogue
+// reduces 16-byte vectors (red.global.add.v4.f32) into the token's output row.
+// The one-CTA kernel picks wn in {256, 128, 64} on the device, per launch, from the
+// groups' row counts: a few experts with many rows (concentrated routing) would otherwise
+// leave most SMs idle, each busy SM streaming its weight tiles alone; narrower tiles
+// spread the same weight bytes over more of the grid (and, being smaller, let more
+// pipeline stages fit in shared memory).  The CTA-pair kernel always uses wn = 256.
 constexpr int kTmRows = 128;  // token rows per tile (MMA M)
-// auto orientation: weights on M only while no group can exceed this many rows
-constexpr int kSwapMaxRows = 16;
-constexpr int kTmN = 256;     // weight rows per tile (MMA N)
+constexpr int kTmN = 256;     // widest weight tile (MMA N)
+constexpr int kWBox = 32;     // weight rows per TMA box of the one-CTA kernel
 // 2 warps (producer, MMA) + 8 epilogue warps: two warps per tensor-memory lane quarter,
 // each draining half of the accumulator's columns
 constexpr int kTmThreads = 64 + 256;
@@ -525,49 +538,107 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                  : "memory");
 }
 
-// Epilogue of one tokens-on-M tile for one epilogue warp: `half` selects the columns this
-// warp drains (gate_up: features [64 half, 64 half + 64) of the tile's 128; down: output
-// columns [128 half, 128 half + 128) of its 256).  The warp's 32 lanes are 32 rows.
+// 16 SwiGLU values of one row (gate and up accumulators, fp32 bits) -> 16 bf16 in h.
+__device__ __forceinline__ void swiglu_store16(const uint32_t* gv, const uint32_t* uv, bf16* dst) {
+    uint32_t pk[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float g0 = __uint_as_float(gv[2 * j]);
+        const float g1 = __uint_as_float(gv[2 * j + 1]);
+        const float h0 = __fdividef(g0, 1.f + __expf(-g0)) * __uint_as_float(uv[2 * j]);
+        const float h1 = __fdividef(g1, 1.f + __expf(-g1)) * __uint_as_float(uv[2 * j + 1]);
+        pk[j] = pack_bf16x2(h0, h1);
+    }
+    uint4* d = reinterpret_cast<uint4*>(dst);
+    d[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    d[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+}
+
+// The warp's 32 rows x 16 columns of w * v (v: fp32 bits, this lane's row) reduced into the
+// token rows through shared memory: a thread holds one row, and a 4-wide reduction per
+// thread and row would touch 32 rows' lines with 16 bytes each; transposed through
+// `stage` (2 KB, 16-byte chunks XOR-swizzled so that both the row-wise writes and the
+// transposed reads are free of bank conflicts) each reduction instruction covers 8 rows x
+// 64 contiguous bytes: whole 32-byte sectors.
+__device__ __forceinline__ void reduce16_transposed(const Params& p, const uint32_t* v, float w,
+                                                    int tok, bool valid, int col, float* stage,
+                                                    int lane) {
+    const int rr0 = lane >> 2, kq = lane & 3;  // read side: row (of 8), chunk
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        *reinterpret_cast<float4*>(stage + lane * 16 + ((k ^ ((lane >> 1) & 3)) << 2)) =
+            make_float4(w * __uint_as_float(v[4 * k]), w * __uint_as_float(v[4 * k + 1]),
+                        w * __uint_as_float(v[4 * k + 2]), w * __uint_as_float(v[4 * k + 3]));
+    __syncwarp();
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+        const int rr = it * 8 + rr0;
+        const float4 val =
+            *reinterpret_cast<const float4*>(stage + rr * 16 + ((kq ^ ((rr >> 1) & 3)) << 2));
+        const int tok_r = __shfl_sync(0xffffffffu, tok, rr);
+        const bool valid_r = __shfl_sync(0xffffffffu, valid ? 1 : 0, rr) != 0;
+        if (valid_r)
+            red_add_v4(p.acc_out + static_cast<size_t>(tok_r) * p.out_cols + col + 4 * kq, val.x,
+                       val.y, val.z, val.w);
+    }
+    __syncwarp();
+}
+
+// Epilogue of one tokens-on-M tile (wn weight rows) for one epilogue warp: `half` selects
+// the columns this warp drains (gate_up: features [wn/4 half, wn/4 (half + 1)) of the
+// tile's wn/2; down: output columns [wn/2 half, wn/2 (half + 1)) of its wn).  The warp's
+// 32 lanes are 32 rows.
 template <bool GATE_UP>
 __device__ __forceinline__ void tm_epilogue(const Params& p, uint32_t tbase, int row, bool valid,
-                                            int tile_i, int half, float* stage) {
+                                            int tile_i, int half, float* stage, int wn,
+                                            int id_base = -1) {
+    const int lane = threadIdx.x & 31;
     if (GATE_UP) {
-        bf16* hrow = p.h_out + static_cast<size_t>(row) * p.out_cols + tile_i * kBM + half * 64;
+        const int F = wn >> 1;        // features of the tile
+        const int hc = F >> 1;        // features of this warp: 64, 32 or 16
+        bf16* hrow = p.h_out + static_cast<size_t>(row) * p.out_cols + tile_i * F + half * hc;
+        if (hc >= 32) {
 #pragma unroll 1
-        for (int c0 = 0; c0 < 64; c0 += 32) {
-            uint32_t gv[32], uv[32];
-            tmem_ld32(tbase + half * 64 + c0, gv);
-            tmem_ld32(tbase + kBM + half * 64 + c0, uv);
-            tmem_ld_wait();
-            if (valid) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float g0 = __uint_as_float(gv[2 * j]);
-                    const float g1 = __uint_as_float(gv[2 * j + 1]);
-                    const float h0 = __fdividef(g0, 1.f + __expf(-g0)) * __uint_as_float(uv[2 * j]);
-                    const float h1 = __fdividef(g1, 1.f + __expf(-g1)) * __uint_as_float(uv[2 * j + 1]);
-                    pk[j] = pack_bf16x2(h0, h1);
+            for (int c0 = 0; c0 < hc; c0 += 32) {
+                uint32_t gv[32], uv[32];
+                tmem_ld32(tbase + half * hc + c0, gv);
+                tmem_ld32(tbase + F + half * hc + c0, uv);
+                tmem_ld_wait();
+                if (valid) {
+                    swiglu_store16(gv, uv, hrow + c0);
+                    swiglu_store16(gv + 16, uv + 16, hrow + c0 + 16);
                 }
-                uint4* dst = reinterpret_cast<uint4*>(hrow + c0);
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
             }
+        } else {
+            uint32_t gv[16], uv[16];
+            tmem_ld16(tbase + half * hc, gv);
+            tmem_ld16(tbase + F + half * hc, uv);
+            tmem_ld_wait();
+            if (valid) swiglu_store16(gv, uv, hrow);
         }
     } else {
-        const float w = (valid && p.sorted_w) ? __ldg(p.sorted_w + row) : 1.f;
-        const int tok = valid ? (p.sorted_token ? __ldg(p.sorted_token + row) : row) : 0;
-        const int col0 = tile_i * kTmN + half * 128;
-        const int lane = threadIdx.x & 31;
+        const int hc = wn >> 1;  // output columns of this warp: 128, 64 or 32
+        // token and weight of this row: the extra dense group's row r is token r - id_base,
+        // scaled by xg_weight[token]
+        float w = 1.f;
+        int tok = 0;
+        if (valid && id_base >= 0) {
+            tok = row - id_base;
+            w = __ldg(p.xg_weight + tok);
+        } else if (valid) {
+            tok = p.sorted_token ? __ldg(p.sorted_token + row) : row;
+            w = p.sorted_w ? __ldg(p.sorted_w + row) : 1.f;
+        }
+        const int col0 = tile_i * wn + half * hc;
+        const uint32_t tcol = tbase + half * hc;
         // a warp with a handful of rows (a few tokens per expert) reduces row by row: the
-        // transpose below would move 32 rows through shared memory for 2 or 3 of them
+        // transpose would move 32 rows through shared memory for 2 or 3 of them
         const bool sparse = __popc(__ballot_sync(0xffffffffu, valid)) <= 4;
         if (p.acc_out && sparse) {
 #pragma unroll 1
-            for (int c0 = 0; c0 < 128; c0 += 32) {
+            for (int c0 = 0; c0 < hc; c0 += 32) {
                 uint32_t v[32];
-                tmem_ld32(tbase + half * 128 + c0, v);
+                tmem_ld32(tcol + c0, v);
                 tmem_ld_wait();
                 if (valid) {
                     float* dst = p.acc_out + static_cast<size_t>(tok) * p.out_cols + col0 + c0;
@@ -578,43 +649,25 @@ __device__ __forceinline__ void tm_epilogue(const Params& p, uint32_t tbase, int
                 }
             }
         } else if (p.acc_out) {
-            // Reductions into the token rows, 16 columns at a time.  A thread holds one
-            // row; a 4-wide reduction per thread and row would touch 32 rows' lines with 16
-            // bytes each.  So the warp's 32 rows x 16 columns go through shared memory
-            // (`stage`, 2 KB, 16-byte chunks XOR-swizzled so that both the row-wise writes
-            // and the transposed reads are free of bank conflicts) and each reduction
-            // instruction then covers 8 rows x 64 contiguous bytes: whole 32-byte sectors.
-            const int rr0 = lane >> 2, kq = lane & 3;  // read side: row (of 8), chunk
+            // 16 columns at a time, the next 16 loaded from tensor memory while these are
+            // reduced (tcgen05.wait::ld only after the shared-memory transpose)
+            uint32_t va[16], vb[16];
+            tmem_ld16(tcol, va);
+            tmem_ld_wait_dep(va);
 #pragma unroll 1
-            for (int c0 = 0; c0 < 128; c0 += 16) {
-                uint32_t v[16];
-                tmem_ld16(tbase + half * 128 + c0, v);
-                tmem_ld_wait();
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    *reinterpret_cast<float4*>(stage + lane * 16 + ((k ^ ((lane >> 1) & 3)) << 2)) =
-                        make_float4(w * __uint_as_float(v[4 * k]), w * __uint_as_float(v[4 * k + 1]),
-                                    w * __uint_as_float(v[4 * k + 2]), w * __uint_as_float(v[4 * k + 3]));
-                __syncwarp();
-#pragma unroll
-                for (int it = 0; it < 4; ++it) {
-                    const int rr = it * 8 + rr0;
-                    const float4 val = *reinterpret_cast<const float4*>(
-                        stage + rr * 16 + ((kq ^ ((rr >> 1) & 3)) << 2));
-                    const int tok_r = __shfl_sync(0xffffffffu, tok, rr);
-                    const bool valid_r = __shfl_sync(0xffffffffu, valid ? 1 : 0, rr) != 0;
-                    if (valid_r)
-                        red_add_v4(p.acc_out + static_cast<size_t>(tok_r) * p.out_cols + col0 + c0 +
-                                       4 * kq,
-                                   val.x, val.y, val.z, val.w);
-                }
-                __syncwarp();
+            for (int c0 = 0; c0 < hc; c0 += 32) {
+                tmem_ld16(tcol + c0 + 16, vb);
+                reduce16_transposed(p, va, w, tok, valid, col0 + c0, stage, lane);
+                tmem_ld_wait_dep(vb);
+                if (c0 + 32 < hc) tmem_ld16(tcol + c0 + 32, va);
+                reduce16_transposed(p, vb, w, tok, valid, col0 + c0 + 16, stage, lane);
+                tmem_ld_wait_dep(va);
             }
         }
 #pragma unroll 1
-        for (int c0 = 0; c0 < 128 && p.y_out; c0 += 32) {
+        for (int c0 = 0; c0 < hc && p.y_out; c0 += 32) {
             uint32_t v[32];
-            tmem_ld32(tbase + half * 128 + c0, v);
+            tmem_ld32(tcol + c0, v);
             tmem_ld_wait();
             if (valid) {
                 float4* dst = reinterpret_cast<float4*>(
@@ -638,34 +691,102 @@ __device__ __forceinline__ float* epi_stage(int* table_end, int warp) {
     return reinterpret_cast<float*>(a) + (warp - 2) * kStageFloatsPerWarp;
 }
 
-template <bool GATE_UP>
+// Shared-memory ring of the one-CTA kernel: 192 KB cut into stages of 128 token rows
+// (16 KB) + wn weight rows: 4 stages at wn = 256, 6 at 128, 8 at 64.
 struct CfgTm {
-    static constexpr int kABytes = kTmRows * kBK * 2;  // 16 KB of token rows
-    static constexpr int kBBytes = kTmN * kBK * 2;     // 32 KB of weight rows
-    static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kStages = 4;
-    static constexpr int kAccCols = kTmN;
-    static constexpr int kTmemCols = 2 * kAccCols;
-    static_assert(kTmemCols <= 512, "accumulators exceed tensor memory");
+    static constexpr int kABytes = kTmRows * kBK * 2;
+    static constexpr int kRingBytes = 192 * 1024;
+    static constexpr int kMaxStages = 8;
+    static constexpr int kTmemCols = 2 * kTmN;  // two accumulators of up to 256 columns
 };
+__device__ __forceinline__ int tm_stage_bytes(int wn) { return CfgTm::kABytes + wn * kBK * 2; }
+__device__ __forceinline__ int tm_num_stages(int wn) {
+    return min(CfgTm::kMaxStages, CfgTm::kRingBytes / tm_stage_bytes(wn));
+}
 
+// Processing order of the one-CTA kernel's tiles when an extra dense group is present:
+// its n_x tiles (table indices n_r .. n_r + n_x - 1, after the routed groups' n_r) take
+// every s-th slot, s = floor((n_r + n_x) / n_x), so that its compute-bound tiles run
+// alongside the weight-streaming routed tiles instead of all at the end.  Returns the
+// table index of slot t.
+__device__ __forceinline__ int tile_of_slot(int t, int n_r, int n_x) {
+    if (n_x <= 0) return t;
+    const int s = (n_r + n_x) / n_x;
+    const int q = t / s;
+    if (t - q * s == s - 1 && q < n_x) return n_r + q;
+    return t - min(n_x, q);
+}
+
+// Per-tile fixed cost, in weight rows, of the width choice below (a tile's share of the
+// pipeline hand-offs and of the epilogue's fixed steps).
+constexpr int kTileCostRows = 16;
+
+// The group table of the one-CTA tokens-on-M kernel, and its tile width.  Warp 2 counts
+// the 128-row blocks of every group (row_blocks), picks the weight rows per tile
+//   wn = argmin over {256, 128, 64} of ceil(row_blocks * nf(wn) / gridDim.x) * (wn + c)
+// (nf(wn) = nf256 * 256 / wn feature blocks per row block; ties to the wider tile) --
+// the most weight rows any CTA streams, plus a per-tile cost -- and writes
+// g_tile[g] = (row blocks of the groups before g) * nf(wn).
+__device__ __forceinline__ void build_tile_table_tm(const Params& p, int* g_off, int* g_tile,
+                                                    int* total_slot, int* wn_slot, int warp,
+                                                    int lane) {
+    for (int i = threadIdx.x; i <= p.G; i += blockDim.x)
+        g_off[i] = p.offsets ? (p.xg && i == p.G ? p.offsets[i - 1] + p.xg_rows : p.offsets[i])
+                             : (i == 0 ? 0 : p.rows_total);
+    __syncthreads();
+    if (warp == 2) {
+        const int per = (p.G + 31) / 32;
+        const int gb = min(lane * per, p.G), ge = min(gb + per, p.G);
+        int local = 0;
+        for (int g = gb; g < ge; ++g) local += (g_off[g + 1] - g_off[g] + kTmRows - 1) / kTmRows;
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const long long rb = __shfl_sync(0xffffffffu, incl, 31);
+        int wn = kTmN;
+        if (p.tm_adaptive) {
+            long long best = -1;
+            for (int c = kTmN; c >= 64; c >>= 1) {
+                const long long tiles = rb * p.nf * (kTmN / c);
+                const long long cost = (tiles + gridDim.x - 1) / gridDim.x * (c + kTileCostRows);
+                if (best < 0 || cost < best) { best = cost; wn = c; }
+            }
+        }
+        const int nf = p.nf * (kTmN / wn);
+        int run = incl - local;
+        for (int g = gb; g < ge; ++g) {
+            g_tile[g] = run * nf;
+            run += (g_off[g + 1] - g_off[g] + kTmRows - 1) / kTmRows;
+        }
+        if (lane == 31) {
+            g_tile[p.G] = incl * nf;
+            *total_slot = incl * nf;
+            *wn_slot = wn;
+        }
+    }
+}
 
 template <bool GATE_UP>
 __global__ void __launch_bounds__(kTmThreads, 1)
 grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
-                       const __grid_constant__ CUtensorMap map_act, Params p) {
-    using C = CfgTm<GATE_UP>;
+                       const __grid_constant__ CUtensorMap map_act,
+                       const __grid_constant__ CUtensorMap map_w2, Params p) {
+    using C = CfgTm;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
-    uint64_t* empty = full + C::kStages;
-    uint64_t* tfull = empty + C::kStages;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kRingBytes);
+    uint64_t* empty = full + C::kMaxStages;
+    uint64_t* tfull = empty + C::kMaxStages;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* total_slot = reinterpret_cast<int*>(tmem_slot + 2);
+    int* wn_slot = reinterpret_cast<int*>(tmem_slot + 3);
     int* g_off = reinterpret_cast<int*>(tmem_slot + 4);
     int* g_tile = g_off + (p.G + 1);
 
@@ -674,7 +795,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
     const bool gather = GATE_UP && p.gather_tok != nullptr;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
+        for (int s = 0; s < C::kMaxStages; ++s) {
             mbar_init(&full[s], gather ? 1 + 32 : 1);
             mbar_init(&empty[s], 1);
         }
@@ -688,6 +809,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&map_w);
+        if (p.xg) tma_prefetch_desc(&map_w2);
         if (!gather) tma_prefetch_desc(&map_act);
     }
     if (warp == 1) {
@@ -696,31 +818,42 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
     }
     grid_dep_wait();
     grid_dep_launch();
-    build_tile_table(p, kTmRows, g_off, g_tile, total_slot, warp, lane);
+    build_tile_table_tm(p, g_off, g_tile, total_slot, wn_slot, warp, lane);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int total = *total_slot;
+    const int wn = *wn_slot;               // weight rows per tile
+    const int stage_bytes = tm_stage_bytes(wn);
+    const int nstages = tm_num_stages(wn);
+    // tiles of the routed groups, and of the extra dense group (interleaved, tile_of_slot)
+    const int n_routed = p.xg ? g_tile[p.G - 1] : total;
+    const int n_extra = total - n_routed;
+    const int x_base = p.xg ? g_off[p.G - 1] : -1;  // first row of the extra group
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
         // token rows (A): one TMA box of 128 rows when contiguous, else the lanes gather
-        // them with cp.async; weight rows (B): two TMA boxes of 128 rows.
+        // them with cp.async; weight rows (B): wn rows in boxes of 32.
         if (gather || lane == 0) {
             const uint64_t pol_w = policy_evict_first();
             const uint64_t pol_a = policy_evict_last();
+            const uint32_t w_bytes = static_cast<uint32_t>(wn) * kBK * 2;
             int stage = 0;
             uint32_t phase = 0, filled = 0, fill_phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const Tile t = decode_tile(tile, g_tile, g_off, p.G, kTmRows);
-                // gate_up: gate rows g*2f + i*128 and up rows g*2f + f + i*128;
-                // down: rows g*D + i*256 and the next 128
-                const int wr0 = t.g * p.w_group_rows + t.i * (GATE_UP ? kBM : kTmN);
-                const int wr1 = GATE_UP ? wr0 + p.up_rows : wr0 + kBM;
+            for (int slot = blockIdx.x; slot < total && ok; slot += gridDim.x) {
+                const Tile t = decode_tile(tile_of_slot(slot, n_routed, n_extra), g_tile, g_off,
+                                           p.G, kTmRows);
+                const bool ex = p.xg && t.g == p.G - 1;
+                const CUtensorMap* mw = ex ? &map_w2 : &map_w;
+                // gate_up: gate rows g*2f + i*wn/2 and up rows f further; down: g*D + i*wn
+                // (the extra group's weights are a matrix of their own: g = 0 there)
+                const int wr0 = (ex ? 0 : t.g * p.w_group_rows) + t.i * (GATE_UP ? wn / 2 : wn);
                 RowGather<kTmRows> rg;
-                if (gather) rg.plan(p.gather_tok, t.row0, t.row_end, p.nk * kBK, lane);
+                if (gather)
+                    rg.plan(p.gather_tok, t.row0, t.row_end, p.nk * kBK, lane, ex ? x_base : -1);
                 for (int kk = 0; kk < p.nk; ++kk) {
                     bool got = mbar_wait(&empty[stage], phase ^ 1u, kWaitBudgetNs, abort_flag);
                     if (gather) got = __all_sync(0xffffffffu, got);
@@ -730,14 +863,25 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
                         ok = false;
                         break;
                     }
-                    uint8_t* st = smem + stage * C::kStageBytes;
+                    uint8_t* st = smem + stage * stage_bytes;
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(&full[stage], gather ? C::kBBytes : C::kStageBytes);
+                        mbar_arrive_expect_tx(&full[stage], gather ? w_bytes : stage_bytes);
                         if (!gather)
                             tma_load_2d(st, &map_act, &full[stage], kk * kBK, t.row0, pol_a);
-                        tma_load_2d(st + C::kABytes, &map_w, &full[stage], kk * kBK, wr0, pol_w);
-                        tma_load_2d(st + C::kABytes + kBM * kBK * 2, &map_w, &full[stage],
-                                    kk * kBK, wr1, pol_w);
+                        uint8_t* bt = st + C::kABytes;
+                        if (GATE_UP) {
+                            const int F = wn / 2;
+                            for (int b = 0; b < F; b += kWBox) {
+                                tma_load_2d(bt + b * kBK * 2, mw, &full[stage], kk * kBK,
+                                            wr0 + b, pol_w);
+                                tma_load_2d(bt + (F + b) * kBK * 2, mw, &full[stage],
+                                            kk * kBK, wr0 + p.up_rows + b, pol_w);
+                            }
+                        } else {
+                            for (int b = 0; b < wn; b += kWBox)
+                                tma_load_2d(bt + b * kBK * 2, mw, &full[stage], kk * kBK,
+                                            wr0 + b, pol_w);
+                        }
                     }
                     if (gather) {
                         rg.issue(smem_u32(st), p.x, kk * kBK, lane);
@@ -745,12 +889,12 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
                     }
                     filled |= 1u << stage;
                     fill_phase = (fill_phase & ~(1u << stage)) | (phase << stage);
-                    if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+                    if (++stage == nstages) { stage = 0; phase ^= 1u; }
                 }
             }
             if (gather) cp_async_wait_all();
             if (!ok && lane == 0) {
-                for (int s = 0; s < C::kStages; ++s)
+                for (int s = 0; s < nstages; ++s)
                     if (filled & (1u << s))
                         mbar_wait(&full[s], (fill_phase >> s) & 1u, kDrainBudgetNs, nullptr);
             }
@@ -759,11 +903,11 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(kTmRows, kTmN);
+            const uint32_t idesc = idesc_bf16_f32(kTmRows, wn);
             int stage = 0;
             uint32_t phase = 0, abuf = 0, aphase = 0;
             bool ok = true, issued = false;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            for (int slot = blockIdx.x; slot < total && ok; slot += gridDim.x) {
                 if (!mbar_wait(&tempty[abuf], aphase ^ 1u, kWaitBudgetNs, abort_flag)) {
                     set_status(p.status, MOE_ERR_TIMEOUT);
                     *abort_flag = 1;
@@ -771,7 +915,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d0 = tmem_base + abuf * C::kAccCols;
+                const uint32_t d0 = tmem_base + abuf * wn;
                 for (int kk = 0; kk < p.nk; ++kk) {
                     if (!mbar_wait(&full[stage], phase, kWaitBudgetNs, abort_flag)) {
                         set_status(p.status, MOE_ERR_TIMEOUT);
@@ -781,7 +925,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
                     }
                     tc_fence_after();
                     if (gather) fence_proxy_async_smem();
-                    const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
+                    const uint32_t a0 = smem_u32(smem + stage * stage_bytes);
                     const uint32_t b0 = a0 + C::kABytes;
 #pragma unroll
                     for (int s = 0; s < kBK / 16; ++s)
@@ -789,7 +933,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
                                   (kk | s) != 0 ? 1u : 0u);
                     issued = true;
                     umma_commit(&empty[stage]);
-                    if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+                    if (++stage == nstages) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
                 umma_commit(&tfull[abuf]);
@@ -807,8 +951,10 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
         const int q = warp & 3;
         if (GATE_UP) clear_accumulator(p, threadIdx.x - 64, kTmEpiThreads);
         uint32_t abuf = 0, aphase = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const Tile t = decode_tile(tile, g_tile, g_off, p.G, kTmRows);
+        for (int slot = blockIdx.x; slot < total; slot += gridDim.x) {
+            const Tile t = decode_tile(tile_of_slot(slot, n_routed, n_extra), g_tile, g_off, p.G,
+                                       kTmRows);
+            const bool ex = p.xg && t.g == p.G - 1;
             const bool ready = mbar_wait(&tfull[abuf], aphase, kWaitBudgetNs, abort_flag);
             if (!epilogue_bar_and<kTmEpiThreads>(ready)) {
                 set_status(p.status, MOE_ERR_TIMEOUT);
@@ -816,11 +962,11 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
                 break;
             }
             tc_fence_after();
-            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                   abuf * C::kAccCols;
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + abuf * wn;
             const int row = t.row0 + q * 32 + lane;
             tm_epilogue<GATE_UP>(p, tbase, row, row < t.row_end, t.i, (warp - 2) >> 2,
-                                 GATE_UP ? nullptr : epi_stage(g_tile + p.G + 1, warp));
+                                 GATE_UP ? nullptr : epi_stage(g_tile + p.G + 1, warp), wn,
+                                 ex ? x_base : -1);
             tc_fence_before();
             mbar_arrive(&tempty[abuf]);
             abuf ^= 1u;
@@ -1016,7 +1162,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_w,
                                    abuf * C::kAccCols;
             const int row = t.row0 + static_cast<int>(rank) * kTmRows + q * 32 + lane;
             tm_epilogue<GATE_UP>(p, tbase, row, row < t.row_end, t.i, (warp - 2) >> 2,
-                                 GATE_UP ? nullptr : epi_stage(g_tile + p.G + 1, warp));
+                                 GATE_UP ? nullptr : epi_stage(g_tile + p.G + 1, warp), kTmN);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_tempty0 + abuf * 8);
@@ -1082,17 +1228,17 @@ cudaError_t launch_tpl(const CUtensorMap& mw, const CUtensorMap& ma, const Param
 }
 
 template <bool GATE_UP>
-cudaError_t launch_tm(const CUtensorMap& mw, const CUtensorMap& ma, const Params& p, int grid,
-                      cudaStream_t s, bool pdl) {
-    using C = CfgTm<GATE_UP>;
-    const size_t smem = 1024 + static_cast<size_t>(C::kStages) * C::kStageBytes +
-                        (2 * C::kStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int) +
+cudaError_t launch_tm(const CUtensorMap& mw, const CUtensorMap& ma, const CUtensorMap& mw2,
+                      const Params& p, int grid, cudaStream_t s, bool pdl) {
+    using C = CfgTm;
+    const size_t smem = 1024 + static_cast<size_t>(C::kRingBytes) +
+                        (2 * C::kMaxStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int) +
                         (GATE_UP ? 0 : kEpiStageBytes);
     auto kfn = grouped_gemm_tm_kernel<GATE_UP>;
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    err = launch_kernel(kfn, dim3(grid), dim3(kTmThreads), smem, s, pdl, mw, ma, p);
+    err = launch_kernel(kfn, dim3(grid), dim3(kTmThreads), smem, s, pdl, mw, ma, mw2, p);
     count_launches(1);
     return err;
 }
@@ -1150,7 +1296,16 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
     const uint64_t w_group_rows = a.gate_up ? 2ull * a.f : static_cast<uint64_t>(a.D);
     CUtensorMap mw, ma;
     cudaError_t err;
-    if ((err = make_map(&mw, a.w, w_group_rows * a.E, K, kBM)) != cudaSuccess) return err;  // 128-row boxes
+    // weight boxes: 32 rows for the one-CTA tokens-on-M kernel (its tile width is chosen on
+    // the device), 128 rows otherwise
+    if ((err = make_map(&mw, a.w, w_group_rows * a.E, K, kind == Kind::kTm ? kWBox : kBM)) !=
+        cudaSuccess)
+        return err;
+    // the extra dense group's weights (one CTA tokens-on-M only), else a copy of mw
+    CUtensorMap mw2 = mw;
+    if (a.xg_w != nullptr &&
+        (err = make_map(&mw2, a.xg_w, w_group_rows, K, kWBox)) != cudaSuccess)
+        return err;
     // the activation map is only read when the rows are contiguous (no gather); with a
     // gather it still has to be a valid descriptor, so it covers the first row of x
     const void* act = a.act;
@@ -1191,19 +1346,27 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
     p.ksplit = kind == Kind::kSwap && a.ksplit > 1 ? a.ksplit : 1;
     p.zero_acc = a.gate_up ? a.zero_acc : nullptr;
     p.zero_n4 = a.zero_floats / 4;
+    p.tm_adaptive = kind == Kind::kTm ? 1 : 0;
+    if (a.xg_w != nullptr) {
+        p.xg = 1;
+        p.G = a.E + 1;
+        p.xg_rows = a.xg_rows;
+        p.xg_weight = a.xg_weight;
+    }
     p.split_stride = static_cast<long long>(a.rows) * p.out_cols;
     // persistent grids: one CTA (or pair) per SM, fewer when the tiles cannot fill them
     const int rows_per_tile = kind == Kind::kPair ? CfgPair::kPairRows : (tm ? kTmRows : 16);
-    const long long max_tiles =
-        (static_cast<long long>(ceil_div(a.rows, rows_per_tile)) + a.E) * p.nf * p.ksplit;
+    // (the one-CTA tokens-on-M kernel may cut its tiles up to 4x narrower on the device)
+    const long long max_tiles = (static_cast<long long>(ceil_div(a.rows, rows_per_tile)) + p.G) *
+                                p.nf * p.ksplit * (kind == Kind::kTm ? 4 : 1);
     if (kind == Kind::kPair) {
         const int npairs = static_cast<int>(std::min<long long>(max_tiles, num_sms / 2));
         return a.gate_up ? launch_pair<true>(mw, ma, p, npairs, s, true)
                          : launch_pair<false>(mw, ma, p, npairs, s, true);
     }
     const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
-    if (tm) return a.gate_up ? launch_tm<true>(mw, ma, p, grid, s, pdl)
-                             : launch_tm<false>(mw, ma, p, grid, s, pdl);
+    if (tm) return a.gate_up ? launch_tm<true>(mw, ma, mw2, p, grid, s, pdl)
+                             : launch_tm<false>(mw, ma, mw2, p, grid, s, pdl);
     switch (BN) {
         case 16: return a.gate_up ? launch_tpl<16, true>(mw, ma, p, grid, s, pdl) : launch_tpl<16, false>(mw, ma, p, grid, s, pdl);
         case 32: return a.gate_up ? launch_tpl<32, true>(mw, ma, p, grid, s, pdl) : launch_tpl<32, false>(mw, ma, p, grid, s, pdl);
@@ -1214,44 +1377,74 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
 
 }  // namespace
 
-cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s,
-                                bool pdl) {
-    if (a.rows == 0 || a.E == 0) return cudaSuccess;
-    if (a.E > kMaxGroups) return cudaErrorInvalidValue;
-    cudaError_t err = get_encoder();
-    if (err != cudaSuccess) return err;
+namespace {
+
+// Kernel kind and weights-on-M tile height for a launch (see launch_grouped_gemm).
+bool pick_kind(const GroupedGemmLaunch& a, int num_sms, Kind* kind, int* BN) {
     // tokens on M needs f (gate_up) or D (down) in 128- or 256-wide blocks
     const bool tm_ok = a.gate_up ? (a.f % 128 == 0) : (a.D % 256 == 0);
     const bool gathered = a.gate_up && a.gather_tok != nullptr;
     const bool pair_ok = tm_ok && (!gathered || a.gather_buf != nullptr) && num_sms >= 2;
+    const int routed_rows = a.rows - (a.xg_w != nullptr ? a.xg_rows : 0);
     // weights on M: tiles adapt per group up to BN, sized for groups up to 8x the average
     // (skewed routing) but never past the largest possible group
-    const int max_rows = a.max_group_rows > 0 ? a.max_group_rows : a.rows;
-    const long long avg8 = 8ll * a.rows / a.E;
+    const int max_rows = a.max_group_rows > 0 ? a.max_group_rows : routed_rows;
+    const long long avg8 = 8ll * routed_rows / a.E;
     const int bn_rows = static_cast<int>(std::min<long long>(max_rows, std::max(avg8, 16ll)));
-    const int BN = a.block_rows ? a.block_rows : pick_block_rows(bn_rows, 1);
-    if (BN != 16 && BN != 32 && BN != 64 && BN != 128) return cudaErrorInvalidValue;
-
-    // Orientation.  Weights on M (token tiles of 16..128 rows) when asked for, or while no
-    // group can hold more than kSwapMaxRows rows (a handful of tokens: the weight-read-bound
-    // regime, where a 128-row token tile would be nearly empty).  Otherwise tokens on M:
-    // both orientations stream each weight tile once per row block and are within a few
-    // percent of each other on 2-row groups, but tokens on M keeps features along the
-    // accumulator's columns (16-byte stores and vector reductions in the epilogue) and wins
-    // clearly once groups hold tens of rows.  CTA pairs once the groups average a full
-    // 256-row pair tile's half (their rows must be contiguous: x is gathered first).
+    *BN = a.block_rows ? a.block_rows : pick_block_rows(bn_rows, 1);
+    if (*BN != 16 && *BN != 32 && *BN != 64 && *BN != 128) return false;
     if (a.ksplit > 1 && (a.gate_up || !a.y_out || a.acc_out || a.final_out ||
                          (a.f / kBK) % a.ksplit != 0))
-        return cudaErrorInvalidValue;
-    Kind kind;
+        return false;
+    // Orientation.  Weights on M (token tiles of 16..128 rows) when asked for (the router's
+    // split-reduction logits GEMM), or when the tokens-on-M tiles do not divide the shape.
+    // Otherwise tokens on M: both orientations stream each weight tile once per row block
+    // and are within a few percent of each other on 2-row groups, but tokens on M keeps
+    // features along the accumulator's columns (16-byte stores and vector reductions in
+    // the epilogue), wins clearly once groups hold tens of rows, and picks its tile width
+    // on the device, so that a few experts (a handful of tokens, or concentrated routing)
+    // still spread their weight reads over the whole GPU.  CTA pairs once the groups
+    // average a full 256-row pair tile's half (their rows must be contiguous: x is
+    // gathered first).
     if (a.orientation == 1 || a.block_rows || !tm_ok || a.ksplit > 1)
-        kind = Kind::kSwap;
+        *kind = Kind::kSwap;
     else if (a.orientation == 2)
-        kind = Kind::kTm;
-    else if (a.orientation == 3 || a.rows / a.E >= 128)
-        kind = pair_ok ? Kind::kPair : Kind::kTm;
+        *kind = Kind::kTm;
+    else if (a.orientation == 3 || routed_rows / a.E >= 128)
+        *kind = pair_ok ? Kind::kPair : Kind::kTm;
     else
-        kind = max_rows <= kSwapMaxRows ? Kind::kSwap : Kind::kTm;
+        *kind = Kind::kTm;
+    return true;
+}
+
+}  // namespace
+
+int grouped_gemm_launches(const GroupedGemmLaunch& a, int num_sms) {
+    Kind kind;
+    int BN;
+    if (a.rows == 0 || a.E == 0 || !pick_kind(a, num_sms, &kind, &BN)) return 0;
+    return (kind == Kind::kPair && a.gate_up && a.gather_tok != nullptr) ? 2 : 1;
+}
+
+bool grouped_gemm_takes_extra_group(const GroupedGemmLaunch& a, int num_sms) {
+    Kind kind;
+    int BN;
+    return pick_kind(a, num_sms, &kind, &BN) && kind == Kind::kTm;
+}
+
+cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s,
+                                bool pdl) {
+    if (a.rows == 0 || a.E == 0) return cudaSuccess;
+    if (a.E + (a.xg_w != nullptr ? 1 : 0) > kMaxGroups) return cudaErrorInvalidValue;
+    cudaError_t err = get_encoder();
+    if (err != cudaSuccess) return err;
+    Kind kind;
+    int BN;
+    if (!pick_kind(a, num_sms, &kind, &BN)) return cudaErrorInvalidValue;
+    // an extra dense group (the shared expert) rides only on the one-CTA tokens-on-M kernel
+    if (a.xg_w != nullptr &&
+        (kind != Kind::kTm || a.offsets == nullptr || (!a.gate_up && a.xg_weight == nullptr)))
+        return cudaErrorInvalidValue;
     return launch_kind(a, kind, BN, num_sms, s, pdl);
 }
 

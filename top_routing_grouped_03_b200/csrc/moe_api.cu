@@ -55,7 +55,8 @@ Layout layout(long long T, long long D, long long E, long long K, long long f, l
         return r;
     };
     L.status = take(kAlign);
-    L.counters = take(sizeof(unsigned) * static_cast<size_t>((T + 7) / 8));
+    // one completion ticket per 8-token block, and one for the router's last block
+    L.counters = take(sizeof(unsigned) * static_cast<size_t>((T + 7) / 8 + 1));
     L.counts = take(sizeof(int32_t) * E);
     L.zero_end = o;
     // depends on T, E and K only, so any workspace sized for the same T, E, K has it here
@@ -74,7 +75,9 @@ Layout layout(long long T, long long D, long long E, long long K, long long f, l
     L.sorted_w = take(sizeof(float) * T * K);
     L.slot_to_row = take(sizeof(int32_t) * T * K);
     L.x_sorted = take(2 * T * K * D);
-    L.h = take(2 * T * K * f);
+    // h: the routed rows, then room for the shared expert's T rows when it runs as an extra
+    // group of the routed launches (f_s = f)
+    L.h = take(2 * (T * K + T) * f);
     L.h_s = take(2 * T * fs);
     L.out_acc = take(sizeof(float) * T * D);
     L.y_sorted = take(sizeof(float) * T * K * D);
@@ -96,6 +99,186 @@ inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s
 template <class P>
 P* at(void* ws, size_t off) {
     return reinterpret_cast<P*>(static_cast<uint8_t*>(ws) + off);
+}
+
+// Host checks of moe_layer_forward's parameters (out may be NULL when only planning).
+int check_layer(const moe_layer_params* p, const moe_bf16* out) {
+    if (!p) return MOE_ERR_ARG;
+    const int T = p->T, E = p->E, K = p->K;
+    int rc = check_shape(T, p->D, E, K, p->f, p->f_s);
+    if (rc) return rc;
+    const bool shared = p->f_s > 0;
+    if (!p->w_router || !p->w_gate_up || !p->w_down) return MOE_ERR_ARG;
+    if (shared && (!p->w_shared_gate || !p->w_shared_gate_up || !p->w_shared_down)) return MOE_ERR_ARG;
+    if (!shared && (p->w_shared_gate || p->w_shared_gate_up || p->w_shared_down)) return MOE_ERR_ARG;
+    if (p->score_mode != MOE_SCORE_SOFTMAX && p->score_mode != MOE_SCORE_SIGMOID) return MOE_ERR_ARG;
+    if (!(p->capacity_factor >= 0.f) || !std::isfinite(p->capacity_factor) || p->min_capacity < 0)
+        return MOE_ERR_ARG;
+    if (!aligned16(p->x) || !aligned16(p->w_router) || !aligned16(p->w_gate_up) ||
+        !aligned16(p->w_down) || !aligned16(out) || !aligned16(p->residual) ||
+        (shared && (!aligned16(p->w_shared_gate) || !aligned16(p->w_shared_gate_up) ||
+                    !aligned16(p->w_shared_down))))
+        return MOE_ERR_ALIGN;
+    return MOE_OK;
+}
+
+// Every launch of one layer call, and the choices that shape them.
+struct LayerPlan {
+    RouterLaunch r;
+    PermuteLaunch pm;
+    GroupedGemmLaunch up, dn, su, sd;
+    CombineLaunch c;
+    bool tc_router, det, fuse_shared, shared_launches;
+};
+
+LayerPlan plan_layer(const moe_layer_params* p, moe_bf16* out, void* workspace, int sms) {
+    const int T = p->T, D = p->D, E = p->E, K = p->K, f = p->f, fs = p->f_s;
+    const Layout L = layout(T, D, E, K, f, fs);
+    const bool shared = fs > 0;
+    // expert capacity (assignments per expert), or -1: dropless
+    const long long capacity = p->capacity_factor > 0.f
+                                   ? moe_expert_capacity(T, K, E, p->capacity_factor, p->min_capacity)
+                                   : -1;
+    LayerPlan q{};
+    q.det = (p->flags & MOE_FLAG_DETERMINISTIC) != 0;
+    q.tc_router = router_uses_tensor_cores(T, E);
+    int* status = at<int>(workspace, L.status);
+    // the router counts into the workspace (cleared with the header); the permutation
+    // copies the counts out when the caller asks for them
+    int32_t* counts = at<int32_t>(workspace, L.counts);
+    int32_t* idx = p->topk_idx_out ? p->topk_idx_out : at<int32_t>(workspace, L.topk_idx);
+    float* tw = p->topk_w_out ? p->topk_w_out : at<float>(workspace, L.topk_w);
+    float* sgate = at<float>(workspace, L.sgate);
+    float* out_acc = at<float>(workspace, L.out_acc);
+    const bool use_acc = !q.det || shared;
+
+    PermuteLaunch& pm = q.pm;
+    pm.topk_idx = idx;
+    pm.topk_w = tw;
+    // tensor-core router (many tokens): no per-entry count atomics in the selection; the
+    // permutation counts from its chunk histograms
+    pm.counts = q.tc_router ? nullptr : counts;
+    pm.counts_out = p->expert_counts_out;
+    pm.T = T; pm.E = E; pm.K = K;
+    pm.offsets = at<int32_t>(workspace, L.offsets);
+    pm.sorted_token = at<int32_t>(workspace, L.sorted_token);
+    pm.sorted_w = at<float>(workspace, L.sorted_w);
+    pm.slot_to_row = at<int32_t>(workspace, L.slot_to_row);
+    pm.dense_offsets = at<int32_t>(workspace, L.dense_offsets);
+    pm.status = status;
+    pm.hist = at<int32_t>(workspace, L.perm_hist);
+    pm.capacity = capacity;
+
+    RouterLaunch& r = q.r;
+    r.x = reinterpret_cast<const bf16*>(p->x);
+    r.w_router = reinterpret_cast<const bf16*>(p->w_router);
+    r.logit_bias = p->logit_bias;
+    r.w_shared_gate = shared ? reinterpret_cast<const bf16*>(p->w_shared_gate) : nullptr;
+    r.T = T; r.D = D; r.E = E; r.K = K;
+    r.logits = at<float>(workspace, L.logits);
+    r.counters = at<unsigned>(workspace, L.counters);
+    r.topk_idx = idx;
+    r.topk_w = tw;
+    r.counts = q.tc_router ? nullptr : counts;
+    r.shared_gate = sgate;
+    r.status = status;
+    r.zero_acc = use_acc && !q.tc_router ? out_acc : nullptr;
+    r.zero_cols = D;
+    r.score_mode = p->score_mode;
+    r.select_bias = p->select_bias;
+    r.bf16_weights = (p->flags & MOE_FLAG_BF16_WEIGHTS) ? 1 : 0;
+    // small problems: the router's last CTA also runs the permutation (one launch fewer)
+    if (router_can_fuse_permute(T, E, K)) {
+        r.fuse_perm = 1;
+        r.perm = pm;
+    }
+
+    const int rows = T * K;
+    GroupedGemmLaunch& up = q.up;
+    up.gate_up = true;
+    up.w = p->w_gate_up;
+    up.act = p->x;
+    up.gather_tok = pm.sorted_token;
+    up.gather_buf = at<bf16>(workspace, L.x_sorted);
+    up.offsets = pm.offsets;
+    up.rows = rows; up.E = E; up.D = D; up.f = f;
+    up.max_group_rows = capacity >= 0 && capacity < T ? static_cast<int>(capacity) : T;
+    up.h_out = at<bf16>(workspace, L.h);
+    up.status = status;
+    up.zero_acc = use_acc && q.tc_router ? out_acc : nullptr;
+    up.zero_floats = static_cast<long long>(T) * D;
+    // The shared expert (same width as the routed ones) runs as one more, dense group of the
+    // routed gate_up and down launches when they take the one-CTA tokens-on-M kernel: its
+    // compute-bound tiles then interleave with the weight-streaming routed tiles instead of
+    // running as two launches of their own.  Its rows follow the routed rows in h.
+    q.fuse_shared = shared && !q.det && fs == f && grouped_gemm_takes_extra_group(up, sms);
+    q.shared_launches = shared && !q.fuse_shared;
+    if (q.fuse_shared) {
+        up.xg_w = p->w_shared_gate_up;
+        up.xg_rows = T;
+        up.rows = rows + T;
+    }
+
+    GroupedGemmLaunch& dn = q.dn;
+    dn.gate_up = false;
+    dn.w = p->w_down;
+    dn.act = up.h_out;
+    dn.offsets = pm.offsets;
+    dn.sorted_token = pm.sorted_token;
+    dn.sorted_w = q.det ? nullptr : pm.sorted_w;
+    dn.rows = rows; dn.E = E; dn.D = D; dn.f = f;
+    dn.max_group_rows = up.max_group_rows;
+    dn.acc_out = q.det ? nullptr : out_acc;
+    dn.y_out = q.det ? at<float>(workspace, L.y_sorted) : nullptr;
+    dn.status = status;
+    if (q.fuse_shared) {
+        dn.xg_w = p->w_shared_down;
+        dn.xg_rows = T;
+        dn.xg_weight = sgate;
+        dn.rows = rows + T;
+    }
+    // without the fixed-order combine, the last launch also writes the bf16 output after a
+    // grid-wide step
+    unsigned* done = at<unsigned>(workspace, L.status + 64);  // inside the cleared header
+    const bf16* residual = reinterpret_cast<const bf16*>(p->residual);
+    GroupedGemmLaunch& last = q.shared_launches ? q.sd : dn;
+    if (!q.det) {
+        last.final_out = reinterpret_cast<bf16*>(out);
+        last.final_rows = T;
+        last.done = done;
+        last.final_residual = residual;
+        last.barrier_budget_ns = grid_wait_budget_ns();
+    }
+    if (q.shared_launches) {
+        GroupedGemmLaunch& su = q.su;
+        su.gate_up = true;
+        su.w = p->w_shared_gate_up;
+        su.act = p->x;
+        su.offsets = pm.dense_offsets;
+        su.rows = T; su.E = 1; su.D = D; su.f = fs;
+        su.h_out = at<bf16>(workspace, L.h_s);
+        su.status = status;
+        GroupedGemmLaunch& sd = q.sd;
+        sd.gate_up = false;
+        sd.w = p->w_shared_down;
+        sd.act = su.h_out;
+        sd.offsets = pm.dense_offsets;
+        sd.sorted_token = nullptr;
+        sd.sorted_w = sgate;
+        sd.rows = T; sd.E = 1; sd.D = D; sd.f = fs;
+        sd.acc_out = out_acc;
+        sd.status = status;
+    }
+    // fixed order: out_acc's shared part (if any) + the routed rows in slot order
+    CombineLaunch& c = q.c;
+    c.residual = residual;
+    c.out_acc = use_acc ? out_acc : nullptr;
+    c.y_sorted = q.det ? at<float>(workspace, L.y_sorted) : nullptr;
+    c.slot_to_row = pm.slot_to_row;
+    c.topk_w = q.det ? tw : nullptr;
+    c.T = T; c.D = D; c.K = K;
+    c.out = reinterpret_cast<bf16*>(out);
+    return q;
 }
 
 }  // namespace
@@ -292,182 +475,70 @@ int moe_combine(const float* out_acc, const float* y_sorted, const int32_t* slot
 
 int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace, size_t ws_bytes,
                       void* stream) {
-    if (!p) return MOE_ERR_ARG;
-    const int T = p->T, D = p->D, E = p->E, K = p->K, f = p->f, fs = p->f_s;
-    int rc = check_shape(T, D, E, K, f, fs);
+    int rc = check_layer(p, out);
     if (rc) return rc;
-    const bool shared = fs > 0;
-    if (!p->w_router || !p->w_gate_up || !p->w_down) return MOE_ERR_ARG;
-    if (T > 0 && (!p->x || !out)) return MOE_ERR_ARG;
-    if (shared && (!p->w_shared_gate || !p->w_shared_gate_up || !p->w_shared_down)) return MOE_ERR_ARG;
-    if (!shared && (p->w_shared_gate || p->w_shared_gate_up || p->w_shared_down)) return MOE_ERR_ARG;
-    if (p->score_mode != MOE_SCORE_SOFTMAX && p->score_mode != MOE_SCORE_SIGMOID) return MOE_ERR_ARG;
-    if (!(p->capacity_factor >= 0.f) || !std::isfinite(p->capacity_factor) || p->min_capacity < 0)
-        return MOE_ERR_ARG;
-    // expert capacity (assignments per expert), or -1: dropless
-    const long long capacity = p->capacity_factor > 0.f
-                                   ? moe_expert_capacity(T, K, E, p->capacity_factor, p->min_capacity)
-                                   : -1;
-    if (!aligned16(p->x) || !aligned16(p->w_router) || !aligned16(p->w_gate_up) ||
-        !aligned16(p->w_down) || !aligned16(out) || !aligned16(p->residual) ||
-        (shared && (!aligned16(p->w_shared_gate) || !aligned16(p->w_shared_gate_up) ||
-                    !aligned16(p->w_shared_down))))
-        return MOE_ERR_ALIGN;
+    if (p->T > 0 && (!p->x || !out)) return MOE_ERR_ARG;
     if (!workspace) return MOE_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return MOE_ERR_ALIGN;
-    const Layout L = layout(T, D, E, K, f, fs);
+    const Layout L = layout(p->T, p->D, p->E, p->K, p->f, p->f_s);
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-    if (T == 0) return MOE_OK;
+    if (p->T == 0) return MOE_OK;
 
     cudaStream_t s = as_stream(stream);
     const int sms = num_sms_current();
-    const bool det = (p->flags & MOE_FLAG_DETERMINISTIC) != 0;
+    LayerPlan q = plan_layer(p, out, workspace, sms);
     auto mark = [&](int i) {
         return p->step_events == nullptr || p->step_events[i] == nullptr ||
                cudaEventRecord(reinterpret_cast<cudaEvent_t>(p->step_events[i]), s) == cudaSuccess;
     };
-    int* status = at<int>(workspace, L.status);
-    int32_t* counts = p->expert_counts_out ? p->expert_counts_out : at<int32_t>(workspace, L.counts);
-    int32_t* idx = p->topk_idx_out ? p->topk_idx_out : at<int32_t>(workspace, L.topk_idx);
-    float* tw = p->topk_w_out ? p->topk_w_out : at<float>(workspace, L.topk_w);
-    float* sgate = at<float>(workspace, L.sgate);
-    float* out_acc = at<float>(workspace, L.out_acc);
 
     if (!mark(MOE_EV_START)) return MOE_ERR_CUDA;
     // the only clear: status word, router tickets, expert counts (a few KB); the fp32
     // accumulator is cleared by the CUDA-core router kernel, or (tensor-core router, many
     // tokens) by the gate_up kernel's epilogue warps while its first tiles accumulate
     if (cudaMemsetAsync(workspace, 0, L.zero_end, s) != cudaSuccess) return MOE_ERR_CUDA;
-    if (p->expert_counts_out && cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    const bool use_acc = !det || shared;
-
-    const bool tc_router = router_uses_tensor_cores(T, E);
-    RouterLaunch r{};
-    r.x = reinterpret_cast<const bf16*>(p->x);
-    r.w_router = reinterpret_cast<const bf16*>(p->w_router);
-    r.logit_bias = p->logit_bias;
-    r.w_shared_gate = shared ? reinterpret_cast<const bf16*>(p->w_shared_gate) : nullptr;
-    r.T = T; r.D = D; r.E = E; r.K = K;
-    r.logits = at<float>(workspace, L.logits);
-    r.counters = at<unsigned>(workspace, L.counters);
-    r.topk_idx = idx;
-    r.topk_w = tw;
-    // tensor-core router (many tokens): no per-entry count atomics in the selection; the
-    // permutation counts from its chunk histograms
-    r.counts = tc_router ? nullptr : counts;
-    r.shared_gate = sgate;
-    r.status = status;
-    r.zero_acc = use_acc && !tc_router ? out_acc : nullptr;
-    r.zero_cols = D;
-    r.score_mode = p->score_mode;
-    r.select_bias = p->select_bias;
-    r.bf16_weights = (p->flags & MOE_FLAG_BF16_WEIGHTS) ? 1 : 0;
     if (!mark(MOE_EV_ROUTER)) return MOE_ERR_CUDA;
-    if ((tc_router ? launch_router_tc(r, sms, s) : launch_router(r, sms, s)) != cudaSuccess)
+    if ((q.tc_router ? launch_router_tc(q.r, sms, s) : launch_router(q.r, sms, s)) != cudaSuccess)
         return MOE_ERR_CUDA;
-
-    PermuteLaunch pm{};
-    pm.topk_idx = idx;
-    pm.topk_w = tw;
-    pm.counts = tc_router ? nullptr : counts;
-    pm.counts_out = tc_router ? p->expert_counts_out : nullptr;
-    pm.T = T; pm.E = E; pm.K = K;
-    pm.offsets = at<int32_t>(workspace, L.offsets);
-    pm.sorted_token = at<int32_t>(workspace, L.sorted_token);
-    pm.sorted_w = at<float>(workspace, L.sorted_w);
-    pm.slot_to_row = at<int32_t>(workspace, L.slot_to_row);
-    pm.dense_offsets = at<int32_t>(workspace, L.dense_offsets);
-    pm.status = status;
-    pm.hist = at<int32_t>(workspace, L.perm_hist);
-    pm.capacity = capacity;
-    if (!mark(MOE_EV_PERMUTE) || launch_permute(pm, s, true) != cudaSuccess) return MOE_ERR_CUDA;
-
-    const int rows = T * K;
-    GroupedGemmLaunch up{};
-    up.gate_up = true;
-    up.w = p->w_gate_up;
-    up.act = p->x;
-    up.gather_tok = pm.sorted_token;
-    up.gather_buf = at<bf16>(workspace, L.x_sorted);
-    up.offsets = pm.offsets;
-    up.rows = rows; up.E = E; up.D = D; up.f = f;
-    up.max_group_rows = capacity >= 0 && capacity < T ? static_cast<int>(capacity) : T;
-    up.h_out = at<bf16>(workspace, L.h);
-    up.status = status;
-    up.zero_acc = use_acc && tc_router ? out_acc : nullptr;
-    up.zero_floats = static_cast<long long>(T) * D;
-    if (!mark(MOE_EV_GATE_UP) || launch_grouped_gemm(up, sms, s, true) != cudaSuccess)
+    if (!mark(MOE_EV_PERMUTE)) return MOE_ERR_CUDA;
+    if (!q.r.fuse_perm && launch_permute(q.pm, s, true) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!mark(MOE_EV_GATE_UP) || launch_grouped_gemm(q.up, sms, s, true) != cudaSuccess)
         return MOE_ERR_CUDA;
-
-    GroupedGemmLaunch dn{};
-    dn.gate_up = false;
-    dn.w = p->w_down;
-    dn.act = up.h_out;
-    dn.offsets = pm.offsets;
-    dn.sorted_token = pm.sorted_token;
-    dn.sorted_w = det ? nullptr : pm.sorted_w;
-    dn.rows = rows; dn.E = E; dn.D = D; dn.f = f;
-    dn.max_group_rows = up.max_group_rows;
-    dn.acc_out = det ? nullptr : out_acc;
-    dn.y_out = det ? at<float>(workspace, L.y_sorted) : nullptr;
-    dn.status = status;
-    // without the fixed-order combine, the last down launch also writes the bf16 output
-    unsigned* done = at<unsigned>(workspace, L.status + 64);  // inside the cleared header
-    const bf16* residual = reinterpret_cast<const bf16*>(p->residual);
-    if (!det && !shared) {
-        dn.final_out = reinterpret_cast<bf16*>(out);
-        dn.final_rows = T;
-        dn.done = done;
-        dn.final_residual = residual;
-        dn.barrier_budget_ns = grid_wait_budget_ns();
-    }
-    if (!mark(MOE_EV_DOWN) || launch_grouped_gemm(dn, sms, s, true) != cudaSuccess)
+    if (!mark(MOE_EV_DOWN) || launch_grouped_gemm(q.dn, sms, s, true) != cudaSuccess)
         return MOE_ERR_CUDA;
-
     if (!mark(MOE_EV_SHARED)) return MOE_ERR_CUDA;
-    if (shared) {
-        GroupedGemmLaunch su{};
-        su.gate_up = true;
-        su.w = p->w_shared_gate_up;
-        su.act = p->x;
-        su.offsets = pm.dense_offsets;
-        su.rows = T; su.E = 1; su.D = D; su.f = fs;
-        su.h_out = at<bf16>(workspace, L.h_s);
-        su.status = status;
-        if (launch_grouped_gemm(su, sms, s, true) != cudaSuccess) return MOE_ERR_CUDA;
-        GroupedGemmLaunch sd{};
-        sd.gate_up = false;
-        sd.w = p->w_shared_down;
-        sd.act = su.h_out;
-        sd.offsets = pm.dense_offsets;
-        sd.sorted_token = nullptr;
-        sd.sorted_w = sgate;
-        sd.rows = T; sd.E = 1; sd.D = D; sd.f = fs;
-        sd.acc_out = out_acc;
-        sd.status = status;
-        if (!det) {
-            sd.final_out = reinterpret_cast<bf16*>(out);
-            sd.final_rows = T;
-            sd.done = done;
-            sd.final_residual = residual;
-            sd.barrier_budget_ns = grid_wait_budget_ns();
-        }
-        if (launch_grouped_gemm(sd, sms, s, true) != cudaSuccess) return MOE_ERR_CUDA;
-    }
-
-    if (!det) return mark(MOE_EV_COMBINE) && mark(MOE_EV_END) ? MOE_OK : MOE_ERR_CUDA;
-    // fixed order: out_acc's shared part (if any) + the routed rows in slot order
-    CombineLaunch c{};
-    c.residual = residual;
-    c.out_acc = use_acc ? out_acc : nullptr;
-    c.y_sorted = det ? at<float>(workspace, L.y_sorted) : nullptr;
-    c.slot_to_row = pm.slot_to_row;
-    c.topk_w = det ? tw : nullptr;
-    c.T = T; c.D = D; c.K = K;
-    c.out = reinterpret_cast<bf16*>(out);
-    if (!mark(MOE_EV_COMBINE) || launch_combine(c, sms, s, true) != cudaSuccess) return MOE_ERR_CUDA;
+    if (q.shared_launches &&
+        (launch_grouped_gemm(q.su, sms, s, true) != cudaSuccess ||
+         launch_grouped_gemm(q.sd, sms, s, true) != cudaSuccess))
+        return MOE_ERR_CUDA;
+    if (!mark(MOE_EV_COMBINE)) return MOE_ERR_CUDA;
+    if (q.det && launch_combine(q.c, sms, s, true) != cudaSuccess) return MOE_ERR_CUDA;
     return mark(MOE_EV_END) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_layer_plan(const moe_layer_params* p, unsigned* step_mask, int* launches) {
+    int rc = check_layer(p, nullptr);
+    if (rc) return rc;
+    unsigned mask = 0;
+    int n = 0;
+    if (p->T > 0) {
+        const int sms = num_sms_current();
+        // nothing is dereferenced: the plan only needs the workspace's layout
+        const LayerPlan q = plan_layer(p, nullptr, reinterpret_cast<void*>(kAlign), sms);
+        const int nr = q.tc_router ? 2 : 1;
+        const int np = q.r.fuse_perm ? 0 : (permute_chunks(static_cast<long long>(p->T) * p->K) > 1 ? 2 : 1);
+        const int nu = grouped_gemm_launches(q.up, sms), nd = grouped_gemm_launches(q.dn, sms);
+        const int ns = q.shared_launches ? grouped_gemm_launches(q.su, sms) + grouped_gemm_launches(q.sd, sms) : 0;
+        const int nc = q.det ? 1 : 0;
+        const int per[] = {nr, np, nu, nd, ns, nc};
+        for (int i = 0; i < 6; ++i) {
+            if (per[i]) mask |= 1u << (MOE_EV_ROUTER + i);
+            n += per[i];
+        }
+    }
+    if (step_mask) *step_mask = mask;
+    if (launches) *launches = n;
+    return MOE_OK;
 }
 
 int moe_read_device_status(void* workspace, void* stream) {

@@ -207,6 +207,18 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// tcgen05.wait::ld that also takes r as an operand, so that no use of the registers a
+// tcgen05.ld is still filling can be scheduled before the wait (for loads left in flight
+// while other work runs).
+__device__ __forceinline__ void tmem_ld_wait_dep(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+}
+
 // Shared-memory matrix descriptor of a K-major operand tile stored the way a TMA load
 // with 128-byte swizzle writes it: rows of 64 bf16 (128 B), 8-row atoms of 1024 B.
 // Start address >> 4 in bits [0,14); leading byte offset (unused for this layout, 16 B)

@@ -26,6 +26,7 @@
 #include <cfloat>
 
 #include "common.cuh"
+#include "permute_body.cuh"
 
 namespace moe {
 namespace {
@@ -285,6 +286,21 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
             a.shared_gate[token] = 1.f / (1.f + expf(-g));
         }
     }
+    if (!a.fuse_perm) return;
+
+    // ---- the last token block to finish its selection also groups every (token, slot)
+    //      entry by expert: the routing and the counts of all blocks are then complete
+    __shared__ int s_perm;
+    __threadfence();  // this CTA's routing and counts are visible before its ticket
+    __syncthreads();
+    if (tid == 0) {
+        const unsigned prev = atomicAdd(&a.counters[gridDim.x], 1u);
+        s_perm = (prev == gridDim.x - 1) ? 1 : 0;
+    }
+    __syncthreads();
+    if (!s_perm) return;
+    __threadfence();
+    permute_scatter_chunk<kRouterThreads>(a.perm, a.T * a.K, 1, 0, reinterpret_cast<int*>(xs));
 }
 
 
@@ -306,16 +322,29 @@ __global__ void __launch_bounds__(kRouterThreads) router_select_kernel(RouterLau
         const uint4* xv = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(token) * a.D);
         const uint4* wv = reinterpret_cast<const uint4*>(a.w_shared_gate);
         float acc = 0.f;
-        for (int c = lane; c < a.D / 8; c += 32) {
-            const uint4 x8 = __ldg(xv + c), w8 = __ldg(wv + c);
-            acc = fmaf(bf16_lo(x8.x), bf16_lo(w8.x), acc);
-            acc = fmaf(bf16_hi(x8.x), bf16_hi(w8.x), acc);
-            acc = fmaf(bf16_lo(x8.y), bf16_lo(w8.y), acc);
-            acc = fmaf(bf16_hi(x8.y), bf16_hi(w8.y), acc);
-            acc = fmaf(bf16_lo(x8.z), bf16_lo(w8.z), acc);
-            acc = fmaf(bf16_hi(x8.z), bf16_hi(w8.z), acc);
-            acc = fmaf(bf16_lo(x8.w), bf16_lo(w8.w), acc);
-            acc = fmaf(bf16_hi(x8.w), bf16_hi(w8.w), acc);
+        // 8 chunks of x and w_s per lane in flight at a time (D = 4096 is 16 chunks a lane:
+        // two round trips to memory instead of sixteen)
+        constexpr int kBatch = 8;
+        for (int c0 = lane; c0 < a.D / 8; c0 += 32 * kBatch) {
+            uint4 x8[kBatch], w8[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int c = c0 + 32 * u;
+                const bool in = c < a.D / 8;
+                x8[u] = in ? __ldg(xv + c) : make_uint4(0, 0, 0, 0);
+                w8[u] = in ? __ldg(wv + c) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                acc = fmaf(bf16_lo(x8[u].x), bf16_lo(w8[u].x), acc);
+                acc = fmaf(bf16_hi(x8[u].x), bf16_hi(w8[u].x), acc);
+                acc = fmaf(bf16_lo(x8[u].y), bf16_lo(w8[u].y), acc);
+                acc = fmaf(bf16_hi(x8[u].y), bf16_hi(w8[u].y), acc);
+                acc = fmaf(bf16_lo(x8[u].z), bf16_lo(w8[u].z), acc);
+                acc = fmaf(bf16_hi(x8[u].z), bf16_hi(w8[u].z), acc);
+                acc = fmaf(bf16_lo(x8[u].w), bf16_lo(w8[u].w), acc);
+                acc = fmaf(bf16_hi(x8[u].w), bf16_hi(w8[u].w), acc);
+            }
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -335,7 +364,15 @@ cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bo
     n_eb = max(1, min(n_eb, ceil_div(rows_total, rows_per_pass)));
     int per_cta = ceil_div(ceil_div(rows_total, n_eb), rows_per_pass) * rows_per_pass;
     n_eb = ceil_div(rows_total, per_cta);
-    const size_t smem = static_cast<size_t>(kTokensPerCta) * a.D * sizeof(bf16);
+    size_t smem = static_cast<size_t>(kTokensPerCta) * a.D * sizeof(bf16);
+    if (a.fuse_perm) {
+        if (!router_can_fuse_permute(a.T, a.E, a.K) || a.perm.counts != a.counts)
+            return cudaErrorInvalidValue;
+        // the permutation reuses the token staging area (its tables: 8 warps' counts and
+        // three per-expert arrays)
+        smem = std::max(smem, sizeof(int) * (static_cast<size_t>(kRouterThreads / 32) * a.E +
+                                             3 * a.E + 1));
+    }
     cudaError_t err = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
@@ -347,6 +384,11 @@ cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bo
 
 
 bool router_uses_tensor_cores(int T, int E) { return T >= 256 && E % 128 == 0; }
+
+bool router_can_fuse_permute(int T, int E, int K) {
+    return !router_uses_tensor_cores(T, E) && E <= kRouterThreads &&
+           static_cast<long long>(T) * K <= 4096;
+}
 
 int router_tc_max_planes(int T) { return std::min(16, std::max(1, 512 / ceil_div(T, 128))); }
 
