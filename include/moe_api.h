@@ -265,6 +265,48 @@ typedef struct moe_layer_params {
 } moe_layer_params;
 
 /*
+ * Expert parallelism ("1.6 混合专家（MoE）", expert parallelism; "Qwen3.8-Flash-Next 架构笔记 ·
+ * 04 / FFN & MOE", system costs): the E experts are spread over G devices, rank r holding
+ * experts [r*El, (r+1)*El) with El = E / G.  Every rank routes and permutes its own tokens
+ * (moe_route, moe_permute); the rows bound for rank d are then the contiguous range
+ * [offsets[d*El], offsets[(d+1)*El]) of its expert-sorted order, so dispatch is one
+ * all-to-all of the rows gathered into that order (moe_ep_dispatch_rows), with the
+ * per-expert counts of those ranges exchanged first ([G, El] int32, counts[d*El + e] to
+ * rank d).  The receiving rank groups what it received by expert (moe_ep_recv_layout), runs
+ * moe_grouped_swiglu on its El experts gathering the received rows through recv_row
+ * (sorted_token = recv_row, expert_offsets = recv_offsets, unweighted, y_sorted output),
+ * puts the outputs back into receive order (moe_ep_return_rows) and sends them back with
+ * the reverse all-to-all; each source then has its rows' expert outputs in its own sorted
+ * order and sums them with moe_combine (y_sorted, slot_to_row, topk_w).  The exchanges
+ * themselves are the caller's (NCCL all-to-all over NVLink between one process per GPU).
+ */
+
+/* x_sorted[r] = x[sorted_token[r]] for r < rows: the token rows in expert-sorted order,
+ * ready to send ([rows, D] bf16, D a multiple of 8).  */
+MOE_API int moe_ep_dispatch_rows(const moe_bf16* x, const int32_t* sorted_token, int rows, int D,
+                                 moe_bf16* x_sorted, void* stream);
+
+/*
+ * Receive side of the dispatch: recv_counts [G, El] (device) holds the rows source s sent for
+ * local expert e; the receive buffer holds n = sum(recv_counts) rows, source by source,
+ * each source's rows in expert order.  Writes recv_offsets [El+1] (rows of local expert e
+ * are [recv_offsets[e], recv_offsets[e+1]) of the expert-major order) and recv_row [n]
+ * (expert-major row j reads receive-buffer row recv_row[j]; within an expert, sources in
+ * rank order).  G * El <= 512.  workspace: NULL or a layer workspace whose status word
+ * records MOE_ERR_DEVICE when the counts do not add up to n -- every group is then empty and
+ * recv_row is not written.
+ */
+MOE_API int moe_ep_recv_layout(const int32_t* recv_counts, int G, int El, int n,
+                               int32_t* recv_offsets, int32_t* recv_row, void* workspace,
+                               void* stream);
+
+/* y_ret[recv_row[j], :] = y[j, :] for j < n: expert outputs (fp32 [n, D], expert-major, as
+ * moe_grouped_swiglu wrote them) back into receive-buffer order for the return all-to-all;
+ * D a multiple of 4; a recv_row entry outside [0, n) is skipped. */
+MOE_API int moe_ep_return_rows(const float* y, const int32_t* recv_row, int n, int D,
+                               float* y_ret, void* stream);
+
+/*
  * The expert capacity the layer applies: max(min_capacity, ceil(capacity_factor * T * K / E))
  * assignments per expert -- the batch's T*K (token, expert) assignments spread over E
  * experts, times the capacity factor (for top-1 routing this is the pages' tokens / experts

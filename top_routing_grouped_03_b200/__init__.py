@@ -91,6 +91,12 @@ def lib() -> ctypes.CDLL:
         L.moe_route_noalloc.restype = I
         L.moe_launch_count.argtypes = []
         L.moe_launch_count.restype = ctypes.c_ulonglong
+        L.moe_ep_dispatch_rows.argtypes = [P, P, I, I, P, P]
+        L.moe_ep_dispatch_rows.restype = I
+        L.moe_ep_recv_layout.argtypes = [P, I, I, I, P, P, P, P]
+        L.moe_ep_recv_layout.restype = I
+        L.moe_ep_return_rows.argtypes = [P, P, I, I, P, P]
+        L.moe_ep_return_rows.restype = I
         L.moe_layer_plan.argtypes = [ctypes.POINTER(LayerParams), P, P]
         L.moe_layer_plan.restype = I
         L.moe_set_grid_wait_budget_ns.argtypes = [ctypes.c_ulonglong]
@@ -240,6 +246,33 @@ def combine(T, D, K, out=None, out_acc=None, y_sorted=None, slot_to_row=None, to
                            _p(topk_w, F32), _p(shared_out, BF16), _p(shared_gate, F32), T, D, K,
                            _p(out, BF16), _stream(stream))
     _check(rc, "moe_combine")
+    return out
+
+
+def ep_dispatch_rows(x, sorted_token, rows, stream=None):
+    """x_sorted [rows, D] bf16 = x[sorted_token[:rows]] (moe_ep_dispatch_rows)."""
+    out = torch.empty((rows, x.shape[1]), dtype=BF16, device=x.device)
+    _check(lib().moe_ep_dispatch_rows(_p(x, BF16), _p(sorted_token, I32), rows, x.shape[1],
+                                      _p(out, BF16), _stream(stream)), "moe_ep_dispatch_rows")
+    return out
+
+
+def ep_recv_layout(recv_counts, n, workspace=None, stream=None):
+    """(recv_offsets [El+1], recv_row [n]) from the received counts [G, El] (device int32)."""
+    G, El = recv_counts.shape
+    off = torch.empty((El + 1,), dtype=I32, device=recv_counts.device)
+    row = torch.empty((n,), dtype=I32, device=recv_counts.device)
+    _check(lib().moe_ep_recv_layout(_p(recv_counts, I32), G, El, n, _p(off), _p(row),
+                                    _p(workspace, U8), _stream(stream)), "moe_ep_recv_layout")
+    return off, row
+
+
+def ep_return_rows(y, recv_row, stream=None):
+    """y_ret [n, D] fp32 with y_ret[recv_row[j]] = y[j] (moe_ep_return_rows)."""
+    n, D = y.shape
+    out = torch.empty_like(y)
+    _check(lib().moe_ep_return_rows(_p(y, F32), _p(recv_row, I32), n, D, _p(out, F32),
+                                    _stream(stream)), "moe_ep_return_rows")
     return out
 
 

@@ -11,7 +11,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoe_b200.so")
-SOURCES = ["router.cu", "permute.cu", "grouped_gemm.cu", "combine.cu", "moe_api.cu",
+SOURCES = ["router.cu", "permute.cu", "grouped_gemm.cu", "combine.cu", "ep.cu", "moe_api.cu",
            "route_noalloc.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

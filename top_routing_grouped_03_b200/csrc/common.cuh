@@ -188,6 +188,14 @@ cudaError_t launch_gather_rows(const bf16* x, const int32_t* tok, int rows, int 
 cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s,
                                 bool pdl = false);
 
+// expert parallelism (ep.cu): receive-side grouping and the return of the expert rows
+size_t ep_recv_layout_smem(int G, int El);
+cudaError_t launch_ep_recv_layout(const int32_t* recv_counts, int G, int El, int n,
+                                  int32_t* recv_offsets, int32_t* recv_row, int* status,
+                                  cudaStream_t s);
+cudaError_t launch_ep_return_rows(const float* y, const int32_t* recv_row, int n, int D,
+                                  float* y_ret, int num_sms, cudaStream_t s);
+
 struct CombineLaunch {
     const bf16* residual;  // [T, D] added before the bf16 rounding, or NULL
     const float* out_acc;

@@ -541,6 +541,41 @@ int moe_layer_plan(const moe_layer_params* p, unsigned* step_mask, int* launches
     return MOE_OK;
 }
 
+int moe_ep_dispatch_rows(const moe_bf16* x, const int32_t* sorted_token, int rows, int D,
+                         moe_bf16* x_sorted, void* stream) {
+    if (rows < 0 || D <= 0 || D % 8) return MOE_ERR_ARG;
+    if (rows > 0 && (!x || !sorted_token || !x_sorted)) return MOE_ERR_ARG;
+    if (!aligned16(x) || !aligned16(x_sorted)) return MOE_ERR_ALIGN;
+    return launch_gather_rows(reinterpret_cast<const bf16*>(x), sorted_token, rows, D,
+                              reinterpret_cast<bf16*>(x_sorted), num_sms_current(),
+                              as_stream(stream), false) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+int moe_ep_recv_layout(const int32_t* recv_counts, int G, int El, int n, int32_t* recv_offsets,
+                       int32_t* recv_row, void* workspace, void* stream) {
+    if (G <= 0 || El <= 0 || n < 0) return MOE_ERR_ARG;
+    if (static_cast<long long>(G) * El > 512) return MOE_ERR_UNSUPPORTED;
+    if (!recv_counts || !recv_offsets || (n > 0 && !recv_row)) return MOE_ERR_ARG;
+    return launch_ep_recv_layout(recv_counts, G, El, n, recv_offsets, recv_row,
+                                 workspace ? at<int>(workspace, 0) : nullptr,
+                                 as_stream(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+int moe_ep_return_rows(const float* y, const int32_t* recv_row, int n, int D, float* y_ret,
+                       void* stream) {
+    if (n < 0 || D <= 0 || D % 4) return MOE_ERR_ARG;
+    if (n > 0 && (!y || !recv_row || !y_ret)) return MOE_ERR_ARG;
+    if (!aligned16(y) || !aligned16(y_ret)) return MOE_ERR_ALIGN;
+    return launch_ep_return_rows(y, recv_row, n, D, y_ret, num_sms_current(),
+                                 as_stream(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
 int moe_read_device_status(void* workspace, void* stream) {
     if (!workspace) return MOE_ERR_WORKSPACE;
     cudaStream_t s = as_stream(stream);

@@ -66,6 +66,10 @@ CONFIGS = {
 # the prefill layer's per-expert shape (512 rows per expert, D=4096, f=1536) with 32 experts:
 # the same kernels and tiles on ~1.2 GB of weights, small enough for profiler captures
 CONFIGS["prefill_e32"] = LayerConfig("prefill_e32", T=2048, D=4096, E=32, K=8, f=1536)
+# the fine-grained layer's per-expert shape (~80 rows per expert, D=4096, f=f_s=1024, top-10,
+# shared expert) with 64 experts and 512 tokens: 1.6 GB of weights, for profiler captures
+CONFIGS["finegrained_e64"] = LayerConfig("finegrained_e64", T=512, D=4096, E=64, K=10, f=1024,
+                                         f_s=1024)
 ZIPF_TOKENS = (1, 16, 128, 1024, 16384)
 for _t in ZIPF_TOKENS:
     CONFIGS[f"zipf@T{_t}"] = LayerConfig(f"zipf@T{_t}", T=_t, D=4096, E=128, K=8, f=1536,
