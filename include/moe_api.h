@@ -30,6 +30,9 @@
  *     T >= 0 and T*K < 2^31.  Others return MOE_ERR_UNSUPPORTED.
  *   - Calls that share a workspace must not overlap on the GPU (same stream, or
  *     ordered by events).
+ *   - The library keeps per-process host caches (TMA tensor maps by base address and
+ *     shape, the kernels' shared-memory limits per device) so that a call does little host
+ *     work; calls after a cudaDeviceReset are not supported.
  */
 #ifndef MOE_API_H
 #define MOE_API_H

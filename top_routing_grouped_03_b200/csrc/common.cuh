@@ -67,6 +67,12 @@ void count_launches(unsigned n);
 // Bound, in nanoseconds, of the layer's grid-wide wait (moe_set_grid_wait_budget_ns).
 unsigned long long grid_wait_budget_ns();
 
+// Lets kernel `fn` use `bytes` of dynamic shared memory on the current device: calls
+// cudaFuncSetAttribute only when the limit this process last set there for fn is smaller
+// (the attribute is per device and function; the layer would otherwise set it on every
+// launch).
+cudaError_t set_smem_limit(const void* fn, size_t bytes);
+
 // ---------------------------------------------------------------- kernel launchers
 // (defined in the .cu files, called by the C entry points in moe_api.cu)
 

@@ -101,9 +101,7 @@ cudaError_t launch_ep_recv_layout(const int32_t* recv_counts, int G, int El, int
                                   int32_t* recv_offsets, int32_t* recv_row, int* status,
                                   cudaStream_t s) {
     const size_t smem = ep_recv_layout_smem(G, El);
-    cudaError_t err = cudaFuncSetAttribute(ep_recv_layout_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
+    cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(ep_recv_layout_kernel), smem);
     if (err != cudaSuccess) return err;
     err = launch_kernel(ep_recv_layout_kernel, dim3(1), dim3(kLayoutThreads), smem, s, false,
                         recv_counts, G, El, n, recv_offsets, recv_row, status);

@@ -35,6 +35,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <unordered_map>
 
 #include "common.cuh"
 #include "ptx.cuh"
@@ -1199,7 +1200,8 @@ cudaError_t get_encoder() {
 }
 
 // 2-D bf16 view [rows, cols] (cols contiguous), box [box_rows, 64], 128-byte swizzle.
-cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, int box_rows) {
+cudaError_t encode_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                       int box_rows) {
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};
     cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
@@ -1211,6 +1213,45 @@ cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// encode_map through a per-process cache keyed by (base, rows, cols, box): a descriptor
+// depends on nothing else, and a layer call would otherwise encode 4 to 8 of them on the
+// host.  The cache is bounded (cleared when full).
+cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, int box_rows) {
+    struct Key {
+        const void* base;
+        uint64_t rows, cols;
+        int box;
+        bool operator==(const Key& o) const {
+            return base == o.base && rows == o.rows && cols == o.cols && box == o.box;
+        }
+    };
+    struct Hash {
+        size_t operator()(const Key& k) const {
+            size_t h = std::hash<const void*>()(k.base);
+            h = h * 1000003u ^ std::hash<uint64_t>()(k.rows);
+            h = h * 1000003u ^ std::hash<uint64_t>()(k.cols);
+            return h * 1000003u ^ static_cast<size_t>(k.box);
+        }
+    };
+    static std::mutex mu;
+    static std::unordered_map<Key, CUtensorMap, Hash> cache;
+    const Key key{base, rows, cols, box_rows};
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = cache.find(key);
+        if (it != cache.end()) {
+            *m = it->second;
+            return cudaSuccess;
+        }
+    }
+    const cudaError_t err = encode_map(m, base, rows, cols, box_rows);
+    if (err != cudaSuccess) return err;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache.size() >= 4096) cache.clear();
+    cache.emplace(key, *m);
+    return cudaSuccess;
+}
+
 template <int BN, bool GATE_UP>
 cudaError_t launch_tpl(const CUtensorMap& mw, const CUtensorMap& ma, const Params& p, int grid,
                        cudaStream_t s, bool pdl) {
@@ -1219,8 +1260,7 @@ cudaError_t launch_tpl(const CUtensorMap& mw, const CUtensorMap& ma, const Param
                         (2 * C::kStages + 5) * 8 + 16 +
                         2 * (p.G + 1) * sizeof(int);
     auto kfn = grouped_gemm_kernel<BN, GATE_UP>;
-    cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
+    cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(kfn), smem);
     if (err != cudaSuccess) return err;
     err = launch_kernel(kfn, dim3(grid), dim3(kThreads), smem, s, pdl, mw, ma, p);
     count_launches(1);
@@ -1235,8 +1275,7 @@ cudaError_t launch_tm(const CUtensorMap& mw, const CUtensorMap& ma, const CUtens
                         (2 * C::kMaxStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int) +
                         (GATE_UP ? 0 : kEpiStageBytes);
     auto kfn = grouped_gemm_tm_kernel<GATE_UP>;
-    cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
+    cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(kfn), smem);
     if (err != cudaSuccess) return err;
     err = launch_kernel(kfn, dim3(grid), dim3(kTmThreads), smem, s, pdl, mw, ma, mw2, p);
     count_launches(1);
@@ -1251,8 +1290,7 @@ cudaError_t launch_pair(const CUtensorMap& mw, const CUtensorMap& ma, const Para
                         (2 * C::kStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int) +
                         (GATE_UP ? 0 : kEpiStageBytes);
     auto kfn = grouped_gemm_pair_kernel<GATE_UP>;
-    cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
+    cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(kfn), smem);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(2 * npairs);

@@ -5,6 +5,8 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
+#include <vector>
 
 #include "common.cuh"
 
@@ -12,6 +14,29 @@ namespace moe {
 
 std::atomic<unsigned long long> g_launches{0};
 void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+cudaError_t set_smem_limit(const void* fn, size_t bytes) {
+    struct Entry {
+        const void* fn;
+        int dev;
+        size_t bytes;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> set;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    Entry* e = nullptr;
+    for (Entry& x : set)
+        if (x.fn == fn && x.dev == dev) e = &x;
+    if (e != nullptr && e->bytes >= bytes) return cudaSuccess;
+    const cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(bytes));
+    if (err != cudaSuccess) return err;
+    if (e != nullptr) e->bytes = bytes;
+    else set.push_back(Entry{fn, dev, bytes});
+    return cudaSuccess;
+}
 
 constexpr unsigned long long kDefaultGridWaitNs = 2000000000ull;  // 2 s
 std::atomic<unsigned long long> g_grid_wait_ns{kDefaultGridWaitNs};

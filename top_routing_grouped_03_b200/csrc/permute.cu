@@ -102,8 +102,7 @@ cudaError_t launch_permute(const PermuteLaunch& a, cudaStream_t s, bool pdl) {
         if (err != cudaSuccess) return err;
     }
     const size_t smem = sizeof(int) * (static_cast<size_t>(kPermWarps) * a.E + 3 * a.E + 1);
-    err = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
+    err = set_smem_limit(reinterpret_cast<const void*>(permute_scatter_kernel), smem);
     if (err != cudaSuccess) return err;
     err = launch_kernel(permute_scatter_kernel, dim3(chunks), dim3(kPermThreads), smem, s,
                         pdl || chunks > 1, a, chunk_len, chunks);

@@ -172,6 +172,22 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
         for (int i = b + tid; i < e; i += kRouterThreads) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 
+    // ---- bring this warp's first expert rows toward L2 while the token rows are staged
+    //      (the two DRAM round trips overlap instead of following each other)
+    {
+        const int e_first = blockIdx.y * experts_per_cta + warp * kExpertsPerWarp;
+        const int e_stop = min(blockIdx.y * experts_per_cta + experts_per_cta, rows_total);
+#pragma unroll
+        for (int u = 0; u < kExpertsPerWarp; ++u) {
+            const int e = e_first + u;
+            if (e >= e_stop) break;
+            const char* row = reinterpret_cast<const char*>(
+                (e < E) ? a.w_router + static_cast<size_t>(e) * D : a.w_shared_gate);
+            for (int l = lane; l < D * 2 / 128; l += 32)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(row + l * 128));
+        }
+    }
+
     // ---- stage the 8 token rows (zeros past T)
     const int vec_per_row = D / 8;
     const uint4* xsrc = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0) * D);
@@ -373,8 +389,7 @@ cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bo
         smem = std::max(smem, sizeof(int) * (static_cast<size_t>(kRouterThreads / 32) * a.E +
                                              3 * a.E + 1));
     }
-    cudaError_t err = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
+    cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(router_kernel), smem);
     if (err != cudaSuccess) return err;
     err = launch_kernel(router_kernel, dim3(n_tb, n_eb), dim3(kRouterThreads), smem, s, pdl, a,
                         per_cta);
