@@ -185,8 +185,10 @@ def test_layer_plan_names_the_launched_steps(lib):
     # a shared expert of another width keeps its two launches
     assert _plan(lib, 4096, 4096, 512, 10, 1024, 512) == (
         {"router", "permute", "gate_up", "down", "shared"}, 8)
-    # prefill: CTA pairs, whose gate_up first copies the token rows into expert order
-    assert _plan(lib, 8192, 4096, 128, 8, 1536) == ({"router", "permute", "gate_up", "down"}, 7)
+    # prefill: CTA pairs, whose gate_up first copies the token rows into expert order and
+    # whose down writes weighted bf16 rows that a fixed-order combine sums
+    assert _plan(lib, 8192, 4096, 128, 8, 1536) == (
+        {"router", "permute", "gate_up", "down", "combine"}, 8)
     # E > 256 with few tokens: the permutation is a launch of its own
     assert _plan(lib, 70, 256, 512, 16, 128) == ({"router", "permute", "gate_up", "down"}, 4)
     assert _plan(lib, 0, 256, 16, 4, 128) == (set(), 0)

@@ -62,6 +62,14 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineLaunch a) {
                 acc[7] = fmaf(w, hi.w, acc[7]);
             }
         }
+        if (a.y16_sorted) {
+            const uint4* ys = reinterpret_cast<const uint4*>(a.y16_sorted);
+            for (int k = 0; k < a.K; ++k) {
+                const int row = __ldg(a.slot_to_row + t * a.K + k);
+                if (row < 0) continue;  // dropped past its expert's capacity
+                add8(acc, __ldcs(ys + static_cast<size_t>(row) * vec + c), 1.f);
+            }
+        }
         if (a.shared_out) {
             const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.shared_out) + i);
             add8(acc, v, __ldg(a.shared_gate + t));

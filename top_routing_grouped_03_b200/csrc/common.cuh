@@ -150,6 +150,7 @@ struct GroupedGemmLaunch {
     bf16* h_out;                // gate_up: [rows, f]
     float* acc_out;             // down: [T, D] scatter-add target or NULL
     float* y_out;               // down: [rows, D] fp32 or NULL
+    bf16* y16_out;              // down: [rows, D] bf16 (w * v per sorted row) or NULL
     int* status;
     // gate_up only: when gather_tok != NULL, act is the token matrix x [T, D] and row r of
     // the expert-ordered problem is x[gather_tok[r]] (gathered inside the kernel)
@@ -187,6 +188,8 @@ struct GroupedGemmLaunch {
 // true when launch_grouped_gemm would run `a` on the one-CTA tokens-on-M kernel (the one
 // that can carry an extra dense group)
 bool grouped_gemm_takes_extra_group(const GroupedGemmLaunch& a, int num_sms);
+// true when launch_grouped_gemm would run `a` on CTA pairs
+bool grouped_gemm_uses_pairs(const GroupedGemmLaunch& a, int num_sms);
 // kernels launch_grouped_gemm launches for `a` (0 when it has nothing to do)
 int grouped_gemm_launches(const GroupedGemmLaunch& a, int num_sms);
 cudaError_t launch_gather_rows(const bf16* x, const int32_t* tok, int rows, int D, bf16* out,
@@ -206,6 +209,7 @@ struct CombineLaunch {
     const bf16* residual;  // [T, D] added before the bf16 rounding, or NULL
     const float* out_acc;
     const float* y_sorted;
+    const bf16* y16_sorted;  // [T*K, D] bf16 rows already weighted (instead of y_sorted), or NULL
     const int32_t* slot_to_row;
     const float* topk_w;
     const bf16* shared_out;

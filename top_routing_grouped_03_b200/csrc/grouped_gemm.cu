@@ -84,6 +84,7 @@ struct Params {
     bf16* h_out;
     float* acc_out;
     float* y_out;
+    bf16* y16_out;     // down: w * v per sorted row as bf16 [rows, out_cols], or NULL
     int* status;
     const int32_t* gather_tok;  // gate_up: B rows are x[gather_tok[row]] (cp.async), or NULL
     const bf16* x;              // the token matrix the gather reads, [*, K] bf16
@@ -268,18 +269,19 @@ struct RowGather {
         }
     }
 
-    // copies columns [k0, k0 + 64) of the planned rows into the tile at smem_tile (rows
-    // past the group are zero-filled)
+    // copies columns [k0, k0 + 64) of the planned rows into the tile at smem_tile.  Rows
+    // past the group are not written at all: the MMA row they feed is independent of the
+    // others and the epilogue never reads it back, so whatever the stage held stays there
+    // (a group of 2 rows costs one copy instruction per stage, not ROWS / 4).
     __device__ __forceinline__ void issue(uint32_t smem_tile, const bf16* x, int k0,
                                           int lane) const {
         const int c = lane & 7;
 #pragma unroll
         for (int u = 0; u < kChunks; ++u) {
-            // branch-free: rows past the group get a zero fill (no global read)
+            if (__ballot_sync(0xffffffffu, (valid >> u) & 1u) == 0) break;  // rows ascend
             const int r = (lane >> 3) + 4 * u;
-            const bool live = (valid >> u) & 1u;
-            cp_async_16(smem_tile + r * 128 + ((c ^ (r & 7)) << 4), x + src_off[u] + k0,
-                        live ? 16u : 0u);
+            if ((valid >> u) & 1u)
+                cp_async_16(smem_tile + r * 128 + ((c ^ (r & 7)) << 4), x + src_off[u] + k0, 16u);
         }
     }
 };
@@ -525,8 +527,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
 // spread the same weight bytes over more of the grid (and, being smaller, let more
 // pipeline stages fit in shared memory).  The CTA-pair kernel always uses wn = 256.
 constexpr int kTmRows = 128;  // token rows per tile (MMA M)
+// weights on M while no group can exceed this many rows (a handful of tokens): measured
+// faster than tokens on M there (one token: 47 vs 50 us for gate_up at the Zipf T=1 shape)
+constexpr int kSwapMaxRows = 16;
 constexpr int kTmN = 256;     // widest weight tile (MMA N)
-constexpr int kWBox = 32;     // weight rows per TMA box of the one-CTA kernel
+// Weight tensor maps of the one-CTA kernel: one per box height (128, 64, 32 rows), so that a
+// stage of any tile width takes at most two weight loads (many small boxes per stage cut the
+// rate at which one SM streams weights); index by box_index().
+constexpr int kNumBoxes = 3;
+__host__ __device__ constexpr int box_rows_of(int i) { return 128 >> i; }
+__device__ __forceinline__ int box_index(int rows) { return rows >= 128 ? 0 : (rows >= 64 ? 1 : 2); }
+
+struct TmMaps {
+    CUtensorMap w[kNumBoxes];   // routed experts' weights
+    CUtensorMap w2[kNumBoxes];  // the extra dense group's weights (copies of w without one)
+};
 // 2 warps (producer, MMA) + 8 epilogue warps: two warps per tensor-memory lane quarter,
 // each draining half of the accumulator's columns
 constexpr int kTmThreads = 64 + 256;
@@ -666,6 +681,23 @@ __device__ __forceinline__ void tm_epilogue(const Params& p, uint32_t tbase, int
             }
         }
 #pragma unroll 1
+        for (int c0 = 0; c0 < hc && p.y16_out; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(tcol + c0, v);
+            tmem_ld_wait();
+            if (valid) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    pk[j] = pack_bf16x2(w * __uint_as_float(v[2 * j]), w * __uint_as_float(v[2 * j + 1]));
+                uint4* dst = reinterpret_cast<uint4*>(
+                    p.y16_out + static_cast<size_t>(row) * p.out_cols + col0 + c0);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            }
+        }
+#pragma unroll 1
         for (int c0 = 0; c0 < hc && p.y_out; c0 += 32) {
             uint32_t v[32];
             tmem_ld32(tcol + c0, v);
@@ -720,7 +752,7 @@ __device__ __forceinline__ int tile_of_slot(int t, int n_r, int n_x) {
 
 // Per-tile fixed cost, in weight rows, of the width choice below (a tile's share of the
 // pipeline hand-offs and of the epilogue's fixed steps).
-constexpr int kTileCostRows = 16;
+constexpr int kTileCostRows = 128;
 
 // The group table of the one-CTA tokens-on-M kernel, and its tile width.  Warp 2 counts
 // the 128-row blocks of every group (row_blocks), picks the weight rows per tile
@@ -772,9 +804,8 @@ __device__ __forceinline__ void build_tile_table_tm(const Params& p, int* g_off,
 
 template <bool GATE_UP>
 __global__ void __launch_bounds__(kTmThreads, 1)
-grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
-                       const __grid_constant__ CUtensorMap map_act,
-                       const __grid_constant__ CUtensorMap map_w2, Params p) {
+grouped_gemm_tm_kernel(const __grid_constant__ TmMaps maps,
+                       const __grid_constant__ CUtensorMap map_act, Params p) {
     using C = CfgTm;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -809,8 +840,10 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&map_w);
-        if (p.xg) tma_prefetch_desc(&map_w2);
+        for (int i = 0; i < kNumBoxes; ++i) {
+            tma_prefetch_desc(&maps.w[i]);
+            if (p.xg) tma_prefetch_desc(&maps.w2[i]);
+        }
         if (!gather) tma_prefetch_desc(&map_act);
     }
     if (warp == 1) {
@@ -848,7 +881,9 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
                 const Tile t = decode_tile(tile_of_slot(slot, n_routed, n_extra), g_tile, g_off,
                                            p.G, kTmRows);
                 const bool ex = p.xg && t.g == p.G - 1;
-                const CUtensorMap* mw = ex ? &map_w2 : &map_w;
+                // one box per gate / up block (gate_up) or up to two 128-row boxes (down)
+                const int box = GATE_UP ? wn / 2 : (wn >= 128 ? 128 : wn);
+                const CUtensorMap* mw = ex ? &maps.w2[box_index(box)] : &maps.w[box_index(box)];
                 // gate_up: gate rows g*2f + i*wn/2 and up rows f further; down: g*D + i*wn
                 // (the extra group's weights are a matrix of their own: g = 0 there)
                 const int wr0 = (ex ? 0 : t.g * p.w_group_rows) + t.i * (GATE_UP ? wn / 2 : wn);
@@ -872,14 +907,14 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
                         uint8_t* bt = st + C::kABytes;
                         if (GATE_UP) {
                             const int F = wn / 2;
-                            for (int b = 0; b < F; b += kWBox) {
+                            for (int b = 0; b < F; b += box) {
                                 tma_load_2d(bt + b * kBK * 2, mw, &full[stage], kk * kBK,
                                             wr0 + b, pol_w);
                                 tma_load_2d(bt + (F + b) * kBK * 2, mw, &full[stage],
                                             kk * kBK, wr0 + p.up_rows + b, pol_w);
                             }
                         } else {
-                            for (int b = 0; b < wn; b += kWBox)
+                            for (int b = 0; b < wn; b += box)
                                 tma_load_2d(bt + b * kBK * 2, mw, &full[stage], kk * kBK,
                                             wr0 + b, pol_w);
                         }
@@ -1268,8 +1303,8 @@ cudaError_t launch_tpl(const CUtensorMap& mw, const CUtensorMap& ma, const Param
 }
 
 template <bool GATE_UP>
-cudaError_t launch_tm(const CUtensorMap& mw, const CUtensorMap& ma, const CUtensorMap& mw2,
-                      const Params& p, int grid, cudaStream_t s, bool pdl) {
+cudaError_t launch_tm(const TmMaps& maps, const CUtensorMap& ma, const Params& p, int grid,
+                      cudaStream_t s, bool pdl) {
     using C = CfgTm;
     const size_t smem = 1024 + static_cast<size_t>(C::kRingBytes) +
                         (2 * C::kMaxStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int) +
@@ -1277,7 +1312,7 @@ cudaError_t launch_tm(const CUtensorMap& mw, const CUtensorMap& ma, const CUtens
     auto kfn = grouped_gemm_tm_kernel<GATE_UP>;
     cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(kfn), smem);
     if (err != cudaSuccess) return err;
-    err = launch_kernel(kfn, dim3(grid), dim3(kTmThreads), smem, s, pdl, mw, ma, mw2, p);
+    err = launch_kernel(kfn, dim3(grid), dim3(kTmThreads), smem, s, pdl, maps, ma, p);
     count_launches(1);
     return err;
 }
@@ -1334,16 +1369,23 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
     const uint64_t w_group_rows = a.gate_up ? 2ull * a.f : static_cast<uint64_t>(a.D);
     CUtensorMap mw, ma;
     cudaError_t err;
-    // weight boxes: 32 rows for the one-CTA tokens-on-M kernel (its tile width is chosen on
-    // the device), 128 rows otherwise
-    if ((err = make_map(&mw, a.w, w_group_rows * a.E, K, kind == Kind::kTm ? kWBox : kBM)) !=
-        cudaSuccess)
-        return err;
-    // the extra dense group's weights (one CTA tokens-on-M only), else a copy of mw
-    CUtensorMap mw2 = mw;
-    if (a.xg_w != nullptr &&
-        (err = make_map(&mw2, a.xg_w, w_group_rows, K, kWBox)) != cudaSuccess)
-        return err;
+    // weight boxes of 128 rows; the one-CTA tokens-on-M kernel (tile width chosen on the
+    // device) gets maps with 128-, 64- and 32-row boxes, for the routed experts and for the
+    // extra dense group (copies of the routed ones when there is none)
+    if ((err = make_map(&mw, a.w, w_group_rows * a.E, K, kBM)) != cudaSuccess) return err;
+    TmMaps tmaps;
+    if (kind == Kind::kTm) {
+        for (int i = 0; i < kNumBoxes; ++i) {
+            if ((err = make_map(&tmaps.w[i], a.w, w_group_rows * a.E, K, box_rows_of(i))) !=
+                cudaSuccess)
+                return err;
+            tmaps.w2[i] = tmaps.w[i];
+            if (a.xg_w != nullptr &&
+                (err = make_map(&tmaps.w2[i], a.xg_w, w_group_rows, K, box_rows_of(i))) !=
+                    cudaSuccess)
+                return err;
+        }
+    }
     // the activation map is only read when the rows are contiguous (no gather); with a
     // gather it still has to be a valid descriptor, so it covers the first row of x
     const void* act = a.act;
@@ -1373,6 +1415,7 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
     p.h_out = a.h_out;
     p.acc_out = a.acc_out;
     p.y_out = a.y_out;
+    p.y16_out = a.gate_up ? nullptr : a.y16_out;
     p.status = a.status;
     p.gather_tok = gather ? a.gather_tok : nullptr;
     p.x = reinterpret_cast<const bf16*>(act);
@@ -1403,8 +1446,8 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
                          : launch_pair<false>(mw, ma, p, npairs, s, true);
     }
     const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
-    if (tm) return a.gate_up ? launch_tm<true>(mw, ma, mw2, p, grid, s, pdl)
-                             : launch_tm<false>(mw, ma, mw2, p, grid, s, pdl);
+    if (tm) return a.gate_up ? launch_tm<true>(tmaps, ma, p, grid, s, pdl)
+                             : launch_tm<false>(tmaps, ma, p, grid, s, pdl);
     switch (BN) {
         case 16: return a.gate_up ? launch_tpl<16, true>(mw, ma, p, grid, s, pdl) : launch_tpl<16, false>(mw, ma, p, grid, s, pdl);
         case 32: return a.gate_up ? launch_tpl<32, true>(mw, ma, p, grid, s, pdl) : launch_tpl<32, false>(mw, ma, p, grid, s, pdl);
@@ -1451,7 +1494,7 @@ bool pick_kind(const GroupedGemmLaunch& a, int num_sms, Kind* kind, int* BN) {
     else if (a.orientation == 3 || routed_rows / a.E >= 128)
         *kind = pair_ok ? Kind::kPair : Kind::kTm;
     else
-        *kind = Kind::kTm;
+        *kind = max_rows <= kSwapMaxRows ? Kind::kSwap : Kind::kTm;
     return true;
 }
 
@@ -1462,6 +1505,12 @@ int grouped_gemm_launches(const GroupedGemmLaunch& a, int num_sms) {
     int BN;
     if (a.rows == 0 || a.E == 0 || !pick_kind(a, num_sms, &kind, &BN)) return 0;
     return (kind == Kind::kPair && a.gate_up && a.gather_tok != nullptr) ? 2 : 1;
+}
+
+bool grouped_gemm_uses_pairs(const GroupedGemmLaunch& a, int num_sms) {
+    Kind kind;
+    int BN;
+    return pick_kind(a, num_sms, &kind, &BN) && kind == Kind::kPair;
 }
 
 bool grouped_gemm_takes_extra_group(const GroupedGemmLaunch& a, int num_sms) {

@@ -154,6 +154,8 @@ struct LayerPlan {
     GroupedGemmLaunch up, dn, su, sd;
     CombineLaunch c;
     bool tc_router, det, fuse_shared, shared_launches;
+    bool rows_mode;  // down on CTA pairs writes weighted bf16 rows; the combine sums them
+    bool combine;    // a combine launch ends the call
 };
 
 LayerPlan plan_layer(const moe_layer_params* p, moe_bf16* out, void* workspace, int sms) {
@@ -175,7 +177,19 @@ LayerPlan plan_layer(const moe_layer_params* p, moe_bf16* out, void* workspace, 
     float* tw = p->topk_w_out ? p->topk_w_out : at<float>(workspace, L.topk_w);
     float* sgate = at<float>(workspace, L.sgate);
     float* out_acc = at<float>(workspace, L.out_acc);
-    const bool use_acc = !q.det || shared;
+    const int rows = T * K;
+    // When the down projection runs on CTA pairs (many rows per expert: the layer is
+    // tensor-bound), its epilogue writes each row's weighted output as bf16 with plain
+    // stores (into the expert-ordered x copy, free by then) and a fixed-order combine sums a
+    // token's K rows: fp32 reductions of T*K*D values into a [T, D] accumulator larger than
+    // L2 would keep the tensor pipe waiting.
+    GroupedGemmLaunch probe{};
+    probe.gate_up = false;
+    probe.rows = rows; probe.E = E; probe.D = D; probe.f = f;
+    q.rows_mode = !q.det && grouped_gemm_uses_pairs(probe, sms);
+    q.combine = q.det || q.rows_mode;
+    // the fp32 accumulator: every routed row's reductions, or only the shared expert's
+    const bool use_acc = shared || (!q.det && !q.rows_mode);
 
     PermuteLaunch& pm = q.pm;
     pm.topk_idx = idx;
@@ -218,7 +232,6 @@ LayerPlan plan_layer(const moe_layer_params* p, moe_bf16* out, void* workspace, 
         r.perm = pm;
     }
 
-    const int rows = T * K;
     GroupedGemmLaunch& up = q.up;
     up.gate_up = true;
     up.w = p->w_gate_up;
@@ -253,8 +266,9 @@ LayerPlan plan_layer(const moe_layer_params* p, moe_bf16* out, void* workspace, 
     dn.sorted_w = q.det ? nullptr : pm.sorted_w;
     dn.rows = rows; dn.E = E; dn.D = D; dn.f = f;
     dn.max_group_rows = up.max_group_rows;
-    dn.acc_out = q.det ? nullptr : out_acc;
+    dn.acc_out = q.det || q.rows_mode ? nullptr : out_acc;
     dn.y_out = q.det ? at<float>(workspace, L.y_sorted) : nullptr;
+    dn.y16_out = q.rows_mode ? at<bf16>(workspace, L.x_sorted) : nullptr;
     dn.status = status;
     if (q.fuse_shared) {
         dn.xg_w = p->w_shared_down;
@@ -267,7 +281,7 @@ LayerPlan plan_layer(const moe_layer_params* p, moe_bf16* out, void* workspace, 
     unsigned* done = at<unsigned>(workspace, L.status + 64);  // inside the cleared header
     const bf16* residual = reinterpret_cast<const bf16*>(p->residual);
     GroupedGemmLaunch& last = q.shared_launches ? q.sd : dn;
-    if (!q.det) {
+    if (!q.combine) {
         last.final_out = reinterpret_cast<bf16*>(out);
         last.final_rows = T;
         last.done = done;
@@ -299,6 +313,7 @@ LayerPlan plan_layer(const moe_layer_params* p, moe_bf16* out, void* workspace, 
     c.residual = residual;
     c.out_acc = use_acc ? out_acc : nullptr;
     c.y_sorted = q.det ? at<float>(workspace, L.y_sorted) : nullptr;
+    c.y16_sorted = q.rows_mode ? at<bf16>(workspace, L.x_sorted) : nullptr;
     c.slot_to_row = pm.slot_to_row;
     c.topk_w = q.det ? tw : nullptr;
     c.T = T; c.D = D; c.K = K;
@@ -537,7 +552,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
          launch_grouped_gemm(q.sd, sms, s, true) != cudaSuccess))
         return MOE_ERR_CUDA;
     if (!mark(MOE_EV_COMBINE)) return MOE_ERR_CUDA;
-    if (q.det && launch_combine(q.c, sms, s, true) != cudaSuccess) return MOE_ERR_CUDA;
+    if (q.combine && launch_combine(q.c, sms, s, true) != cudaSuccess) return MOE_ERR_CUDA;
     return mark(MOE_EV_END) ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -554,7 +569,7 @@ int moe_layer_plan(const moe_layer_params* p, unsigned* step_mask, int* launches
         const int np = q.r.fuse_perm ? 0 : (permute_chunks(static_cast<long long>(p->T) * p->K) > 1 ? 2 : 1);
         const int nu = grouped_gemm_launches(q.up, sms), nd = grouped_gemm_launches(q.dn, sms);
         const int ns = q.shared_launches ? grouped_gemm_launches(q.su, sms) + grouped_gemm_launches(q.sd, sms) : 0;
-        const int nc = q.det ? 1 : 0;
+        const int nc = q.combine ? 1 : 0;
         const int per[] = {nr, np, nu, nd, ns, nc};
         for (int i = 0; i < 6; ++i) {
             if (per[i]) mask |= 1u << (MOE_EV_ROUTER + i);
