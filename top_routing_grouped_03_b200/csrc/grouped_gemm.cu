@@ -103,6 +103,8 @@ struct Params {
     long long zero_n4;
     // one-CTA tokens-on-M kernel: choose the tile width on the device (else 256 rows)
     int tm_adaptive;
+    // weights-on-M kernel with contiguous token rows: rows per activation TMA box (= BN)
+    int act_box;
     // one-CTA tokens-on-M kernel: group G-1 is an extra dense group (the shared expert):
     // its xg_rows rows follow the routed ones, [offsets[G-1], offsets[G-1] + xg_rows), row
     // r is token r - offsets[G-1], its weights come from the second weight map, and (down)
@@ -269,19 +271,18 @@ struct RowGather {
         }
     }
 
-    // copies columns [k0, k0 + 64) of the planned rows into the tile at smem_tile.  Rows
-    // past the group are not written at all: the MMA row they feed is independent of the
-    // others and the epilogue never reads it back, so whatever the stage held stays there
-    // (a group of 2 rows costs one copy instruction per stage, not ROWS / 4).
+    // copies columns [k0, k0 + 64) of the planned rows into the tile at smem_tile (rows
+    // past the group are zero-filled)
     __device__ __forceinline__ void issue(uint32_t smem_tile, const bf16* x, int k0,
                                           int lane) const {
         const int c = lane & 7;
 #pragma unroll
         for (int u = 0; u < kChunks; ++u) {
-            if (__ballot_sync(0xffffffffu, (valid >> u) & 1u) == 0) break;  // rows ascend
+            // branch-free: rows past the group get a zero fill (no global read)
             const int r = (lane >> 3) + 4 * u;
-            if ((valid >> u) & 1u)
-                cp_async_16(smem_tile + r * 128 + ((c ^ (r & 7)) << 4), x + src_off[u] + k0, 16u);
+            const bool live = (valid >> u) & 1u;
+            cp_async_16(smem_tile + r * 128 + ((c ^ (r & 7)) << 4), x + src_off[u] + k0,
+                        live ? 16u : 0u);
         }
     }
 };
@@ -381,8 +382,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                         if (GATE_UP)
                             tma_load_2d(st + C::kABytes, &map_w, &full[stage], kk * kBK,
                                         wr0 + p.up_rows, pol_w);
-                        if (!gather)
-                            for (int b = 0; b < BN; b += 16)
+                        if (!gather)  // act_box rows per box: one box per stage
+                            for (int b = 0; b < BN; b += p.act_box)
                                 tma_load_2d(st + a_bytes + b * kBK * 2, &map_act, &full[stage],
                                             kk * kBK, t.row0 + b, pol_a);
                     }
@@ -1397,8 +1398,8 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
         act = a.gather_buf;
         gather = false;
     }
-    // activation boxes: 128 rows (tokens on M) or 16 rows (weights on M, bn/16 per stage)
-    if ((err = make_map(&ma, act, gather ? 1 : a.rows, K, gather ? 1 : (tm ? kTmRows : 16))) !=
+    // activation boxes: 128 rows (tokens on M) or BN rows (weights on M: one box per stage)
+    if ((err = make_map(&ma, act, gather ? 1 : a.rows, K, gather ? 1 : (tm ? kTmRows : BN))) !=
         cudaSuccess)
         return err;
     Params p{};
@@ -1428,6 +1429,7 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
     p.zero_acc = a.gate_up ? a.zero_acc : nullptr;
     p.zero_n4 = a.zero_floats / 4;
     p.tm_adaptive = kind == Kind::kTm ? 1 : 0;
+    p.act_box = BN;
     if (a.xg_w != nullptr) {
         p.xg = 1;
         p.G = a.E + 1;
@@ -1452,7 +1454,9 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
         case 16: return a.gate_up ? launch_tpl<16, true>(mw, ma, p, grid, s, pdl) : launch_tpl<16, false>(mw, ma, p, grid, s, pdl);
         case 32: return a.gate_up ? launch_tpl<32, true>(mw, ma, p, grid, s, pdl) : launch_tpl<32, false>(mw, ma, p, grid, s, pdl);
         case 64: return a.gate_up ? launch_tpl<64, true>(mw, ma, p, grid, s, pdl) : launch_tpl<64, false>(mw, ma, p, grid, s, pdl);
-        default: return a.gate_up ? launch_tpl<128, true>(mw, ma, p, grid, s, pdl) : launch_tpl<128, false>(mw, ma, p, grid, s, pdl);
+        case 128: return a.gate_up ? launch_tpl<128, true>(mw, ma, p, grid, s, pdl) : launch_tpl<128, false>(mw, ma, p, grid, s, pdl);
+        // 256 token rows: down only (gate_up's two accumulators would not fit tensor memory)
+        default: return a.gate_up ? cudaErrorInvalidValue : launch_tpl<256, false>(mw, ma, p, grid, s, pdl);
     }
 }
 
@@ -1473,7 +1477,8 @@ bool pick_kind(const GroupedGemmLaunch& a, int num_sms, Kind* kind, int* BN) {
     const long long avg8 = 8ll * routed_rows / a.E;
     const int bn_rows = static_cast<int>(std::min<long long>(max_rows, std::max(avg8, 16ll)));
     *BN = a.block_rows ? a.block_rows : pick_block_rows(bn_rows, 1);
-    if (*BN != 16 && *BN != 32 && *BN != 64 && *BN != 128) return false;
+    if (*BN != 16 && *BN != 32 && *BN != 64 && *BN != 128 && !(*BN == 256 && !a.gate_up))
+        return false;
     if (a.ksplit > 1 && (a.gate_up || !a.y_out || a.acc_out || a.final_out ||
                          (a.f / kBK) % a.ksplit != 0))
         return false;

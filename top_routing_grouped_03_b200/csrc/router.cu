@@ -409,20 +409,23 @@ int router_tc_max_planes(int T) { return std::min(16, std::max(1, 512 / ceil_div
 
 cudaError_t launch_router_tc(const RouterLaunch& a, int num_sms, cudaStream_t s, bool pdl) {
     if (a.T == 0) return cudaSuccess;
-    // logits = x W_r^T: W_r's E rows on the MMA's M side, 128 tokens on N, one dense group.
-    // Few tiles with a long reduction (D) would leave most SMs idle, so the D steps are cut
-    // into S slices (partial planes).  S minimises waves x (steps per slice + a tile's fixed
-    // cost, about 8 steps of 64: pipeline fill, drain and epilogue), ties to fewer planes,
-    // with at least 4 steps per slice.
-    constexpr int kTileCostSteps = 8;
+    // logits = x W_r^T: W_r's E rows on the MMA's M side, BN = 128 or 256 tokens on N, one
+    // dense group.  Few tiles with a long reduction (D) would leave most SMs idle, so the D
+    // steps are cut into S slices (partial planes).  (BN, S) minimises the bytes the busiest
+    // CTA loads -- waves x (steps per slice x (128 + BN) rows of 128 B + a tile's fixed cost,
+    // about 2048 such rows: pipeline fill, drain and epilogue) -- ties to fewer planes and the
+    // narrower tile, with at least 4 steps per slice.  Wider token tiles re-read W_r less.
+    constexpr long long kTileCost = 2048;
     const int nk = a.D / 64;
-    const int base = (a.E / 128) * ceil_div(a.T, 128);
-    int S = 1;
-    long long best = static_cast<long long>(ceil_div(base, num_sms)) * (nk + kTileCostSteps);
-    for (int c = 2; c <= router_tc_max_planes(a.T) && nk % c == 0 && nk / c >= 4; c *= 2) {
-        const long long cost =
-            static_cast<long long>(ceil_div(base * c, num_sms)) * (nk / c + kTileCostSteps);
-        if (cost < best) { best = cost; S = c; }
+    int S = 1, BN = 128;
+    long long best = -1;
+    for (int bn = 128; bn <= 256; bn *= 2) {
+        const int base = (a.E / 128) * ceil_div(a.T, bn);
+        for (int c = 1; c <= router_tc_max_planes(a.T) && nk % c == 0 && nk / c >= 4; c *= 2) {
+            const long long cost = static_cast<long long>(ceil_div(base * c, num_sms)) *
+                                   (static_cast<long long>(nk / c) * (128 + bn) + kTileCost);
+            if (best < 0 || cost < best) { best = cost; S = c; BN = bn; }
+        }
     }
     GroupedGemmLaunch g{};
     g.gate_up = false;
@@ -435,7 +438,7 @@ cudaError_t launch_router_tc(const RouterLaunch& a, int num_sms, cudaStream_t s,
     g.f = a.D;  // reduction length
     g.y_out = a.logits;
     g.status = a.status;
-    g.block_rows = 128;
+    g.block_rows = BN;
     g.ksplit = S;
     cudaError_t err = launch_grouped_gemm(g, num_sms, s, pdl);
     if (err != cudaSuccess) return err;
