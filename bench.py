@@ -542,6 +542,27 @@ def measure(b: Bench, moe, cfg, peaks, src, reps: int, cpu_budget: float, gpu_id
     return row
 
 
+def profile_calls(moe, cfg, dev, n: int, deterministic: bool) -> int:
+    """n eager calls of the layer (each launches the kernels moe_layer_plan lists, in that
+    order), then the plan on stdout: the launch sequence an ncu -s/-c selection counts on."""
+    import torch
+
+    import workloads
+    gen_dev = dev if big_layer(cfg) else "cpu"
+    inp = workloads.make_inputs(cfg, device=gen_dev).to(dev)
+    layer = moe.MoELayer.from_inputs(inp, deterministic=deterministic)
+    out = torch.empty((cfg.T, cfg.D), dtype=torch.bfloat16, device=dev)
+    for _ in range(n):
+        layer(inp.x, out=out)
+    torch.cuda.synchronize()
+    if layer.device_status() != 0:
+        raise RuntimeError("device status is not ok")
+    steps, launches = layer.plan(cfg.T)
+    print(json.dumps({"workload": describe(cfg), "calls": n, "steps": steps,
+                      "launches_per_call": launches}), flush=True)
+    return 0
+
+
 def dry_run(args, rank, world):
     """Launcher check without a GPU: every rank joins a gloo group, reports a synthetic
     per-rank time, and rank 0 prints the contract line built from the slowest rank."""
@@ -579,6 +600,10 @@ def main():
                          "profiler runs that flush caches themselves)")
     ap.add_argument("--dry-run", action="store_true",
                     help="check the multi-rank launch path on CPU (gloo), no GPU work")
+    ap.add_argument("--profile-calls", type=int, default=0,
+                    help="run this many eager layer calls of --config and exit, no timing "
+                         "(a fixed launch sequence for an external profiler; --deterministic "
+                         "applies)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -613,6 +638,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
+    if args.profile_calls > 0:
+        return profile_calls(moe, cfg, dev, args.profile_calls, args.deterministic)
     b = Bench(dev, args.flush_mib)
     w = Workload(moe, cfg, dev, deterministic=args.deterministic)
     stream = torch.cuda.current_stream()

@@ -70,6 +70,10 @@ CONFIGS["prefill_e32"] = LayerConfig("prefill_e32", T=2048, D=4096, E=32, K=8, f
 # shared expert) with 64 experts and 512 tokens: 1.6 GB of weights, for profiler captures
 CONFIGS["finegrained_e64"] = LayerConfig("finegrained_e64", T=512, D=4096, E=64, K=10, f=1024,
                                          f_s=1024)
+# the fine-grained layer's router (T=4096, D=4096, E=512, K=10, shared gate) with narrow
+# experts (f=f_s=128): the same router kernels on 1.6 GB of weights, for profiler captures
+CONFIGS["finegrained_router"] = LayerConfig("finegrained_router", T=4096, D=4096, E=512, K=10,
+                                            f=128, f_s=128)
 # one token on the prefill/Zipf expert shape (D=4096, f=1536, top-8) with 16 experts: the
 # few-token kernels on 0.6 GB of weights, for profiler captures
 CONFIGS["zipf_e16@T1"] = LayerConfig("zipf_e16@T1", T=1, D=4096, E=16, K=8, f=1536)
