@@ -101,8 +101,6 @@ struct Params {
     // accumulator) before their first tile -- they would otherwise wait for it idle
     float* zero_acc;
     long long zero_n4;
-    // one-CTA tokens-on-M kernel: choose the tile width on the device (else 256 rows)
-    int tm_adaptive;
     // weights-on-M kernel with contiguous token rows: rows per activation TMA box (= BN)
     int act_box;
     // one-CTA tokens-on-M kernel: group G-1 is an extra dense group (the shared expert):
@@ -518,31 +516,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
 
 // ---------------------------------------------------------------- tokens-on-M variant
 // For groups with more than a handful of rows: the MMA's M side holds 128 token rows and
-// its N side wn weight rows (gate_up: the gate and up rows of the same wn/2 features;
-// down: wn output features), one tcgen05.mma of 128 x wn x 16 per 16 of K.  Each
+// its N side 256 weight rows (gate_up: the gate and up rows of the same 128 features;
+// down: 256 output features), one tcgen05.mma of 128 x 256 x 16 per 16 of K.  Each
 // epilogue thread owns one row, so h is written with 16-byte stores and the down epilogue
-// reduces 16-byte vectors (red.global.add.v4.f32) into the token's output row.
-// The one-CTA kernel picks wn in {256, 128, 64} on the device, per launch, from the
-// groups' row counts: a few experts with many rows (concentrated routing) would otherwise
-// leave most SMs idle, each busy SM streaming its weight tiles alone; narrower tiles
-// spread the same weight bytes over more of the grid (and, being smaller, let more
-// pipeline stages fit in shared memory).  The CTA-pair kernel always uses wn = 256.
+// reduces 16-byte vectors (red.global.add.v4.f32) into the token's output row.  The
+// one-CTA kernel can carry one extra, dense group (the shared expert) whose weights come
+// from a second tensor map; the CTA-pair kernel shares the tile shape.
 constexpr int kTmRows = 128;  // token rows per tile (MMA M)
 // weights on M while no group can exceed this many rows (a handful of tokens): measured
 // faster than tokens on M there (one token: 47 vs 50 us for gate_up at the Zipf T=1 shape)
 constexpr int kSwapMaxRows = 16;
-constexpr int kTmN = 256;     // widest weight tile (MMA N)
-// Weight tensor maps of the one-CTA kernel: one per box height (128, 64, 32 rows), so that a
-// stage of any tile width takes at most two weight loads (many small boxes per stage cut the
-// rate at which one SM streams weights); index by box_index().
-constexpr int kNumBoxes = 3;
-__host__ __device__ constexpr int box_rows_of(int i) { return 128 >> i; }
-__device__ __forceinline__ int box_index(int rows) { return rows >= 128 ? 0 : (rows >= 64 ? 1 : 2); }
-
-struct TmMaps {
-    CUtensorMap w[kNumBoxes];   // routed experts' weights
-    CUtensorMap w2[kNumBoxes];  // the extra dense group's weights (copies of w without one)
-};
+constexpr int kTmN = 256;     // weight rows per tile (MMA N)
 // 2 warps (producer, MMA) + 8 epilogue warps: two warps per tensor-memory lane quarter,
 // each draining half of the accumulator's columns
 constexpr int kTmThreads = 64 + 256;
@@ -725,18 +709,15 @@ __device__ __forceinline__ float* epi_stage(int* table_end, int warp) {
     return reinterpret_cast<float*>(a) + (warp - 2) * kStageFloatsPerWarp;
 }
 
-// Shared-memory ring of the one-CTA kernel: 192 KB cut into stages of 128 token rows
-// (16 KB) + wn weight rows: 4 stages at wn = 256, 6 at 128, 8 at 64.
 struct CfgTm {
-    static constexpr int kABytes = kTmRows * kBK * 2;
-    static constexpr int kRingBytes = 192 * 1024;
-    static constexpr int kMaxStages = 8;
-    static constexpr int kTmemCols = 2 * kTmN;  // two accumulators of up to 256 columns
+    static constexpr int kABytes = kTmRows * kBK * 2;  // 16 KB of token rows
+    static constexpr int kBBytes = kTmN * kBK * 2;     // 32 KB of weight rows
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = 4;
+    static constexpr int kAccCols = kTmN;
+    static constexpr int kTmemCols = 2 * kAccCols;
+    static_assert(kTmemCols <= 512, "accumulators exceed tensor memory");
 };
-__device__ __forceinline__ int tm_stage_bytes(int wn) { return CfgTm::kABytes + wn * kBK * 2; }
-__device__ __forceinline__ int tm_num_stages(int wn) {
-    return min(CfgTm::kMaxStages, CfgTm::kRingBytes / tm_stage_bytes(wn));
-}
 
 // Processing order of the one-CTA kernel's tiles when an extra dense group is present:
 // its n_x tiles (table indices n_r .. n_r + n_x - 1, after the routed groups' n_r) take
@@ -751,19 +732,10 @@ __device__ __forceinline__ int tile_of_slot(int t, int n_r, int n_x) {
     return t - min(n_x, q);
 }
 
-// Per-tile fixed cost, in weight rows, of the width choice below (a tile's share of the
-// pipeline hand-offs and of the epilogue's fixed steps).
-constexpr int kTileCostRows = 128;
-
-// The group table of the one-CTA tokens-on-M kernel, and its tile width.  Warp 2 counts
-// the 128-row blocks of every group (row_blocks), picks the weight rows per tile
-//   wn = argmin over {256, 128, 64} of ceil(row_blocks * nf(wn) / gridDim.x) * (wn + c)
-// (nf(wn) = nf256 * 256 / wn feature blocks per row block; ties to the wider tile) --
-// the most weight rows any CTA streams, plus a per-tile cost -- and writes
-// g_tile[g] = (row blocks of the groups before g) * nf(wn).
+// The group table of the one-CTA tokens-on-M kernel: as build_tile_table, except that with
+// an extra dense group (p.xg) the last group's end is offsets[G-1] + xg_rows.
 __device__ __forceinline__ void build_tile_table_tm(const Params& p, int* g_off, int* g_tile,
-                                                    int* total_slot, int* wn_slot, int warp,
-                                                    int lane) {
+                                                    int* total_slot, int warp, int lane) {
     for (int i = threadIdx.x; i <= p.G; i += blockDim.x)
         g_off[i] = p.offsets ? (p.xg && i == p.G ? p.offsets[i - 1] + p.xg_rows : p.offsets[i])
                              : (i == 0 ? 0 : p.rows_total);
@@ -772,54 +744,42 @@ __device__ __forceinline__ void build_tile_table_tm(const Params& p, int* g_off,
         const int per = (p.G + 31) / 32;
         const int gb = min(lane * per, p.G), ge = min(gb + per, p.G);
         int local = 0;
-        for (int g = gb; g < ge; ++g) local += (g_off[g + 1] - g_off[g] + kTmRows - 1) / kTmRows;
+        for (int g = gb; g < ge; ++g) local += group_tiles(p, g_off[g + 1] - g_off[g], kTmRows);
         int incl = local;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int v = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += v;
         }
-        const long long rb = __shfl_sync(0xffffffffu, incl, 31);
-        int wn = kTmN;
-        if (p.tm_adaptive) {
-            long long best = -1;
-            for (int c = kTmN; c >= 64; c >>= 1) {
-                const long long tiles = rb * p.nf * (kTmN / c);
-                const long long cost = (tiles + gridDim.x - 1) / gridDim.x * (c + kTileCostRows);
-                if (best < 0 || cost < best) { best = cost; wn = c; }
-            }
-        }
-        const int nf = p.nf * (kTmN / wn);
         int run = incl - local;
         for (int g = gb; g < ge; ++g) {
-            g_tile[g] = run * nf;
-            run += (g_off[g + 1] - g_off[g] + kTmRows - 1) / kTmRows;
+            g_tile[g] = run;
+            run += group_tiles(p, g_off[g + 1] - g_off[g], kTmRows);
         }
         if (lane == 31) {
-            g_tile[p.G] = incl * nf;
-            *total_slot = incl * nf;
-            *wn_slot = wn;
+            g_tile[p.G] = incl;
+            *total_slot = incl;
         }
     }
 }
 
 template <bool GATE_UP>
 __global__ void __launch_bounds__(kTmThreads, 1)
-grouped_gemm_tm_kernel(const __grid_constant__ TmMaps maps,
-                       const __grid_constant__ CUtensorMap map_act, Params p) {
+grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
+                       const __grid_constant__ CUtensorMap map_act,
+                       const __grid_constant__ CUtensorMap map_w2, Params p) {
     using C = CfgTm;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kRingBytes);
-    uint64_t* empty = full + C::kMaxStages;
-    uint64_t* tfull = empty + C::kMaxStages;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+    uint64_t* empty = full + C::kStages;
+    uint64_t* tfull = empty + C::kStages;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* total_slot = reinterpret_cast<int*>(tmem_slot + 2);
-    int* wn_slot = reinterpret_cast<int*>(tmem_slot + 3);
     int* g_off = reinterpret_cast<int*>(tmem_slot + 4);
     int* g_tile = g_off + (p.G + 1);
 
@@ -828,7 +788,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ TmMaps maps,
     const bool gather = GATE_UP && p.gather_tok != nullptr;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kMaxStages; ++s) {
+        for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&full[s], gather ? 1 + 32 : 1);
             mbar_init(&empty[s], 1);
         }
@@ -841,10 +801,8 @@ grouped_gemm_tm_kernel(const __grid_constant__ TmMaps maps,
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        for (int i = 0; i < kNumBoxes; ++i) {
-            tma_prefetch_desc(&maps.w[i]);
-            if (p.xg) tma_prefetch_desc(&maps.w2[i]);
-        }
+        tma_prefetch_desc(&map_w);
+        if (p.xg) tma_prefetch_desc(&map_w2);
         if (!gather) tma_prefetch_desc(&map_act);
     }
     if (warp == 1) {
@@ -853,15 +811,12 @@ grouped_gemm_tm_kernel(const __grid_constant__ TmMaps maps,
     }
     grid_dep_wait();
     grid_dep_launch();
-    build_tile_table_tm(p, g_off, g_tile, total_slot, wn_slot, warp, lane);
+    build_tile_table_tm(p, g_off, g_tile, total_slot, warp, lane);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int total = *total_slot;
-    const int wn = *wn_slot;               // weight rows per tile
-    const int stage_bytes = tm_stage_bytes(wn);
-    const int nstages = tm_num_stages(wn);
     // tiles of the routed groups, and of the extra dense group (interleaved, tile_of_slot)
     const int n_routed = p.xg ? g_tile[p.G - 1] : total;
     const int n_extra = total - n_routed;
@@ -870,11 +825,10 @@ grouped_gemm_tm_kernel(const __grid_constant__ TmMaps maps,
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
         // token rows (A): one TMA box of 128 rows when contiguous, else the lanes gather
-        // them with cp.async; weight rows (B): wn rows in boxes of 32.
+        // them with cp.async; weight rows (B): two TMA boxes of 128 rows.
         if (gather || lane == 0) {
             const uint64_t pol_w = policy_evict_first();
             const uint64_t pol_a = policy_evict_last();
-            const uint32_t w_bytes = static_cast<uint32_t>(wn) * kBK * 2;
             int stage = 0;
             uint32_t phase = 0, filled = 0, fill_phase = 0;
             bool ok = true;
@@ -882,12 +836,12 @@ grouped_gemm_tm_kernel(const __grid_constant__ TmMaps maps,
                 const Tile t = decode_tile(tile_of_slot(slot, n_routed, n_extra), g_tile, g_off,
                                            p.G, kTmRows);
                 const bool ex = p.xg && t.g == p.G - 1;
-                // one box per gate / up block (gate_up) or up to two 128-row boxes (down)
-                const int box = GATE_UP ? wn / 2 : (wn >= 128 ? 128 : wn);
-                const CUtensorMap* mw = ex ? &maps.w2[box_index(box)] : &maps.w[box_index(box)];
-                // gate_up: gate rows g*2f + i*wn/2 and up rows f further; down: g*D + i*wn
-                // (the extra group's weights are a matrix of their own: g = 0 there)
-                const int wr0 = (ex ? 0 : t.g * p.w_group_rows) + t.i * (GATE_UP ? wn / 2 : wn);
+                const CUtensorMap* mw = ex ? &map_w2 : &map_w;
+                // gate_up: gate rows g*2f + i*128 and up rows g*2f + f + i*128; down: rows
+                // g*D + i*256 and the next 128 (the extra group's weights are a matrix of
+                // their own: g = 0 there)
+                const int wr0 = (ex ? 0 : t.g * p.w_group_rows) + t.i * (GATE_UP ? kBM : kTmN);
+                const int wr1 = GATE_UP ? wr0 + p.up_rows : wr0 + kBM;
                 RowGather<kTmRows> rg;
                 if (gather)
                     rg.plan(p.gather_tok, t.row0, t.row_end, p.nk * kBK, lane, ex ? x_base : -1);
@@ -900,25 +854,14 @@ grouped_gemm_tm_kernel(const __grid_constant__ TmMaps maps,
                         ok = false;
                         break;
                     }
-                    uint8_t* st = smem + stage * stage_bytes;
+                    uint8_t* st = smem + stage * C::kStageBytes;
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(&full[stage], gather ? w_bytes : stage_bytes);
+                        mbar_arrive_expect_tx(&full[stage], gather ? C::kBBytes : C::kStageBytes);
                         if (!gather)
                             tma_load_2d(st, &map_act, &full[stage], kk * kBK, t.row0, pol_a);
-                        uint8_t* bt = st + C::kABytes;
-                        if (GATE_UP) {
-                            const int F = wn / 2;
-                            for (int b = 0; b < F; b += box) {
-                                tma_load_2d(bt + b * kBK * 2, mw, &full[stage], kk * kBK,
-                                            wr0 + b, pol_w);
-                                tma_load_2d(bt + (F + b) * kBK * 2, mw, &full[stage],
-                                            kk * kBK, wr0 + p.up_rows + b, pol_w);
-                            }
-                        } else {
-                            for (int b = 0; b < wn; b += box)
-                                tma_load_2d(bt + b * kBK * 2, mw, &full[stage], kk * kBK,
-                                            wr0 + b, pol_w);
-                        }
+                        tma_load_2d(st + C::kABytes, mw, &full[stage], kk * kBK, wr0, pol_w);
+                        tma_load_2d(st + C::kABytes + kBM * kBK * 2, mw, &full[stage], kk * kBK,
+                                    wr1, pol_w);
                     }
                     if (gather) {
                         rg.issue(smem_u32(st), p.x, kk * kBK, lane);
@@ -926,12 +869,12 @@ grouped_gemm_tm_kernel(const __grid_constant__ TmMaps maps,
                     }
                     filled |= 1u << stage;
                     fill_phase = (fill_phase & ~(1u << stage)) | (phase << stage);
-                    if (++stage == nstages) { stage = 0; phase ^= 1u; }
+                    if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
                 }
             }
             if (gather) cp_async_wait_all();
             if (!ok && lane == 0) {
-                for (int s = 0; s < nstages; ++s)
+                for (int s = 0; s < C::kStages; ++s)
                     if (filled & (1u << s))
                         mbar_wait(&full[s], (fill_phase >> s) & 1u, kDrainBudgetNs, nullptr);
             }
@@ -940,7 +883,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ TmMaps maps,
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(kTmRows, wn);
+            constexpr uint32_t idesc = idesc_bf16_f32(kTmRows, kTmN);
             int stage = 0;
             uint32_t phase = 0, abuf = 0, aphase = 0;
             bool ok = true, issued = false;
@@ -952,7 +895,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ TmMaps maps,
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d0 = tmem_base + abuf * wn;
+                const uint32_t d0 = tmem_base + abuf * C::kAccCols;
                 for (int kk = 0; kk < p.nk; ++kk) {
                     if (!mbar_wait(&full[stage], phase, kWaitBudgetNs, abort_flag)) {
                         set_status(p.status, MOE_ERR_TIMEOUT);
@@ -962,7 +905,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ TmMaps maps,
                     }
                     tc_fence_after();
                     if (gather) fence_proxy_async_smem();
-                    const uint32_t a0 = smem_u32(smem + stage * stage_bytes);
+                    const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
                     const uint32_t b0 = a0 + C::kABytes;
 #pragma unroll
                     for (int s = 0; s < kBK / 16; ++s)
@@ -970,7 +913,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ TmMaps maps,
                                   (kk | s) != 0 ? 1u : 0u);
                     issued = true;
                     umma_commit(&empty[stage]);
-                    if (++stage == nstages) { stage = 0; phase ^= 1u; }
+                    if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
                 umma_commit(&tfull[abuf]);
@@ -999,10 +942,11 @@ grouped_gemm_tm_kernel(const __grid_constant__ TmMaps maps,
                 break;
             }
             tc_fence_after();
-            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + abuf * wn;
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   abuf * C::kAccCols;
             const int row = t.row0 + q * 32 + lane;
             tm_epilogue<GATE_UP>(p, tbase, row, row < t.row_end, t.i, (warp - 2) >> 2,
-                                 GATE_UP ? nullptr : epi_stage(g_tile + p.G + 1, warp), wn,
+                                 GATE_UP ? nullptr : epi_stage(g_tile + p.G + 1, warp), kTmN,
                                  ex ? x_base : -1);
             tc_fence_before();
             mbar_arrive(&tempty[abuf]);
@@ -1304,16 +1248,16 @@ cudaError_t launch_tpl(const CUtensorMap& mw, const CUtensorMap& ma, const Param
 }
 
 template <bool GATE_UP>
-cudaError_t launch_tm(const TmMaps& maps, const CUtensorMap& ma, const Params& p, int grid,
-                      cudaStream_t s, bool pdl) {
+cudaError_t launch_tm(const CUtensorMap& mw, const CUtensorMap& ma, const CUtensorMap& mw2,
+                      const Params& p, int grid, cudaStream_t s, bool pdl) {
     using C = CfgTm;
-    const size_t smem = 1024 + static_cast<size_t>(C::kRingBytes) +
-                        (2 * C::kMaxStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int) +
+    const size_t smem = 1024 + static_cast<size_t>(C::kStages) * C::kStageBytes +
+                        (2 * C::kStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int) +
                         (GATE_UP ? 0 : kEpiStageBytes);
     auto kfn = grouped_gemm_tm_kernel<GATE_UP>;
     cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(kfn), smem);
     if (err != cudaSuccess) return err;
-    err = launch_kernel(kfn, dim3(grid), dim3(kTmThreads), smem, s, pdl, maps, ma, p);
+    err = launch_kernel(kfn, dim3(grid), dim3(kTmThreads), smem, s, pdl, mw, ma, mw2, p);
     count_launches(1);
     return err;
 }
@@ -1370,23 +1314,12 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
     const uint64_t w_group_rows = a.gate_up ? 2ull * a.f : static_cast<uint64_t>(a.D);
     CUtensorMap mw, ma;
     cudaError_t err;
-    // weight boxes of 128 rows; the one-CTA tokens-on-M kernel (tile width chosen on the
-    // device) gets maps with 128-, 64- and 32-row boxes, for the routed experts and for the
-    // extra dense group (copies of the routed ones when there is none)
+    // weight boxes of 128 rows; the extra dense group's weights (one-CTA tokens-on-M
+    // kernel only) in a map of their own, else a copy of mw
     if ((err = make_map(&mw, a.w, w_group_rows * a.E, K, kBM)) != cudaSuccess) return err;
-    TmMaps tmaps;
-    if (kind == Kind::kTm) {
-        for (int i = 0; i < kNumBoxes; ++i) {
-            if ((err = make_map(&tmaps.w[i], a.w, w_group_rows * a.E, K, box_rows_of(i))) !=
-                cudaSuccess)
-                return err;
-            tmaps.w2[i] = tmaps.w[i];
-            if (a.xg_w != nullptr &&
-                (err = make_map(&tmaps.w2[i], a.xg_w, w_group_rows, K, box_rows_of(i))) !=
-                    cudaSuccess)
-                return err;
-        }
-    }
+    CUtensorMap mw2 = mw;
+    if (a.xg_w != nullptr && (err = make_map(&mw2, a.xg_w, w_group_rows, K, kBM)) != cudaSuccess)
+        return err;
     // the activation map is only read when the rows are contiguous (no gather); with a
     // gather it still has to be a valid descriptor, so it covers the first row of x
     const void* act = a.act;
@@ -1428,7 +1361,6 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
     p.ksplit = kind == Kind::kSwap && a.ksplit > 1 ? a.ksplit : 1;
     p.zero_acc = a.gate_up ? a.zero_acc : nullptr;
     p.zero_n4 = a.zero_floats / 4;
-    p.tm_adaptive = kind == Kind::kTm ? 1 : 0;
     p.act_box = BN;
     if (a.xg_w != nullptr) {
         p.xg = 1;
@@ -1439,17 +1371,16 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
     p.split_stride = static_cast<long long>(a.rows) * p.out_cols;
     // persistent grids: one CTA (or pair) per SM, fewer when the tiles cannot fill them
     const int rows_per_tile = kind == Kind::kPair ? CfgPair::kPairRows : (tm ? kTmRows : 16);
-    // (the one-CTA tokens-on-M kernel may cut its tiles up to 4x narrower on the device)
     const long long max_tiles = (static_cast<long long>(ceil_div(a.rows, rows_per_tile)) + p.G) *
-                                p.nf * p.ksplit * (kind == Kind::kTm ? 4 : 1);
+                                p.nf * p.ksplit;
     if (kind == Kind::kPair) {
         const int npairs = static_cast<int>(std::min<long long>(max_tiles, num_sms / 2));
         return a.gate_up ? launch_pair<true>(mw, ma, p, npairs, s, true)
                          : launch_pair<false>(mw, ma, p, npairs, s, true);
     }
     const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
-    if (tm) return a.gate_up ? launch_tm<true>(tmaps, ma, p, grid, s, pdl)
-                             : launch_tm<false>(tmaps, ma, p, grid, s, pdl);
+    if (tm) return a.gate_up ? launch_tm<true>(mw, ma, mw2, p, grid, s, pdl)
+                             : launch_tm<false>(mw, ma, mw2, p, grid, s, pdl);
     switch (BN) {
         case 16: return a.gate_up ? launch_tpl<16, true>(mw, ma, p, grid, s, pdl) : launch_tpl<16, false>(mw, ma, p, grid, s, pdl);
         case 32: return a.gate_up ? launch_tpl<32, true>(mw, ma, p, grid, s, pdl) : launch_tpl<32, false>(mw, ma, p, grid, s, pdl);

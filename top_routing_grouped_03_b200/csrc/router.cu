@@ -90,16 +90,21 @@ __device__ __forceinline__ void select_topk_nv(const float* lg, int planes, size
             key[j] = (e < E) ? sc[j] + (select_bias ? __ldg(select_bias + e) : 0.f) : -FLT_MAX;
         }
     }
+    // Each lane keeps the best of its own keys (lowest expert on ties); a round takes the
+    // warp's best of those, and only the lane that owned the winner retires it and looks
+    // for its next best.
+    float lv = -FLT_MAX;
+    int li = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+        const int e = j * 32 + lane;
+        if (e < E && key[j] > lv) { lv = key[j]; li = e; }  // strict: lowest e per lane
+    }
     float my_sc = 0.f;
     int my_i = 0;
     for (int k = 0; k < K; ++k) {
-        float bv = -FLT_MAX;
-        int bi = 0x7fffffff;
-#pragma unroll
-        for (int j = 0; j < NV; ++j) {
-            const int e = j * 32 + lane;
-            if (e < E && key[j] > bv) { bv = key[j]; bi = e; }  // strict: lowest e per lane
-        }
+        float bv = lv;
+        int bi = li;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
             const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
@@ -108,9 +113,16 @@ __device__ __forceinline__ void select_topk_nv(const float* lg, int planes, size
         }
         // the winner's score comes from its owner lane, which also retires it
         float wsc = 0.f;
+        if ((bi & 31) == lane) {
+            lv = -FLT_MAX;
+            li = 0x7fffffff;
 #pragma unroll
-        for (int j = 0; j < NV; ++j)
-            if (j * 32 + lane == bi) { wsc = sc[j]; key[j] = -INFINITY; }
+            for (int j = 0; j < NV; ++j) {
+                const int e = j * 32 + lane;
+                if (e == bi) { wsc = sc[j]; key[j] = -INFINITY; }
+                else if (e < E && key[j] > lv) { lv = key[j]; li = e; }
+            }
+        }
         wsc = __shfl_sync(0xffffffffu, wsc, bi & 31);
         if (lane == k) { my_sc = wsc; my_i = bi; }
     }
@@ -324,7 +336,7 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
 // planes (no bias yet), the planes added in order and the bias on load; the shared gate's
 // dot product w_s . x_t is done here by the same warp.  (The layer's accumulator is
 // cleared by the gate_up kernel on this path.)
-__global__ void __launch_bounds__(kRouterThreads) router_select_kernel(RouterLaunch a) {
+__global__ void __launch_bounds__(kRouterThreads, 4) router_select_kernel(RouterLaunch a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = blockIdx.x * (kRouterThreads / 32);
     const int nt = min(kRouterThreads / 32, a.T - t0);
