@@ -14,8 +14,6 @@
 namespace moe {
 namespace {
 
-constexpr int kMaxK = 16;  // the largest K the library takes
-
 __device__ __forceinline__ void add8(float (&acc)[8], const uint4 v, float w) {
     acc[0] = fmaf(w, bf16_lo(v.x), acc[0]);
     acc[1] = fmaf(w, bf16_hi(v.x), acc[1]);
@@ -65,20 +63,12 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineLaunch a) {
             }
         }
         if (a.y16_sorted) {
-            // every row of the token in flight at once (K <= 16), then summed in slot order
             const uint4* ys = reinterpret_cast<const uint4*>(a.y16_sorted);
-            int row[kMaxK];
-#pragma unroll
-            for (int k = 0; k < kMaxK; ++k)
-                row[k] = k < a.K ? __ldg(a.slot_to_row + t * a.K + k) : -1;
-            uint4 v[kMaxK];
-#pragma unroll
-            for (int k = 0; k < kMaxK; ++k)  // a dropped pair (row -1) adds nothing
-                v[k] = row[k] >= 0 ? __ldcs(ys + static_cast<size_t>(row[k]) * vec + c)
-                                   : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int k = 0; k < kMaxK; ++k)
-                if (row[k] >= 0) add8(acc, v[k], 1.f);
+            for (int k = 0; k < a.K; ++k) {
+                const int row = __ldg(a.slot_to_row + t * a.K + k);
+                if (row < 0) continue;  // dropped past its expert's capacity
+                add8(acc, __ldcs(ys + static_cast<size_t>(row) * vec + c), 1.f);
+            }
         }
         if (a.shared_out) {
             const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.shared_out) + i);
