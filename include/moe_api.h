@@ -362,11 +362,10 @@ MOE_API int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* wo
  * pointer of p is dereferenced, only p's shapes, flags and which pointers are NULL are
  * read).  *step_mask (if not NULL) gets bit MOE_EV_x set for every step whose interval,
  * between step events x and x + 1, launches a kernel: steps that are fused into another
- * step's kernel (the permutation into the router's last CTA for small problems, the shared
- * expert into the routed launches when it is as wide as the routed experts, the combine
- * into the last down kernel) have their bit clear.  *launches (if not NULL) gets the
- * number of kernels one call launches on the device the caller has current.  Errors as
- * the host checks of moe_layer_forward.
+ * step's kernel (the shared expert into the routed launches when it is as wide as the
+ * routed experts, the combine into the last down kernel) have their bit clear.  *launches
+ * (if not NULL) gets the number of kernels one call launches on the device the caller has
+ * current.  Errors as the host checks of moe_layer_forward.
  */
 MOE_API int moe_layer_plan(const moe_layer_params* p, unsigned* step_mask, int* launches);
 

@@ -173,11 +173,11 @@ def _plan(L, T, D, E, K, f, f_s=0, flags=0):
 
 def test_layer_plan_names_the_launched_steps(lib):
     """moe_layer_plan (host only): which steps launch kernels and how many, per regime."""
-    # decode: the permutation runs in the router's last CTA
-    assert _plan(lib, 64, 2048, 256, 8, 512) == ({"router", "gate_up", "down"}, 3)
+    # decode: router, one-CTA permutation, gate_up, down (which also writes the output)
+    assert _plan(lib, 64, 2048, 256, 8, 512) == ({"router", "permute", "gate_up", "down"}, 4)
     # fixed-order combine: one more kernel
     assert _plan(lib, 64, 2048, 256, 8, 512, flags=1) == (
-        {"router", "gate_up", "down", "combine"}, 4)
+        {"router", "permute", "gate_up", "down", "combine"}, 5)
     # fine-grained + shared: tensor-core router (logits GEMM + selection), chunked
     # permutation (histograms + scatter), the shared expert inside the routed launches
     assert _plan(lib, 4096, 4096, 512, 10, 1024, 1024) == (

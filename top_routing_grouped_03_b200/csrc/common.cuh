@@ -117,14 +117,7 @@ struct RouterLaunch {
     const float* select_bias; // [E] added to the scores for the selection only, or NULL
     int bf16_weights;         // round the renormalised weights to bf16
     int logit_planes;         // tensor-core path: partial-sum planes of [T, E] in logits
-    // CUDA-core router only: the last CTA to finish its selection also runs the
-    // permutation `perm` (one chunk: T*K <= 4096 entries, E <= 256; perm.counts = counts),
-    // taking the ticket counters[ceil(T/8)]
-    int fuse_perm;
-    PermuteLaunch perm;
 };
-// the router kernel can run the permutation of this many (token, slot) entries, E experts
-bool router_can_fuse_permute(int T, int E, int K);
 cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bool pdl = false);
 
 // Router for many tokens: the logits x W_r^T [T, E] (fp32) on the tensor cores through the

@@ -80,8 +80,7 @@ Layout layout(long long T, long long D, long long E, long long K, long long f, l
         return r;
     };
     L.status = take(kAlign);
-    // one completion ticket per 8-token block, and one for the router's last block
-    L.counters = take(sizeof(unsigned) * static_cast<size_t>((T + 7) / 8 + 1));
+    L.counters = take(sizeof(unsigned) * static_cast<size_t>((T + 7) / 8));
     L.counts = take(sizeof(int32_t) * E);
     L.zero_end = o;
     // depends on T, E and K only, so any workspace sized for the same T, E, K has it here
@@ -226,11 +225,6 @@ LayerPlan plan_layer(const moe_layer_params* p, moe_bf16* out, void* workspace, 
     r.score_mode = p->score_mode;
     r.select_bias = p->select_bias;
     r.bf16_weights = (p->flags & MOE_FLAG_BF16_WEIGHTS) ? 1 : 0;
-    // small problems: the router's last CTA also runs the permutation (one launch fewer)
-    if (router_can_fuse_permute(T, E, K)) {
-        r.fuse_perm = 1;
-        r.perm = pm;
-    }
 
     GroupedGemmLaunch& up = q.up;
     up.gate_up = true;
@@ -541,7 +535,7 @@ int moe_layer_forward(const moe_layer_params* p, moe_bf16* out, void* workspace,
     if ((q.tc_router ? launch_router_tc(q.r, sms, s) : launch_router(q.r, sms, s)) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (!mark(MOE_EV_PERMUTE)) return MOE_ERR_CUDA;
-    if (!q.r.fuse_perm && launch_permute(q.pm, s, true) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_permute(q.pm, s, true) != cudaSuccess) return MOE_ERR_CUDA;
     if (!mark(MOE_EV_GATE_UP) || launch_grouped_gemm(q.up, sms, s, true) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (!mark(MOE_EV_DOWN) || launch_grouped_gemm(q.dn, sms, s, true) != cudaSuccess)
@@ -566,7 +560,7 @@ int moe_layer_plan(const moe_layer_params* p, unsigned* step_mask, int* launches
         // nothing is dereferenced: the plan only needs the workspace's layout
         const LayerPlan q = plan_layer(p, nullptr, reinterpret_cast<void*>(kAlign), sms);
         const int nr = q.tc_router ? 2 : 1;
-        const int np = q.r.fuse_perm ? 0 : (permute_chunks(static_cast<long long>(p->T) * p->K) > 1 ? 2 : 1);
+        const int np = permute_chunks(static_cast<long long>(p->T) * p->K) > 1 ? 2 : 1;
         const int nu = grouped_gemm_launches(q.up, sms), nd = grouped_gemm_launches(q.dn, sms);
         const int ns = q.shared_launches ? grouped_gemm_launches(q.su, sms) + grouped_gemm_launches(q.sd, sms) : 0;
         const int nc = q.combine ? 1 : 0;

@@ -1,6 +1,5 @@
-// permute_body.cuh -- the row placement of the permutation, shared by the permutation
-// kernel (1024 threads, one chunk of entries per CTA) and the router kernel's last CTA
-// (256 threads, every entry of a small problem, right after the selection).
+// permute_body.cuh -- the row placement of the permutation kernel (one chunk of entries
+// per CTA), written for any CTA size NT >= E.
 //
 // "MoE" (llm.rainlin.net), section 3.2: each routed expert gathers the tokens routed to
 // it; rows of a group are in ascending (token, slot) order, a stable counting sort by

@@ -26,7 +26,6 @@
 #include <cfloat>
 
 #include "common.cuh"
-#include "permute_body.cuh"
 
 namespace moe {
 namespace {
@@ -314,21 +313,6 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
             a.shared_gate[token] = 1.f / (1.f + expf(-g));
         }
     }
-    if (!a.fuse_perm) return;
-
-    // ---- the last token block to finish its selection also groups every (token, slot)
-    //      entry by expert: the routing and the counts of all blocks are then complete
-    __shared__ int s_perm;
-    __threadfence();  // this CTA's routing and counts are visible before its ticket
-    __syncthreads();
-    if (tid == 0) {
-        const unsigned prev = atomicAdd(&a.counters[gridDim.x], 1u);
-        s_perm = (prev == gridDim.x - 1) ? 1 : 0;
-    }
-    __syncthreads();
-    if (!s_perm) return;
-    __threadfence();
-    permute_scatter_chunk<kRouterThreads>(a.perm, a.T * a.K, 1, 0, reinterpret_cast<int*>(xs));
 }
 
 
@@ -392,15 +376,7 @@ cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bo
     n_eb = max(1, min(n_eb, ceil_div(rows_total, rows_per_pass)));
     int per_cta = ceil_div(ceil_div(rows_total, n_eb), rows_per_pass) * rows_per_pass;
     n_eb = ceil_div(rows_total, per_cta);
-    size_t smem = static_cast<size_t>(kTokensPerCta) * a.D * sizeof(bf16);
-    if (a.fuse_perm) {
-        if (!router_can_fuse_permute(a.T, a.E, a.K) || a.perm.counts != a.counts)
-            return cudaErrorInvalidValue;
-        // the permutation reuses the token staging area (its tables: 8 warps' counts and
-        // three per-expert arrays)
-        smem = std::max(smem, sizeof(int) * (static_cast<size_t>(kRouterThreads / 32) * a.E +
-                                             3 * a.E + 1));
-    }
+    const size_t smem = static_cast<size_t>(kTokensPerCta) * a.D * sizeof(bf16);
     cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(router_kernel), smem);
     if (err != cudaSuccess) return err;
     err = launch_kernel(router_kernel, dim3(n_tb, n_eb), dim3(kRouterThreads), smem, s, pdl, a,
@@ -412,10 +388,6 @@ cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bo
 
 bool router_uses_tensor_cores(int T, int E) { return T >= 256 && E % 128 == 0; }
 
-bool router_can_fuse_permute(int T, int E, int K) {
-    return !router_uses_tensor_cores(T, E) && E <= kRouterThreads &&
-           static_cast<long long>(T) * K <= 4096;
-}
 
 int router_tc_max_planes(int T) { return std::min(16, std::max(1, 512 / ceil_div(T, 128))); }
 
