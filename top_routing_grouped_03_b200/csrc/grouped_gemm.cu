@@ -589,7 +589,8 @@ __device__ __forceinline__ void reduce16_transposed(const Params& p, const uint3
 // the columns this warp drains (gate_up: features [wn/4 half, wn/4 (half + 1)) of the
 // tile's wn/2; down: output columns [wn/2 half, wn/2 (half + 1)) of its wn).  The warp's
 // 32 lanes are 32 rows.
-template <bool GATE_UP>
+// ROWS16: the kernel may write bf16 rows (p.y16_out; the CTA-pair kernel only).
+template <bool GATE_UP, bool ROWS16 = false>
 __device__ __forceinline__ void tm_epilogue(const Params& p, uint32_t tbase, int row, bool valid,
                                             int tile_i, int half, float* stage, int wn,
                                             int id_base = -1) {
@@ -666,7 +667,7 @@ __device__ __forceinline__ void tm_epilogue(const Params& p, uint32_t tbase, int
             }
         }
 #pragma unroll 1
-        for (int c0 = 0; c0 < hc && p.y16_out; c0 += 32) {
+        for (int c0 = 0; c0 < hc && ROWS16 && p.y16_out; c0 += 32) {
             uint32_t v[32];
             tmem_ld32(tcol + c0, v);
             tmem_ld_wait();
@@ -763,7 +764,8 @@ __device__ __forceinline__ void build_tile_table_tm(const Params& p, int* g_off,
     }
 }
 
-template <bool GATE_UP>
+// XG: the launch carries an extra dense group (p.xg); false compiles its handling out.
+template <bool GATE_UP, bool XG>
 __global__ void __launch_bounds__(kTmThreads, 1)
 grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
                        const __grid_constant__ CUtensorMap map_act,
@@ -802,7 +804,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&map_w);
-        if (p.xg) tma_prefetch_desc(&map_w2);
+        if (XG) tma_prefetch_desc(&map_w2);
         if (!gather) tma_prefetch_desc(&map_act);
     }
     if (warp == 1) {
@@ -818,9 +820,9 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
     const uint32_t tmem_base = *tmem_slot;
     const int total = *total_slot;
     // tiles of the routed groups, and of the extra dense group (interleaved, tile_of_slot)
-    const int n_routed = p.xg ? g_tile[p.G - 1] : total;
+    const int n_routed = XG ? g_tile[p.G - 1] : total;
     const int n_extra = total - n_routed;
-    const int x_base = p.xg ? g_off[p.G - 1] : -1;  // first row of the extra group
+    const int x_base = XG ? g_off[p.G - 1] : -1;  // first row of the extra group
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
@@ -833,9 +835,9 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
             uint32_t phase = 0, filled = 0, fill_phase = 0;
             bool ok = true;
             for (int slot = blockIdx.x; slot < total && ok; slot += gridDim.x) {
-                const Tile t = decode_tile(tile_of_slot(slot, n_routed, n_extra), g_tile, g_off,
-                                           p.G, kTmRows);
-                const bool ex = p.xg && t.g == p.G - 1;
+                const Tile t = decode_tile(XG ? tile_of_slot(slot, n_routed, n_extra) : slot,
+                                           g_tile, g_off, p.G, kTmRows);
+                const bool ex = XG && t.g == p.G - 1;
                 const CUtensorMap* mw = ex ? &map_w2 : &map_w;
                 // gate_up: gate rows g*2f + i*128 and up rows g*2f + f + i*128; down: rows
                 // g*D + i*256 and the next 128 (the extra group's weights are a matrix of
@@ -932,9 +934,9 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
         if (GATE_UP) clear_accumulator(p, threadIdx.x - 64, kTmEpiThreads);
         uint32_t abuf = 0, aphase = 0;
         for (int slot = blockIdx.x; slot < total; slot += gridDim.x) {
-            const Tile t = decode_tile(tile_of_slot(slot, n_routed, n_extra), g_tile, g_off, p.G,
-                                       kTmRows);
-            const bool ex = p.xg && t.g == p.G - 1;
+            const Tile t = decode_tile(XG ? tile_of_slot(slot, n_routed, n_extra) : slot, g_tile,
+                                       g_off, p.G, kTmRows);
+            const bool ex = XG && t.g == p.G - 1;
             const bool ready = mbar_wait(&tfull[abuf], aphase, kWaitBudgetNs, abort_flag);
             if (!epilogue_bar_and<kTmEpiThreads>(ready)) {
                 set_status(p.status, MOE_ERR_TIMEOUT);
@@ -1142,8 +1144,9 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_w,
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    abuf * C::kAccCols;
             const int row = t.row0 + static_cast<int>(rank) * kTmRows + q * 32 + lane;
-            tm_epilogue<GATE_UP>(p, tbase, row, row < t.row_end, t.i, (warp - 2) >> 2,
-                                 GATE_UP ? nullptr : epi_stage(g_tile + p.G + 1, warp), kTmN);
+            tm_epilogue<GATE_UP, true>(p, tbase, row, row < t.row_end, t.i, (warp - 2) >> 2,
+                                       GATE_UP ? nullptr : epi_stage(g_tile + p.G + 1, warp),
+                                       kTmN);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_tempty0 + abuf * 8);
@@ -1247,14 +1250,14 @@ cudaError_t launch_tpl(const CUtensorMap& mw, const CUtensorMap& ma, const Param
     return err;
 }
 
-template <bool GATE_UP>
+template <bool GATE_UP, bool XG>
 cudaError_t launch_tm(const CUtensorMap& mw, const CUtensorMap& ma, const CUtensorMap& mw2,
                       const Params& p, int grid, cudaStream_t s, bool pdl) {
     using C = CfgTm;
     const size_t smem = 1024 + static_cast<size_t>(C::kStages) * C::kStageBytes +
                         (2 * C::kStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int) +
                         (GATE_UP ? 0 : kEpiStageBytes);
-    auto kfn = grouped_gemm_tm_kernel<GATE_UP>;
+    auto kfn = grouped_gemm_tm_kernel<GATE_UP, XG>;
     cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(kfn), smem);
     if (err != cudaSuccess) return err;
     err = launch_kernel(kfn, dim3(grid), dim3(kTmThreads), smem, s, pdl, mw, ma, mw2, p);
@@ -1379,8 +1382,11 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
                          : launch_pair<false>(mw, ma, p, npairs, s, true);
     }
     const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
-    if (tm) return a.gate_up ? launch_tm<true>(mw, ma, mw2, p, grid, s, pdl)
-                             : launch_tm<false>(mw, ma, mw2, p, grid, s, pdl);
+    if (tm && p.xg)
+        return a.gate_up ? launch_tm<true, true>(mw, ma, mw2, p, grid, s, pdl)
+                         : launch_tm<false, true>(mw, ma, mw2, p, grid, s, pdl);
+    if (tm) return a.gate_up ? launch_tm<true, false>(mw, ma, mw2, p, grid, s, pdl)
+                             : launch_tm<false, false>(mw, ma, mw2, p, grid, s, pdl);
     switch (BN) {
         case 16: return a.gate_up ? launch_tpl<16, true>(mw, ma, p, grid, s, pdl) : launch_tpl<16, false>(mw, ma, p, grid, s, pdl);
         case 32: return a.gate_up ? launch_tpl<32, true>(mw, ma, p, grid, s, pdl) : launch_tpl<32, false>(mw, ma, p, grid, s, pdl);

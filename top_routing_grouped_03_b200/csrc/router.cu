@@ -89,21 +89,16 @@ __device__ __forceinline__ void select_topk_nv(const float* lg, int planes, size
             key[j] = (e < E) ? sc[j] + (select_bias ? __ldg(select_bias + e) : 0.f) : -FLT_MAX;
         }
     }
-    // Each lane keeps the best of its own keys (lowest expert on ties); a round takes the
-    // warp's best of those, and only the lane that owned the winner retires it and looks
-    // for its next best.
-    float lv = -FLT_MAX;
-    int li = 0x7fffffff;
-#pragma unroll
-    for (int j = 0; j < NV; ++j) {
-        const int e = j * 32 + lane;
-        if (e < E && key[j] > lv) { lv = key[j]; li = e; }  // strict: lowest e per lane
-    }
     float my_sc = 0.f;
     int my_i = 0;
     for (int k = 0; k < K; ++k) {
-        float bv = lv;
-        int bi = li;
+        float bv = -FLT_MAX;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const int e = j * 32 + lane;
+            if (e < E && key[j] > bv) { bv = key[j]; bi = e; }  // strict: lowest e per lane
+        }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
             const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
@@ -112,16 +107,9 @@ __device__ __forceinline__ void select_topk_nv(const float* lg, int planes, size
         }
         // the winner's score comes from its owner lane, which also retires it
         float wsc = 0.f;
-        if ((bi & 31) == lane) {
-            lv = -FLT_MAX;
-            li = 0x7fffffff;
 #pragma unroll
-            for (int j = 0; j < NV; ++j) {
-                const int e = j * 32 + lane;
-                if (e == bi) { wsc = sc[j]; key[j] = -INFINITY; }
-                else if (e < E && key[j] > lv) { lv = key[j]; li = e; }
-            }
-        }
+        for (int j = 0; j < NV; ++j)
+            if (j * 32 + lane == bi) { wsc = sc[j]; key[j] = -INFINITY; }
         wsc = __shfl_sync(0xffffffffu, wsc, bi & 31);
         if (lane == k) { my_sc = wsc; my_i = bi; }
     }
@@ -181,22 +169,6 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
         float4* dst = reinterpret_cast<float4*>(a.zero_acc + static_cast<size_t>(t0) * a.zero_cols);
         const int b = blockIdx.y * per, e = min(b + per, n4);
         for (int i = b + tid; i < e; i += kRouterThreads) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-
-    // ---- bring this warp's first expert rows toward L2 while the token rows are staged
-    //      (the two DRAM round trips overlap instead of following each other)
-    {
-        const int e_first = blockIdx.y * experts_per_cta + warp * kExpertsPerWarp;
-        const int e_stop = min(blockIdx.y * experts_per_cta + experts_per_cta, rows_total);
-#pragma unroll
-        for (int u = 0; u < kExpertsPerWarp; ++u) {
-            const int e = e_first + u;
-            if (e >= e_stop) break;
-            const char* row = reinterpret_cast<const char*>(
-                (e < E) ? a.w_router + static_cast<size_t>(e) * D : a.w_shared_gate);
-            for (int l = lane; l < D * 2 / 128; l += 32)
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(row + l * 128));
-        }
     }
 
     // ---- stage the 8 token rows (zeros past T)
