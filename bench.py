@@ -76,19 +76,15 @@ def layer_bytes(cfg, U: int) -> float:
         4.0 * cfg.T * cfg.D
 
 
-def gate_up_bytes(cfg, U: int, with_shared: bool = False) -> float:
+def gate_up_bytes(cfg, U: int) -> float:
     """Algorithmic bytes of one grouped gate_up launch: gate+up weights of the U experts
-    hit, the T*K gathered token rows read, the T*K x f SwiGLU rows written; with the shared
-    expert inside the launch also its gate+up weights, T more rows in and out."""
+    hit, the T*K gathered token rows read, the T*K x f SwiGLU rows written."""
     rows = cfg.T * cfg.K
-    b = 2.0 * 2 * cfg.D * cfg.f * U + 2.0 * rows * cfg.D + 2.0 * rows * cfg.f
-    if with_shared:
-        b += 2.0 * 2 * cfg.D * cfg.f_s + 2.0 * cfg.T * cfg.D + 2.0 * cfg.T * cfg.f_s
-    return b
+    return 2.0 * 2 * cfg.D * cfg.f * U + 2.0 * rows * cfg.D + 2.0 * rows * cfg.f
 
 
-def gate_up_flops(cfg, with_shared: bool = False) -> float:
-    return 4.0 * cfg.D * cfg.f * cfg.T * cfg.K + (4.0 * cfg.D * cfg.f_s * cfg.T if with_shared else 0.0)
+def gate_up_flops(cfg) -> float:
+    return 4.0 * cfg.D * cfg.f * cfg.T * cfg.K
 
 
 def load_peaks():
@@ -712,9 +708,7 @@ def main():
     peaks, src = load_peaks()
     peak_hbm = peaks["hbm_gbs"]
     peak_tc = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    plan_steps, _ = w.layer.plan(T)
-    in_gu = cfg.f_s > 0 and "shared" not in plan_steps  # shared expert inside the launch
-    gu_bytes, gu_flops = gate_up_bytes(cfg, U, in_gu), gate_up_flops(cfg, in_gu)
+    gu_bytes, gu_flops = gate_up_bytes(cfg, U), gate_up_flops(cfg)
     if gu_flops / (peak_tc * 1e12) > gu_bytes / (peak_hbm * 1e9):
         roof = {"bound": "tensor", "achieved": gu_flops / (gu_ms / 1e3) / 1e12, "peak": peak_tc,
                 "unit": "TFLOP/s", "peak_source": f"{src} (bf16_tflops, burst)",
@@ -728,7 +722,7 @@ def main():
     roof["traffic"] = ncu_traffic("grouped_gemm_gate_up", cfg.name)
     roof["algorithmic_bytes_per_launch"] = gu_bytes
     roof["avg_launch_ms"] = gu_ms
-    roof["kernel"] = "grouped_gemm gate_up + SwiGLU" + (" (with the shared expert)" if in_gu else "")
+    roof["kernel"] = "grouped_gemm gate_up + SwiGLU"
     roof["timing"] = (f"CUDA events around the gate_up launch in {args.steps} eager layer "
                       f"calls right after the timed steps (L2 flushed before each)")
     line = {

@@ -179,10 +179,10 @@ def test_layer_plan_names_the_launched_steps(lib):
     assert _plan(lib, 64, 2048, 256, 8, 512, flags=1) == (
         {"router", "permute", "gate_up", "down", "combine"}, 5)
     # fine-grained + shared: tensor-core router (logits GEMM + selection), chunked
-    # permutation (histograms + scatter), the shared expert inside the routed launches
+    # permutation (histograms + scatter), the shared expert's two launches (the last one
+    # writes the output)
     assert _plan(lib, 4096, 4096, 512, 10, 1024, 1024) == (
-        {"router", "permute", "gate_up", "down"}, 6)
-    # a shared expert of another width keeps its two launches
+        {"router", "permute", "gate_up", "down", "shared"}, 8)
     assert _plan(lib, 4096, 4096, 512, 10, 1024, 512) == (
         {"router", "permute", "gate_up", "down", "shared"}, 8)
     # prefill: CTA pairs, whose gate_up first copies the token rows into expert order and

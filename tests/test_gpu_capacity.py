@@ -72,8 +72,7 @@ CAP_LAYERS = {
     "tc_router_shared": (LayerConfig("tc_router_shared", T=300, D=384, E=128, K=6, f=128,
                                      f_s=256, seed=8), 1.25, 4),
     "few_tokens": (LayerConfig("few_tokens", T=12, D=256, E=8, K=4, f=256, seed=9), 1.0, 0),
-    # shared expert as wide as the routed ones: an extra group of the routed launches, its
-    # rows placed after the kept routed rows
+    # shared expert as wide as the routed ones, with tokens dropped from the routed groups
     "shared_fused": (LayerConfig("shared_fused", T=100, D=256, E=16, K=4, f=256, f_s=256,
                                  seed=16), 0.8, 2),
 }

@@ -54,9 +54,9 @@ SMALL_LAYERS = {
     # at most 16 tokens: weights-on-M grouped GEMMs, routed and shared
     "few_tokens_shared": LayerConfig("few_tokens_shared", T=12, D=256, E=32, K=4, f=256,
                                      f_s=128, seed=9),
-    # shared expert as wide as the routed ones: it runs as an extra, interleaved group of
-    # the routed launches (routed groups of a few to ~50 rows; then many small groups with
-    # the tensor-core router and several shared row blocks)
+    # shared expert as wide as the routed ones, on the tokens-on-M kernel (routed groups of
+    # a few to ~50 rows; then many small groups with the tensor-core router and several
+    # shared row blocks)
     "shared_fused": LayerConfig("shared_fused", T=100, D=256, E=16, K=4, f=256, f_s=256,
                                 seed=16),
     "shared_fused_tc": LayerConfig("shared_fused_tc", T=520, D=512, E=128, K=8, f=256,

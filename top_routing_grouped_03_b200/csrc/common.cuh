@@ -168,19 +168,7 @@ struct GroupedGemmLaunch {
     // kernel, before the down projection adds into it; NULL: nothing to clear
     float* zero_acc;
     long long zero_floats;
-    // one extra dense group after the E routed ones (the shared expert), run inside the same
-    // launch with its tiles interleaved: weights xg_w ([2f, D] gate_up or [D, f] down, the
-    // routed experts' f), rows [offsets[E], offsets[E] + xg_rows) of the sorted problem,
-    // row r being token r - offsets[E]; down scales row r by xg_weight[token].  `rows`
-    // then counts these rows too.  Only the one-CTA tokens-on-M kernel takes it
-    // (grouped_gemm_takes_extra_group); NULL: none
-    const void* xg_w;
-    int xg_rows;
-    const float* xg_weight;
 };
-// true when launch_grouped_gemm would run `a` on the one-CTA tokens-on-M kernel (the one
-// that can carry an extra dense group)
-bool grouped_gemm_takes_extra_group(const GroupedGemmLaunch& a, int num_sms);
 // true when launch_grouped_gemm would run `a` on CTA pairs
 bool grouped_gemm_uses_pairs(const GroupedGemmLaunch& a, int num_sms);
 // kernels launch_grouped_gemm launches for `a` (0 when it has nothing to do)

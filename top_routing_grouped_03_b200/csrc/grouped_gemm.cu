@@ -103,13 +103,6 @@ struct Params {
     long long zero_n4;
     // weights-on-M kernel with contiguous token rows: rows per activation TMA box (= BN)
     int act_box;
-    // one-CTA tokens-on-M kernel: group G-1 is an extra dense group (the shared expert):
-    // its xg_rows rows follow the routed ones, [offsets[G-1], offsets[G-1] + xg_rows), row
-    // r is token r - offsets[G-1], its weights come from the second weight map, and (down)
-    // row r is scaled by xg_weight[token]; its tiles are interleaved with the routed ones
-    int xg;
-    int xg_rows;
-    const float* xg_weight;
 };
 
 // Epilogue threads of every CTA clear their grid-strided share of p.zero_acc.
@@ -255,15 +248,14 @@ struct RowGather {
     uint32_t src_off[kChunks];  // element offset of the chunk's row in x (< 2^31)
     uint32_t valid;
 
-    // id_base >= 0: row r is token r - id_base (a dense group), tok is not read
     __device__ __forceinline__ void plan(const int32_t* tok, int row0, int row_end, int row_len,
-                                         int lane, int id_base = -1) {
+                                         int lane) {
         valid = 0;
 #pragma unroll
         for (int u = 0; u < kChunks; ++u) {
             const int row = row0 + (lane >> 3) + 4 * u;
             const bool ok = row < row_end;
-            const int t = ok ? (id_base >= 0 ? row - id_base : __ldg(tok + row)) : 0;
+            const int t = ok ? __ldg(tok + row) : 0;
             src_off[u] = static_cast<uint32_t>(t) * row_len + (lane & 7) * 8;
             valid |= (ok ? 1u : 0u) << u;
         }
@@ -592,8 +584,7 @@ __device__ __forceinline__ void reduce16_transposed(const Params& p, const uint3
 // ROWS16: the kernel may write bf16 rows (p.y16_out; the CTA-pair kernel only).
 template <bool GATE_UP, bool ROWS16 = false>
 __device__ __forceinline__ void tm_epilogue(const Params& p, uint32_t tbase, int row, bool valid,
-                                            int tile_i, int half, float* stage, int wn,
-                                            int id_base = -1) {
+                                            int tile_i, int half, float* stage, int wn) {
     const int lane = threadIdx.x & 31;
     if (GATE_UP) {
         const int F = wn >> 1;        // features of the tile
@@ -620,17 +611,8 @@ __device__ __forceinline__ void tm_epilogue(const Params& p, uint32_t tbase, int
         }
     } else {
         const int hc = wn >> 1;  // output columns of this warp: 128, 64 or 32
-        // token and weight of this row: the extra dense group's row r is token r - id_base,
-        // scaled by xg_weight[token]
-        float w = 1.f;
-        int tok = 0;
-        if (valid && id_base >= 0) {
-            tok = row - id_base;
-            w = __ldg(p.xg_weight + tok);
-        } else if (valid) {
-            tok = p.sorted_token ? __ldg(p.sorted_token + row) : row;
-            w = p.sorted_w ? __ldg(p.sorted_w + row) : 1.f;
-        }
+        const float w = (valid && p.sorted_w) ? __ldg(p.sorted_w + row) : 1.f;
+        const int tok = valid ? (p.sorted_token ? __ldg(p.sorted_token + row) : row) : 0;
         const int col0 = tile_i * wn + half * hc;
         const uint32_t tcol = tbase + half * hc;
         // a warp with a handful of rows (a few tokens per expert) reduces row by row: the
@@ -720,56 +702,10 @@ struct CfgTm {
     static_assert(kTmemCols <= 512, "accumulators exceed tensor memory");
 };
 
-// Processing order of the one-CTA kernel's tiles when an extra dense group is present:
-// its n_x tiles (table indices n_r .. n_r + n_x - 1, after the routed groups' n_r) take
-// every s-th slot, s = floor((n_r + n_x) / n_x), so that its compute-bound tiles run
-// alongside the weight-streaming routed tiles instead of all at the end.  Returns the
-// table index of slot t.
-__device__ __forceinline__ int tile_of_slot(int t, int n_r, int n_x) {
-    if (n_x <= 0) return t;
-    const int s = (n_r + n_x) / n_x;
-    const int q = t / s;
-    if (t - q * s == s - 1 && q < n_x) return n_r + q;
-    return t - min(n_x, q);
-}
-
-// The group table of the one-CTA tokens-on-M kernel: as build_tile_table, except that with
-// an extra dense group (p.xg) the last group's end is offsets[G-1] + xg_rows.
-__device__ __forceinline__ void build_tile_table_tm(const Params& p, int* g_off, int* g_tile,
-                                                    int* total_slot, int warp, int lane) {
-    for (int i = threadIdx.x; i <= p.G; i += blockDim.x)
-        g_off[i] = p.offsets ? (p.xg && i == p.G ? p.offsets[i - 1] + p.xg_rows : p.offsets[i])
-                             : (i == 0 ? 0 : p.rows_total);
-    __syncthreads();
-    if (warp == 2) {
-        const int per = (p.G + 31) / 32;
-        const int gb = min(lane * per, p.G), ge = min(gb + per, p.G);
-        int local = 0;
-        for (int g = gb; g < ge; ++g) local += group_tiles(p, g_off[g + 1] - g_off[g], kTmRows);
-        int incl = local;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        int run = incl - local;
-        for (int g = gb; g < ge; ++g) {
-            g_tile[g] = run;
-            run += group_tiles(p, g_off[g + 1] - g_off[g], kTmRows);
-        }
-        if (lane == 31) {
-            g_tile[p.G] = incl;
-            *total_slot = incl;
-        }
-    }
-}
-
-// XG: the launch carries an extra dense group (p.xg); false compiles its handling out.
-template <bool GATE_UP, bool XG>
+template <bool GATE_UP>
 __global__ void __launch_bounds__(kTmThreads, 1)
 grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
-                       const __grid_constant__ CUtensorMap map_act,
-                       const __grid_constant__ CUtensorMap map_w2, Params p) {
+                       const __grid_constant__ CUtensorMap map_act, Params p) {
     using C = CfgTm;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -804,7 +740,6 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&map_w);
-        if (XG) tma_prefetch_desc(&map_w2);
         if (!gather) tma_prefetch_desc(&map_act);
     }
     if (warp == 1) {
@@ -813,16 +748,12 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
     }
     grid_dep_wait();
     grid_dep_launch();
-    build_tile_table_tm(p, g_off, g_tile, total_slot, warp, lane);
+    build_tile_table(p, kTmRows, g_off, g_tile, total_slot, warp, lane);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int total = *total_slot;
-    // tiles of the routed groups, and of the extra dense group (interleaved, tile_of_slot)
-    const int n_routed = XG ? g_tile[p.G - 1] : total;
-    const int n_extra = total - n_routed;
-    const int x_base = XG ? g_off[p.G - 1] : -1;  // first row of the extra group
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
@@ -834,19 +765,14 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
             int stage = 0;
             uint32_t phase = 0, filled = 0, fill_phase = 0;
             bool ok = true;
-            for (int slot = blockIdx.x; slot < total && ok; slot += gridDim.x) {
-                const Tile t = decode_tile(XG ? tile_of_slot(slot, n_routed, n_extra) : slot,
-                                           g_tile, g_off, p.G, kTmRows);
-                const bool ex = XG && t.g == p.G - 1;
-                const CUtensorMap* mw = ex ? &map_w2 : &map_w;
-                // gate_up: gate rows g*2f + i*128 and up rows g*2f + f + i*128; down: rows
-                // g*D + i*256 and the next 128 (the extra group's weights are a matrix of
-                // their own: g = 0 there)
-                const int wr0 = (ex ? 0 : t.g * p.w_group_rows) + t.i * (GATE_UP ? kBM : kTmN);
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const Tile t = decode_tile(tile, g_tile, g_off, p.G, kTmRows);
+                // gate_up: gate rows g*2f + i*128 and up rows g*2f + f + i*128;
+                // down: rows g*D + i*256 and the next 128
+                const int wr0 = t.g * p.w_group_rows + t.i * (GATE_UP ? kBM : kTmN);
                 const int wr1 = GATE_UP ? wr0 + p.up_rows : wr0 + kBM;
                 RowGather<kTmRows> rg;
-                if (gather)
-                    rg.plan(p.gather_tok, t.row0, t.row_end, p.nk * kBK, lane, ex ? x_base : -1);
+                if (gather) rg.plan(p.gather_tok, t.row0, t.row_end, p.nk * kBK, lane);
                 for (int kk = 0; kk < p.nk; ++kk) {
                     bool got = mbar_wait(&empty[stage], phase ^ 1u, kWaitBudgetNs, abort_flag);
                     if (gather) got = __all_sync(0xffffffffu, got);
@@ -861,9 +787,9 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
                         mbar_arrive_expect_tx(&full[stage], gather ? C::kBBytes : C::kStageBytes);
                         if (!gather)
                             tma_load_2d(st, &map_act, &full[stage], kk * kBK, t.row0, pol_a);
-                        tma_load_2d(st + C::kABytes, mw, &full[stage], kk * kBK, wr0, pol_w);
-                        tma_load_2d(st + C::kABytes + kBM * kBK * 2, mw, &full[stage], kk * kBK,
-                                    wr1, pol_w);
+                        tma_load_2d(st + C::kABytes, &map_w, &full[stage], kk * kBK, wr0, pol_w);
+                        tma_load_2d(st + C::kABytes + kBM * kBK * 2, &map_w, &full[stage],
+                                    kk * kBK, wr1, pol_w);
                     }
                     if (gather) {
                         rg.issue(smem_u32(st), p.x, kk * kBK, lane);
@@ -889,7 +815,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
             int stage = 0;
             uint32_t phase = 0, abuf = 0, aphase = 0;
             bool ok = true, issued = false;
-            for (int slot = blockIdx.x; slot < total && ok; slot += gridDim.x) {
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
                 if (!mbar_wait(&tempty[abuf], aphase ^ 1u, kWaitBudgetNs, abort_flag)) {
                     set_status(p.status, MOE_ERR_TIMEOUT);
                     *abort_flag = 1;
@@ -933,10 +859,8 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
         const int q = warp & 3;
         if (GATE_UP) clear_accumulator(p, threadIdx.x - 64, kTmEpiThreads);
         uint32_t abuf = 0, aphase = 0;
-        for (int slot = blockIdx.x; slot < total; slot += gridDim.x) {
-            const Tile t = decode_tile(XG ? tile_of_slot(slot, n_routed, n_extra) : slot, g_tile,
-                                       g_off, p.G, kTmRows);
-            const bool ex = XG && t.g == p.G - 1;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const Tile t = decode_tile(tile, g_tile, g_off, p.G, kTmRows);
             const bool ready = mbar_wait(&tfull[abuf], aphase, kWaitBudgetNs, abort_flag);
             if (!epilogue_bar_and<kTmEpiThreads>(ready)) {
                 set_status(p.status, MOE_ERR_TIMEOUT);
@@ -948,8 +872,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
                                    abuf * C::kAccCols;
             const int row = t.row0 + q * 32 + lane;
             tm_epilogue<GATE_UP>(p, tbase, row, row < t.row_end, t.i, (warp - 2) >> 2,
-                                 GATE_UP ? nullptr : epi_stage(g_tile + p.G + 1, warp), kTmN,
-                                 ex ? x_base : -1);
+                                 GATE_UP ? nullptr : epi_stage(g_tile + p.G + 1, warp), kTmN);
             tc_fence_before();
             mbar_arrive(&tempty[abuf]);
             abuf ^= 1u;
@@ -1250,17 +1173,17 @@ cudaError_t launch_tpl(const CUtensorMap& mw, const CUtensorMap& ma, const Param
     return err;
 }
 
-template <bool GATE_UP, bool XG>
-cudaError_t launch_tm(const CUtensorMap& mw, const CUtensorMap& ma, const CUtensorMap& mw2,
-                      const Params& p, int grid, cudaStream_t s, bool pdl) {
+template <bool GATE_UP>
+cudaError_t launch_tm(const CUtensorMap& mw, const CUtensorMap& ma, const Params& p, int grid,
+                      cudaStream_t s, bool pdl) {
     using C = CfgTm;
     const size_t smem = 1024 + static_cast<size_t>(C::kStages) * C::kStageBytes +
                         (2 * C::kStages + 5) * 8 + 16 + 2 * (p.G + 1) * sizeof(int) +
                         (GATE_UP ? 0 : kEpiStageBytes);
-    auto kfn = grouped_gemm_tm_kernel<GATE_UP, XG>;
+    auto kfn = grouped_gemm_tm_kernel<GATE_UP>;
     cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(kfn), smem);
     if (err != cudaSuccess) return err;
-    err = launch_kernel(kfn, dim3(grid), dim3(kTmThreads), smem, s, pdl, mw, ma, mw2, p);
+    err = launch_kernel(kfn, dim3(grid), dim3(kTmThreads), smem, s, pdl, mw, ma, p);
     count_launches(1);
     return err;
 }
@@ -1317,12 +1240,7 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
     const uint64_t w_group_rows = a.gate_up ? 2ull * a.f : static_cast<uint64_t>(a.D);
     CUtensorMap mw, ma;
     cudaError_t err;
-    // weight boxes of 128 rows; the extra dense group's weights (one-CTA tokens-on-M
-    // kernel only) in a map of their own, else a copy of mw
-    if ((err = make_map(&mw, a.w, w_group_rows * a.E, K, kBM)) != cudaSuccess) return err;
-    CUtensorMap mw2 = mw;
-    if (a.xg_w != nullptr && (err = make_map(&mw2, a.xg_w, w_group_rows, K, kBM)) != cudaSuccess)
-        return err;
+    if ((err = make_map(&mw, a.w, w_group_rows * a.E, K, kBM)) != cudaSuccess) return err;  // 128-row boxes
     // the activation map is only read when the rows are contiguous (no gather); with a
     // gather it still has to be a valid descriptor, so it covers the first row of x
     const void* act = a.act;
@@ -1365,12 +1283,6 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
     p.zero_acc = a.gate_up ? a.zero_acc : nullptr;
     p.zero_n4 = a.zero_floats / 4;
     p.act_box = BN;
-    if (a.xg_w != nullptr) {
-        p.xg = 1;
-        p.G = a.E + 1;
-        p.xg_rows = a.xg_rows;
-        p.xg_weight = a.xg_weight;
-    }
     p.split_stride = static_cast<long long>(a.rows) * p.out_cols;
     // persistent grids: one CTA (or pair) per SM, fewer when the tiles cannot fill them
     const int rows_per_tile = kind == Kind::kPair ? CfgPair::kPairRows : (tm ? kTmRows : 16);
@@ -1382,11 +1294,8 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
                          : launch_pair<false>(mw, ma, p, npairs, s, true);
     }
     const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
-    if (tm && p.xg)
-        return a.gate_up ? launch_tm<true, true>(mw, ma, mw2, p, grid, s, pdl)
-                         : launch_tm<false, true>(mw, ma, mw2, p, grid, s, pdl);
-    if (tm) return a.gate_up ? launch_tm<true, false>(mw, ma, mw2, p, grid, s, pdl)
-                             : launch_tm<false, false>(mw, ma, mw2, p, grid, s, pdl);
+    if (tm) return a.gate_up ? launch_tm<true>(mw, ma, p, grid, s, pdl)
+                             : launch_tm<false>(mw, ma, p, grid, s, pdl);
     switch (BN) {
         case 16: return a.gate_up ? launch_tpl<16, true>(mw, ma, p, grid, s, pdl) : launch_tpl<16, false>(mw, ma, p, grid, s, pdl);
         case 32: return a.gate_up ? launch_tpl<32, true>(mw, ma, p, grid, s, pdl) : launch_tpl<32, false>(mw, ma, p, grid, s, pdl);
@@ -1407,7 +1316,7 @@ bool pick_kind(const GroupedGemmLaunch& a, int num_sms, Kind* kind, int* BN) {
     const bool tm_ok = a.gate_up ? (a.f % 128 == 0) : (a.D % 256 == 0);
     const bool gathered = a.gate_up && a.gather_tok != nullptr;
     const bool pair_ok = tm_ok && (!gathered || a.gather_buf != nullptr) && num_sms >= 2;
-    const int routed_rows = a.rows - (a.xg_w != nullptr ? a.xg_rows : 0);
+    const int routed_rows = a.rows;
     // weights on M: tiles adapt per group up to BN, sized for groups up to 8x the average
     // (skewed routing) but never past the largest possible group
     const int max_rows = a.max_group_rows > 0 ? a.max_group_rows : routed_rows;
@@ -1455,25 +1364,16 @@ bool grouped_gemm_uses_pairs(const GroupedGemmLaunch& a, int num_sms) {
     return pick_kind(a, num_sms, &kind, &BN) && kind == Kind::kPair;
 }
 
-bool grouped_gemm_takes_extra_group(const GroupedGemmLaunch& a, int num_sms) {
-    Kind kind;
-    int BN;
-    return pick_kind(a, num_sms, &kind, &BN) && kind == Kind::kTm;
-}
 
 cudaError_t launch_grouped_gemm(const GroupedGemmLaunch& a, int num_sms, cudaStream_t s,
                                 bool pdl) {
     if (a.rows == 0 || a.E == 0) return cudaSuccess;
-    if (a.E + (a.xg_w != nullptr ? 1 : 0) > kMaxGroups) return cudaErrorInvalidValue;
+    if (a.E > kMaxGroups) return cudaErrorInvalidValue;
     cudaError_t err = get_encoder();
     if (err != cudaSuccess) return err;
     Kind kind;
     int BN;
     if (!pick_kind(a, num_sms, &kind, &BN)) return cudaErrorInvalidValue;
-    // an extra dense group (the shared expert) rides only on the one-CTA tokens-on-M kernel
-    if (a.xg_w != nullptr &&
-        (kind != Kind::kTm || a.offsets == nullptr || (!a.gate_up && a.xg_weight == nullptr)))
-        return cudaErrorInvalidValue;
     return launch_kind(a, kind, BN, num_sms, s, pdl);
 }
 

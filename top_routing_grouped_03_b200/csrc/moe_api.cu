@@ -99,9 +99,7 @@ Layout layout(long long T, long long D, long long E, long long K, long long f, l
     L.sorted_w = take(sizeof(float) * T * K);
     L.slot_to_row = take(sizeof(int32_t) * T * K);
     L.x_sorted = take(2 * T * K * D);
-    // h: the routed rows, then room for the shared expert's T rows when it runs as an extra
-    // group of the routed launches (f_s = f)
-    L.h = take(2 * (T * K + T) * f);
+    L.h = take(2 * T * K * f);
     L.h_s = take(2 * T * fs);
     L.out_acc = take(sizeof(float) * T * D);
     L.y_sorted = take(sizeof(float) * T * K * D);
@@ -152,7 +150,7 @@ struct LayerPlan {
     PermuteLaunch pm;
     GroupedGemmLaunch up, dn, su, sd;
     CombineLaunch c;
-    bool tc_router, det, fuse_shared, shared_launches;
+    bool tc_router, det, shared_launches;
     bool rows_mode;  // down on CTA pairs writes weighted bf16 rows; the combine sums them
     bool combine;    // a combine launch ends the call
 };
@@ -239,17 +237,7 @@ LayerPlan plan_layer(const moe_layer_params* p, moe_bf16* out, void* workspace, 
     up.status = status;
     up.zero_acc = use_acc && q.tc_router ? out_acc : nullptr;
     up.zero_floats = static_cast<long long>(T) * D;
-    // The shared expert (same width as the routed ones) runs as one more, dense group of the
-    // routed gate_up and down launches when they take the one-CTA tokens-on-M kernel: its
-    // compute-bound tiles then interleave with the weight-streaming routed tiles instead of
-    // running as two launches of their own.  Its rows follow the routed rows in h.
-    q.fuse_shared = shared && !q.det && fs == f && grouped_gemm_takes_extra_group(up, sms);
-    q.shared_launches = shared && !q.fuse_shared;
-    if (q.fuse_shared) {
-        up.xg_w = p->w_shared_gate_up;
-        up.xg_rows = T;
-        up.rows = rows + T;
-    }
+    q.shared_launches = shared;
 
     GroupedGemmLaunch& dn = q.dn;
     dn.gate_up = false;
@@ -264,12 +252,6 @@ LayerPlan plan_layer(const moe_layer_params* p, moe_bf16* out, void* workspace, 
     dn.y_out = q.det ? at<float>(workspace, L.y_sorted) : nullptr;
     dn.y16_out = q.rows_mode ? at<bf16>(workspace, L.x_sorted) : nullptr;
     dn.status = status;
-    if (q.fuse_shared) {
-        dn.xg_w = p->w_shared_down;
-        dn.xg_rows = T;
-        dn.xg_weight = sgate;
-        dn.rows = rows + T;
-    }
     // without the fixed-order combine, the last launch also writes the bf16 output after a
     // grid-wide step
     unsigned* done = at<unsigned>(workspace, L.status + 64);  // inside the cleared header
