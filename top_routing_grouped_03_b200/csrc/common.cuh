@@ -168,6 +168,15 @@ struct GroupedGemmLaunch {
     // kernel, before the down projection adds into it; NULL: nothing to clear
     float* zero_acc;
     long long zero_floats;
+    // weights-on-M and one-CTA tokens-on-M kernels: let the kernel cut each tile's K steps
+    // into up to ksplit_max slices (1, 2 or 4) when the tiles cannot fill the grid.
+    // gate_up needs `part` (ksplit_max planes of [rows, 2f] fp32) and `tickets` (ticket_cap
+    // words, zero at launch, one per tile; more tiles than that: no split); down needs
+    // acc_out without y_out / y16_out.  0 or 1: no split.
+    int ksplit_max;
+    float* part;
+    unsigned* tickets;
+    int ticket_cap;
 };
 // true when launch_grouped_gemm would run `a` on CTA pairs
 bool grouped_gemm_uses_pairs(const GroupedGemmLaunch& a, int num_sms);

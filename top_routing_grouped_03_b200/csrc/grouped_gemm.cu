@@ -103,6 +103,18 @@ struct Params {
     long long zero_n4;
     // weights-on-M kernel with contiguous token rows: rows per activation TMA box (= BN)
     int act_box;
+    // Split of each tile's K steps chosen on the device (weights-on-M kernel when ksplit is
+    // 1, and the one-CTA tokens-on-M kernel): up to ksplit_max slices, picked from the tile
+    // count so that the (tile, slice) units fill the grid's waves.  down: every slice adds
+    // its partial products into acc_out.  gate_up: every slice writes its fp32 partial sums
+    // to part, [slice][row][gate f | up f] with part_rows rows per slice; the slice that
+    // completes a tile (tickets[tile], zero at launch, ticket_cap of them) adds them in
+    // slice order and applies SwiGLU.
+    int ksplit_max;
+    float* part;
+    int part_rows;
+    unsigned* tickets;
+    int ticket_cap;
 };
 
 // Epilogue threads of every CTA clear their grid-strided share of p.zero_acc.
@@ -239,6 +251,56 @@ __device__ __forceinline__ void build_tile_table(const Params& p, int rows_per_t
     }
 }
 
+// Slices per tile (1, 2 or 4; at most smax; dividing nk with at least kSplitMinSteps K
+// steps each) minimising the time of the (tile, slice) units over `ctas` CTAs: a unit of
+// nk / s K steps costs them plus kSplitRampSteps for its pipeline ramp, epilogue and
+// fix-up, and the units run in ceil(tiles s / ctas) waves.  Integer costs, so every
+// thread gets the same answer; a tie keeps fewer slices.
+constexpr int kSplitSlicesMax = 4;
+constexpr int kSplitMinSteps = 4;
+constexpr int kSplitRampSteps = 4;
+__device__ __forceinline__ int choose_split(int tiles, int ctas, int nk, int smax) {
+    int best = 1;
+    long long best_cost = static_cast<long long>((tiles + ctas - 1) / ctas) * (nk + kSplitRampSteps);
+    for (int s = 2; s <= smax && s <= kSplitSlicesMax; s <<= 1) {
+        if (nk % s != 0 || nk / s < kSplitMinSteps) break;
+        const long long waves = (static_cast<long long>(tiles) * s + ctas - 1) / ctas;
+        const long long cost = waves * (nk / s + kSplitRampSteps);
+        if (cost < best_cost) {
+            best = s;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
+// Slices per tile for this launch (host-fixed ksplit, else chosen on the device).
+__device__ __forceinline__ int tile_split(const Params& p, int tiles, bool gate_up) {
+    if (p.ksplit > 1) return p.ksplit;
+    if (p.ksplit_max <= 1 || tiles == 0) return 1;
+    if (gate_up && (p.part == nullptr || p.tickets == nullptr || tiles > p.ticket_cap)) return 1;
+    return choose_split(tiles, gridDim.x, p.nk, p.ksplit_max);
+}
+
+// gate_up split: once every epilogue thread has written its partial sums of the tile, one
+// ticket per slice (a release/acquire atomic by one thread, ordered with the other epilogue
+// threads' stores and later loads by the barriers); true in every epilogue thread of the
+// CTA that took the last one -- it then sees all slices' partial sums.
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+template <int kThreads>
+__device__ __forceinline__ bool split_tile_done(const Params& p, int tile, int nsplit,
+                                                int first_epi_tid) {
+    epilogue_bar_and<kThreads>(true);
+    bool last = true;
+    if (threadIdx.x == first_epi_tid)
+        last = atom_add_acq_rel_gpu(p.tickets + tile, 1u) == static_cast<unsigned>(nsplit - 1);
+    return epilogue_bar_and<kThreads>(last);
+}
+
 // Per-lane plan for gathering ROWS token rows of x into a 128-byte-swizzled operand tile
 // with cp.async: lane l owns 16-byte chunk c = l % 8 of tile rows l/8 + 4u; that chunk of
 // tile row r lands at r*128 + ((c ^ (r % 8)) * 16).
@@ -331,9 +393,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    // tiles: (group tile, K slice) with the slice varying fastest, so that CTAs working at
+    // units: (group tile, K slice) with the slice varying fastest, so that CTAs working at
     // the same time read different K ranges of the weights
-    const int nsplit = p.ksplit;
+    const int nsplit = tile_split(p, *total_slot, GATE_UP);
     const int total = *total_slot * nsplit;
     const int nks = p.nk / nsplit;  // K steps per slice
 
@@ -453,6 +515,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             const Tile t = decode_tile(tile / nsplit, g_tile, g_off, p.G, BN);
             float* y_slice = p.y_out ? p.y_out + (tile % nsplit) * p.split_stride : nullptr;
+            // gate_up cut into slices: this slice's partial sums, [row][gate f | up f]
+            float* part = (GATE_UP && nsplit > 1)
+                              ? p.part + static_cast<size_t>(tile % nsplit) * p.part_rows * 2 * p.out_cols
+                              : nullptr;
             const bool ready = mbar_wait(&tfull[abuf], aphase, kWaitBudgetNs, abort_flag);
             if (!epilogue_bar_and(ready)) {
                 set_status(p.status, MOE_ERR_TIMEOUT);
@@ -475,7 +541,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                     const int row = t.row0 + c0 + c;
                     if (row >= t.row_end) break;
                     const float g = __uint_as_float(gv[c]);
-                    if (GATE_UP) {
+                    if (GATE_UP && part) {
+                        float* pr = part + static_cast<size_t>(row) * 2 * p.out_cols;
+                        __stcg(pr + feat, g);
+                        __stcg(pr + p.out_cols + feat, __uint_as_float(uv[c]));
+                    } else if (GATE_UP) {
                         const float u = __uint_as_float(uv[c]);
                         const float h = g / (1.f + __expf(-g)) * u;
                         p.h_out[static_cast<size_t>(row) * p.out_cols + feat] = __float2bfloat16_rn(h);
@@ -494,6 +564,39 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
             mbar_arrive(&tempty[abuf]);
             abuf ^= 1u;
             if (abuf == 0) aphase ^= 1u;
+            // the slice that completes the tile: sum the slices' partial sums in slice
+            // order, then SwiGLU into h
+            if (GATE_UP && part && split_tile_done<kEpiThreads>(p, tile / nsplit, nsplit, 64)) {
+                // 4 rows' partial sums in flight at a time
+                const int row_hi = min(t.row0 + BN, t.row_end);
+#pragma unroll 1
+                for (int r0 = t.row0; r0 < row_hi; r0 += 4) {
+                    float gs[4][kSplitSlicesMax], us[4][kSplitSlicesMax];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+#pragma unroll
+                        for (int sl = 0; sl < kSplitSlicesMax; ++sl) {
+                            gs[r][sl] = us[r][sl] = 0.f;
+                            if (sl >= nsplit || r0 + r >= row_hi) continue;
+                            const float* pr = p.part +
+                                (static_cast<size_t>(sl) * p.part_rows + r0 + r) * 2 * p.out_cols;
+                            gs[r][sl] = __ldcg(pr + feat);
+                            us[r][sl] = __ldcg(pr + p.out_cols + feat);
+                        }
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        if (r0 + r >= row_hi) break;
+                        float g = 0.f, u = 0.f;
+#pragma unroll
+                        for (int sl = 0; sl < kSplitSlicesMax; ++sl) {
+                            g += gs[r][sl];  // slices past nsplit hold 0
+                            u += us[r][sl];
+                        }
+                        const float h = g / (1.f + __expf(-g)) * u;
+                        p.h_out[static_cast<size_t>(r0 + r) * p.out_cols + feat] = __float2bfloat16_rn(h);
+                    }
+                }
+            }
         }
     }
 
@@ -512,8 +615,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
 // down: 256 output features), one tcgen05.mma of 128 x 256 x 16 per 16 of K.  Each
 // epilogue thread owns one row, so h is written with 16-byte stores and the down epilogue
 // reduces 16-byte vectors (red.global.add.v4.f32) into the token's output row.  The
-// one-CTA kernel can carry one extra, dense group (the shared expert) whose weights come
-// from a second tensor map; the CTA-pair kernel shares the tile shape.
+// CTA-pair kernel shares the tile shape.
 constexpr int kTmRows = 128;  // token rows per tile (MMA M)
 // weights on M while no group can exceed this many rows (a handful of tokens): measured
 // faster than tokens on M there (one token: 47 vs 50 us for gate_up at the Zipf T=1 shape)
@@ -577,6 +679,57 @@ __device__ __forceinline__ void reduce16_transposed(const Params& p, const uint3
     __syncwarp();
 }
 
+// gate_up cut into K slices, the CTA whose slice completed the tile: h[row, feat0 + j] for
+// the tile's rows [row0, row_end) and its F features, from the slices' partial sums added
+// in slice order.  The epilogue threads share (row, 8-feature chunk) items, so that a tile
+// of a few rows costs one round trip to L2.
+template <int kThreads>
+__device__ __forceinline__ void split_fixup_tile(const Params& p, int row0, int row_end,
+                                                 int feat0, int F, int nsplit, int epi_tid) {
+    const int chunks = F / 8;
+    const int items = (row_end - row0) * chunks;
+#pragma unroll 1
+    for (int it = epi_tid; it < items; it += kThreads) {
+        const int row = row0 + it / chunks;
+        const int f = feat0 + (it % chunks) * 8;
+        float4 a[kSplitSlicesMax][2], b[kSplitSlicesMax][2];
+#pragma unroll
+        for (int sl = 0; sl < kSplitSlicesMax; ++sl) {
+            if (sl >= nsplit) break;
+            const float* pr =
+                p.part + (static_cast<size_t>(sl) * p.part_rows + row) * 2 * p.out_cols + f;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                a[sl][j] = __ldcg(reinterpret_cast<const float4*>(pr) + j);
+                b[sl][j] = __ldcg(reinterpret_cast<const float4*>(pr + p.out_cols) + j);
+            }
+        }
+        float g[8], u[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) g[j] = u[j] = 0.f;
+#pragma unroll
+        for (int sl = 0; sl < kSplitSlicesMax; ++sl) {
+            if (sl >= nsplit) break;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                g[4 * j] += a[sl][j].x; g[4 * j + 1] += a[sl][j].y;
+                g[4 * j + 2] += a[sl][j].z; g[4 * j + 3] += a[sl][j].w;
+                u[4 * j] += b[sl][j].x; u[4 * j + 1] += b[sl][j].y;
+                u[4 * j + 2] += b[sl][j].z; u[4 * j + 3] += b[sl][j].w;
+            }
+        }
+        uint32_t pk[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float h0 = __fdividef(g[2 * j], 1.f + __expf(-g[2 * j])) * u[2 * j];
+            const float h1 = __fdividef(g[2 * j + 1], 1.f + __expf(-g[2 * j + 1])) * u[2 * j + 1];
+            pk[j] = pack_bf16x2(h0, h1);
+        }
+        *reinterpret_cast<uint4*>(p.h_out + static_cast<size_t>(row) * p.out_cols + f) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+}
+
 // Epilogue of one tokens-on-M tile (wn weight rows) for one epilogue warp: `half` selects
 // the columns this warp drains (gate_up: features [wn/4 half, wn/4 (half + 1)) of the
 // tile's wn/2; down: output columns [wn/2 half, wn/2 (half + 1)) of its wn).  The warp's
@@ -584,9 +737,33 @@ __device__ __forceinline__ void reduce16_transposed(const Params& p, const uint3
 // ROWS16: the kernel may write bf16 rows (p.y16_out; the CTA-pair kernel only).
 template <bool GATE_UP, bool ROWS16 = false>
 __device__ __forceinline__ void tm_epilogue(const Params& p, uint32_t tbase, int row, bool valid,
-                                            int tile_i, int half, float* stage, int wn) {
+                                            int tile_i, int half, float* stage, int wn,
+                                            float* part = nullptr) {
     const int lane = threadIdx.x & 31;
-    if (GATE_UP) {
+    if (GATE_UP && part) {
+        // one K slice of the tile: fp32 partial sums of the gate and up features
+        const int F = wn >> 1;
+        const int hc = F >> 1;
+        float* prow = part + static_cast<size_t>(row) * 2 * p.out_cols + tile_i * F + half * hc;
+#pragma unroll 1
+        for (int c0 = 0; c0 < hc; c0 += 32) {
+            uint32_t gv[32], uv[32];
+            tmem_ld32(tbase + half * hc + c0, gv);
+            tmem_ld32(tbase + F + half * hc + c0, uv);
+            tmem_ld_wait();
+            if (valid) {
+                float4* dg = reinterpret_cast<float4*>(prow + c0);
+                float4* du = reinterpret_cast<float4*>(prow + p.out_cols + c0);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    __stcg(dg + j, make_float4(__uint_as_float(gv[4 * j]), __uint_as_float(gv[4 * j + 1]),
+                                               __uint_as_float(gv[4 * j + 2]), __uint_as_float(gv[4 * j + 3])));
+                    __stcg(du + j, make_float4(__uint_as_float(uv[4 * j]), __uint_as_float(uv[4 * j + 1]),
+                                               __uint_as_float(uv[4 * j + 2]), __uint_as_float(uv[4 * j + 3])));
+                }
+            }
+        }
+    } else if (GATE_UP) {
         const int F = wn >> 1;        // features of the tile
         const int hc = F >> 1;        // features of this warp: 64, 32 or 16
         bf16* hrow = p.h_out + static_cast<size_t>(row) * p.out_cols + tile_i * F + half * hc;
@@ -753,7 +930,10 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int total = *total_slot;
+    // units: (tile, K slice), the slice varying fastest
+    const int nsplit = tile_split(p, *total_slot, GATE_UP);
+    const int total = *total_slot * nsplit;
+    const int nks = p.nk / nsplit;  // K steps per slice
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
@@ -766,14 +946,15 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
             uint32_t phase = 0, filled = 0, fill_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const Tile t = decode_tile(tile, g_tile, g_off, p.G, kTmRows);
+                const Tile t = decode_tile(tile / nsplit, g_tile, g_off, p.G, kTmRows);
+                const int kb = (tile % nsplit) * nks;
                 // gate_up: gate rows g*2f + i*128 and up rows g*2f + f + i*128;
                 // down: rows g*D + i*256 and the next 128
                 const int wr0 = t.g * p.w_group_rows + t.i * (GATE_UP ? kBM : kTmN);
                 const int wr1 = GATE_UP ? wr0 + p.up_rows : wr0 + kBM;
                 RowGather<kTmRows> rg;
                 if (gather) rg.plan(p.gather_tok, t.row0, t.row_end, p.nk * kBK, lane);
-                for (int kk = 0; kk < p.nk; ++kk) {
+                for (int kk = kb; kk < kb + nks; ++kk) {
                     bool got = mbar_wait(&empty[stage], phase ^ 1u, kWaitBudgetNs, abort_flag);
                     if (gather) got = __all_sync(0xffffffffu, got);
                     if (!got) {
@@ -824,7 +1005,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
                 }
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + abuf * C::kAccCols;
-                for (int kk = 0; kk < p.nk; ++kk) {
+                for (int kk = 0; kk < nks; ++kk) {
                     if (!mbar_wait(&full[stage], phase, kWaitBudgetNs, abort_flag)) {
                         set_status(p.status, MOE_ERR_TIMEOUT);
                         *abort_flag = 1;
@@ -860,7 +1041,7 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
         if (GATE_UP) clear_accumulator(p, threadIdx.x - 64, kTmEpiThreads);
         uint32_t abuf = 0, aphase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const Tile t = decode_tile(tile, g_tile, g_off, p.G, kTmRows);
+            const Tile t = decode_tile(tile / nsplit, g_tile, g_off, p.G, kTmRows);
             const bool ready = mbar_wait(&tfull[abuf], aphase, kWaitBudgetNs, abort_flag);
             if (!epilogue_bar_and<kTmEpiThreads>(ready)) {
                 set_status(p.status, MOE_ERR_TIMEOUT);
@@ -871,12 +1052,24 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    abuf * C::kAccCols;
             const int row = t.row0 + q * 32 + lane;
-            tm_epilogue<GATE_UP>(p, tbase, row, row < t.row_end, t.i, (warp - 2) >> 2,
-                                 GATE_UP ? nullptr : epi_stage(g_tile + p.G + 1, warp), kTmN);
+            const bool valid = row < t.row_end;
+            const int half = (warp - 2) >> 2;
+            // gate_up cut into slices: this slice's partial sums, [row][gate f | up f]
+            float* part = (GATE_UP && nsplit > 1)
+                              ? p.part + static_cast<size_t>(tile % nsplit) * p.part_rows * 2 * p.out_cols
+                              : nullptr;
+            tm_epilogue<GATE_UP>(p, tbase, row, valid, t.i, half,
+                                 GATE_UP ? nullptr : epi_stage(g_tile + p.G + 1, warp), kTmN, part);
             tc_fence_before();
             mbar_arrive(&tempty[abuf]);
             abuf ^= 1u;
             if (abuf == 0) aphase ^= 1u;
+            // the slice that completes the tile sums the slices' partial sums in slice
+            // order and applies SwiGLU
+            if (GATE_UP && part && split_tile_done<kTmEpiThreads>(p, tile / nsplit, nsplit, 64))
+                split_fixup_tile<kTmEpiThreads>(p, t.row0, min(t.row0 + kTmRows, t.row_end),
+                                                t.i * (kTmN / 2), kTmN / 2, nsplit,
+                                                threadIdx.x - 64);
         }
     }
 
@@ -968,7 +1161,9 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_w,
     if (warp == 0) {
         // ---------------------------------------------------------------- producer (both)
         if (lane == 0) {
-            const uint64_t pol_w = policy_evict_first();
+            // a weight tile is read by every row block of its expert (consecutive tiles, run by
+            // pairs at about the same time): kept in L2 like the token rows for the others
+            const uint64_t pol_w = policy_evict_last();
             const uint64_t pol_a = policy_evict_last();
             int stage = 0;
             uint32_t phase = 0, filled = 0, fill_phase = 0;
@@ -1284,10 +1479,21 @@ cudaError_t launch_kind(const GroupedGemmLaunch& a, Kind kind, int BN, int num_s
     p.zero_n4 = a.zero_floats / 4;
     p.act_box = BN;
     p.split_stride = static_cast<long long>(a.rows) * p.out_cols;
-    // persistent grids: one CTA (or pair) per SM, fewer when the tiles cannot fill them
+    // K split chosen on the device: gate_up needs the partial-sum planes and tickets, down
+    // adds its slices into the fp32 accumulator (not into per-row outputs)
+    const bool auto_split =
+        kind != Kind::kPair && p.ksplit == 1 && a.ksplit_max > 1 &&
+        (a.gate_up ? (a.part != nullptr && a.tickets != nullptr && a.ticket_cap > 0)
+                   : (a.acc_out != nullptr && a.y_out == nullptr && a.y16_out == nullptr));
+    p.ksplit_max = auto_split ? std::min(a.ksplit_max, kSplitSlicesMax) : 1;
+    p.part = a.part;
+    p.part_rows = a.rows;
+    p.tickets = a.tickets;
+    p.ticket_cap = a.ticket_cap;
+    // persistent grids: one CTA (or pair) per SM, fewer when the units cannot fill them
     const int rows_per_tile = kind == Kind::kPair ? CfgPair::kPairRows : (tm ? kTmRows : 16);
     const long long max_tiles = (static_cast<long long>(ceil_div(a.rows, rows_per_tile)) + p.G) *
-                                p.nf * p.ksplit;
+                                p.nf * p.ksplit * p.ksplit_max;
     if (kind == Kind::kPair) {
         const int npairs = static_cast<int>(std::min<long long>(max_tiles, num_sms / 2));
         return a.gate_up ? launch_pair<true>(mw, ma, p, npairs, s, true)
@@ -1333,9 +1539,9 @@ bool pick_kind(const GroupedGemmLaunch& a, int num_sms, Kind* kind, int* BN) {
     // Otherwise tokens on M: both orientations stream each weight tile once per row block
     // and are within a few percent of each other on 2-row groups, but tokens on M keeps
     // features along the accumulator's columns (16-byte stores and vector reductions in
-    // the epilogue), wins clearly once groups hold tens of rows, and picks its tile width
-    // on the device, so that a few experts (a handful of tokens, or concentrated routing)
-    // still spread their weight reads over the whole GPU.  CTA pairs once the groups
+    // the epilogue) and wins clearly once groups hold tens of rows; when a few experts (a
+    // handful of tokens, or concentrated routing) give fewer tiles than the grid has CTAs,
+    // both cut each tile's K steps on the device.  CTA pairs once the groups
     // average a full 256-row pair tile's half (their rows must be contiguous: x is
     // gathered first).
     if (a.orientation == 1 || a.block_rows || !tm_ok || a.ksplit > 1)

@@ -66,10 +66,25 @@ int num_sms_current() {
 
 // Workspace of the whole layer.  The status word is always at offset 0.
 struct Layout {
-    size_t status, counters, counts, perm_hist, logits, offsets, dense_offsets, topk_idx, topk_w, sgate,
-        sorted_token, sorted_w, slot_to_row, x_sorted, h, h_s, out_acc, y_sorted, total;
+    size_t status, counters, counts, tickets, perm_hist, logits, offsets, dense_offsets, topk_idx,
+        topk_w, sgate, sorted_token, sorted_w, slot_to_row, x_sorted, h, h_s, out_acc, y_sorted,
+        part, total;
     size_t zero_end;  // [0, zero_end) is cleared at the start of a layer call
 };
+
+// The routed gate_up may cut its tiles' K steps into up to kSplitMax slices when its tiles
+// cannot fill the GPU (a few tokens, or a few experts), if the slices' fp32 partial sums
+// (kSplitMax planes of [T*K, 2f]) take at most 64 MiB; one ticket per tile, bounded by the
+// tiles of 16-row blocks: min(E, T*K) + T*K/16 + 1 row blocks of f/128 feature blocks.
+constexpr int kSplitMax = 4;
+bool gate_up_split_ok(long long T, long long K, long long f) {
+    return 4ll * kSplitMax * T * K * 2 * f <= (64ll << 20);
+}
+long long gate_up_ticket_cap(long long T, long long E, long long K, long long f) {
+    if (!gate_up_split_ok(T, K, f)) return 0;
+    const long long rows = T * K;
+    return (std::min(E, rows) + rows / 16 + 1) * (f / 128);
+}
 
 Layout layout(long long T, long long D, long long E, long long K, long long f, long long fs) {
     Layout L{};
@@ -82,6 +97,7 @@ Layout layout(long long T, long long D, long long E, long long K, long long f, l
     L.status = take(kAlign);
     L.counters = take(sizeof(unsigned) * static_cast<size_t>((T + 7) / 8));
     L.counts = take(sizeof(int32_t) * E);
+    L.tickets = take(sizeof(unsigned) * gate_up_ticket_cap(T, E, K, f));
     L.zero_end = o;
     // depends on T, E and K only, so any workspace sized for the same T, E, K has it here
     L.perm_hist = take(sizeof(int32_t) * E * permute_chunks(T * K));
@@ -103,6 +119,7 @@ Layout layout(long long T, long long D, long long E, long long K, long long f, l
     L.h_s = take(2 * T * fs);
     L.out_acc = take(sizeof(float) * T * D);
     L.y_sorted = take(sizeof(float) * T * K * D);
+    L.part = take(gate_up_split_ok(T, K, f) ? sizeof(float) * kSplitMax * T * K * 2 * f : 0);
     L.total = o;
     return L;
 }
@@ -233,6 +250,12 @@ LayerPlan plan_layer(const moe_layer_params* p, moe_bf16* out, void* workspace, 
     up.offsets = pm.offsets;
     up.rows = rows; up.E = E; up.D = D; up.f = f;
     up.max_group_rows = capacity >= 0 && capacity < T ? static_cast<int>(capacity) : T;
+    if (gate_up_split_ok(T, K, f)) {
+        up.ksplit_max = kSplitMax;
+        up.part = at<float>(workspace, L.part);
+        up.tickets = at<unsigned>(workspace, L.tickets);
+        up.ticket_cap = static_cast<int>(gate_up_ticket_cap(T, E, K, f));
+    }
     up.h_out = at<bf16>(workspace, L.h);
     up.status = status;
     up.zero_acc = use_acc && q.tc_router ? out_acc : nullptr;
@@ -252,6 +275,8 @@ LayerPlan plan_layer(const moe_layer_params* p, moe_bf16* out, void* workspace, 
     dn.y_out = q.det ? at<float>(workspace, L.y_sorted) : nullptr;
     dn.y16_out = q.rows_mode ? at<bf16>(workspace, L.x_sorted) : nullptr;
     dn.status = status;
+    // K slices add into the accumulator in any order: not with the fixed-order combine
+    dn.ksplit_max = q.det ? 1 : kSplitMax;
     // without the fixed-order combine, the last launch also writes the bf16 output after a
     // grid-wide step
     unsigned* done = at<unsigned>(workspace, L.status + 64);  // inside the cleared header
@@ -283,6 +308,7 @@ LayerPlan plan_layer(const moe_layer_params* p, moe_bf16* out, void* workspace, 
         sd.rows = T; sd.E = 1; sd.D = D; sd.f = fs;
         sd.acc_out = out_acc;
         sd.status = status;
+        sd.ksplit_max = q.det ? 1 : kSplitMax;
     }
     // fixed order: out_acc's shared part (if any) + the routed rows in slot order
     CombineLaunch& c = q.c;

@@ -35,6 +35,11 @@ constexpr int kRouterThreads = 256;
 // E <= 512: at most 16 logits per lane in the selection (select_topk_warp)
 constexpr int kExpertsPerWarp = 2;
 
+// Brings the 128-byte line holding `p` into L2 (no register result, nothing waits on it).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // TopK of one token's logits by one warp, in registers, then the renormalised weights.
 // lg: the token's E logits (bias already added when add_bias is NULL), or `planes` partial
 // sums of them `plane_stride` floats apart, added in plane order.  Writes idx/w of the
@@ -171,12 +176,40 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
         for (int i = b + tid; i < e; i += kRouterThreads) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 
-    // ---- stage the 8 token rows (zeros past T)
+    const int e_begin = blockIdx.y * experts_per_cta;
+    const int e_end = min(e_begin + experts_per_cta, rows_total);
     const int vec_per_row = D / 8;
-    const uint4* xsrc = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0) * D);
-    for (int i = tid; i < kTokensPerCta * vec_per_row; i += kRouterThreads) {
-        const int r = i / vec_per_row;
-        xs[i] = (r < nt) ? __ldg(xsrc + i) : make_uint4(0, 0, 0, 0);
+
+    // ---- pull this CTA's weight rows towards L2 while the token rows are staged (they
+    //      come from HBM on the first token block; 128-byte lines)
+    {
+        const int lines_per_row = D * 2 / 128;
+        const int nlines = (e_end - e_begin) * lines_per_row;
+        for (int i = tid; i < nlines; i += kRouterThreads) {
+            const int e = e_begin + i / lines_per_row;
+            const bf16* wrow = (e < E) ? a.w_router + static_cast<size_t>(e) * D : a.w_shared_gate;
+            prefetch_l2(reinterpret_cast<const char*>(wrow) + (i % lines_per_row) * 128);
+        }
+    }
+
+    // ---- stage the 8 token rows (zeros past T): kBatch loads in flight per thread
+    {
+        constexpr int kBatch = 8;
+        const int nvec = kTokensPerCta * vec_per_row;
+        const uint4* xsrc = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0) * D);
+        for (int i0 = tid; i0 < nvec; i0 += kBatch * kRouterThreads) {
+            uint4 v[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int i = i0 + u * kRouterThreads;
+                v[u] = (i < nvec && i / vec_per_row < nt) ? __ldg(xsrc + i) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int i = i0 + u * kRouterThreads;
+                if (i < nvec) xs[i] = v[u];
+            }
+        }
     }
     __syncthreads();
 
@@ -184,8 +217,6 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
     //      a time (one unpack of x serves all of them), each lane keeps kUnroll chunks of
     //      16-byte weight loads per row in flight
     constexpr int kUnroll = 4;
-    const int e_begin = blockIdx.y * experts_per_cta;
-    const int e_end = min(e_begin + experts_per_cta, rows_total);
     for (int e0 = e_begin + warp * kExpertsPerWarp; e0 < e_end;
          e0 += (kRouterThreads / 32) * kExpertsPerWarp) {
         const uint4* wv[kExpertsPerWarp];
