@@ -169,7 +169,7 @@ struct GroupedGemmLaunch {
     float* zero_acc;
     long long zero_floats;
     // weights-on-M and one-CTA tokens-on-M kernels: let the kernel cut each tile's K steps
-    // into up to ksplit_max slices (1, 2 or 4) when the tiles cannot fill the grid.
+    // into up to ksplit_max slices (1 to 4) when the tiles cannot fill the grid.
     // gate_up needs `part` (ksplit_max planes of [rows, 2f] fp32) and `tickets` (ticket_cap
     // words, zero at launch, one per tile; more tiles than that: no split); down needs
     // acc_out without y_out / y16_out.  0 or 1: no split.

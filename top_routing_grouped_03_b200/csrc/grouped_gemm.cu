@@ -251,21 +251,25 @@ __device__ __forceinline__ void build_tile_table(const Params& p, int rows_per_t
     }
 }
 
-// Slices per tile (1, 2 or 4; at most smax; dividing nk with at least kSplitMinSteps K
-// steps each) minimising the time of the (tile, slice) units over `ctas` CTAs: a unit of
-// nk / s K steps costs them plus kSplitRampSteps for its pipeline ramp, epilogue and
-// fix-up, and the units run in ceil(tiles s / ctas) waves.  Integer costs, so every
-// thread gets the same answer; a tie keeps fewer slices.
+// Slices per tile (1 to 4, at most smax, each of at least kSplitMinSteps K steps; slice j
+// of s takes steps [j nk / s, (j + 1) nk / s)) minimising the time of the (tile, slice)
+// units over `ctas` CTAs: a unit costs its K steps (at most ceil(nk / s)) plus
+// kSplitRampSteps for its pipeline ramp, epilogue and fix-up, and the units run in
+// ceil(tiles s / ctas) waves.  Integer costs, so every thread gets the same answer; a tie
+// keeps fewer slices.
 constexpr int kSplitSlicesMax = 4;
 constexpr int kSplitMinSteps = 4;
 constexpr int kSplitRampSteps = 4;
+__device__ __forceinline__ int slice_begin(int nk, int nsplit, int slice) {
+    return slice * nk / nsplit;
+}
 __device__ __forceinline__ int choose_split(int tiles, int ctas, int nk, int smax) {
     int best = 1;
     long long best_cost = static_cast<long long>((tiles + ctas - 1) / ctas) * (nk + kSplitRampSteps);
-    for (int s = 2; s <= smax && s <= kSplitSlicesMax; s <<= 1) {
-        if (nk % s != 0 || nk / s < kSplitMinSteps) break;
+    for (int s = 2; s <= smax && s <= kSplitSlicesMax; ++s) {
+        if (nk / s < kSplitMinSteps) break;
         const long long waves = (static_cast<long long>(tiles) * s + ctas - 1) / ctas;
-        const long long cost = waves * (nk / s + kSplitRampSteps);
+        const long long cost = waves * ((nk + s - 1) / s + kSplitRampSteps);
         if (cost < best_cost) {
             best = s;
             best_cost = cost;
@@ -397,7 +401,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
     // the same time read different K ranges of the weights
     const int nsplit = tile_split(p, *total_slot, GATE_UP);
     const int total = *total_slot * nsplit;
-    const int nks = p.nk / nsplit;  // K steps per slice
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
@@ -414,11 +417,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
                 const Tile t = decode_tile(tile / nsplit, g_tile, g_off, p.G, BN);
-                const int kb = (tile % nsplit) * nks;
+                const int kb = slice_begin(p.nk, nsplit, tile % nsplit);
+                const int ke = slice_begin(p.nk, nsplit, tile % nsplit + 1);
                 const int wr0 = t.g * p.w_group_rows + t.i * kBM;
                 RowGather<BN> rg;
                 if (gather) rg.plan(p.gather_tok, t.row0, t.row_end, p.nk * kBK, lane);
-                for (int kk = kb; kk < kb + nks; ++kk) {
+                for (int kk = kb; kk < ke; ++kk) {
                     bool got = mbar_wait(&empty[stage], phase ^ 1u, kWaitBudgetNs, abort_flag);
                     if (gather) got = __all_sync(0xffffffffu, got);
                     if (!got) {
@@ -472,6 +476,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + abuf * C::kAccCols;
                 constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
+                const int nks = slice_begin(p.nk, nsplit, tile % nsplit + 1) -
+                                slice_begin(p.nk, nsplit, tile % nsplit);
                 for (int kk = 0; kk < nks; ++kk) {
                     if (!mbar_wait(&full[stage], phase, kWaitBudgetNs, abort_flag)) {
                         set_status(p.status, MOE_ERR_TIMEOUT);
@@ -933,7 +939,6 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
     // units: (tile, K slice), the slice varying fastest
     const int nsplit = tile_split(p, *total_slot, GATE_UP);
     const int total = *total_slot * nsplit;
-    const int nks = p.nk / nsplit;  // K steps per slice
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
@@ -947,14 +952,15 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
                 const Tile t = decode_tile(tile / nsplit, g_tile, g_off, p.G, kTmRows);
-                const int kb = (tile % nsplit) * nks;
+                const int kb = slice_begin(p.nk, nsplit, tile % nsplit);
+                const int ke = slice_begin(p.nk, nsplit, tile % nsplit + 1);
                 // gate_up: gate rows g*2f + i*128 and up rows g*2f + f + i*128;
                 // down: rows g*D + i*256 and the next 128
                 const int wr0 = t.g * p.w_group_rows + t.i * (GATE_UP ? kBM : kTmN);
                 const int wr1 = GATE_UP ? wr0 + p.up_rows : wr0 + kBM;
                 RowGather<kTmRows> rg;
                 if (gather) rg.plan(p.gather_tok, t.row0, t.row_end, p.nk * kBK, lane);
-                for (int kk = kb; kk < kb + nks; ++kk) {
+                for (int kk = kb; kk < ke; ++kk) {
                     bool got = mbar_wait(&empty[stage], phase ^ 1u, kWaitBudgetNs, abort_flag);
                     if (gather) got = __all_sync(0xffffffffu, got);
                     if (!got) {
@@ -1005,6 +1011,8 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
                 }
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + abuf * C::kAccCols;
+                const int nks = slice_begin(p.nk, nsplit, tile % nsplit + 1) -
+                                slice_begin(p.nk, nsplit, tile % nsplit);
                 for (int kk = 0; kk < nks; ++kk) {
                     if (!mbar_wait(&full[stage], phase, kWaitBudgetNs, abort_flag)) {
                         set_status(p.status, MOE_ERR_TIMEOUT);

@@ -154,10 +154,13 @@ __device__ __forceinline__ void select_topk_warp(const float* lg, int planes,
 #undef MOE_SELECT
 }
 
+// dsplit: warps per expert pair, each over D / dsplit of the dot products (1, 2, 4 or 8)
 __global__ void __launch_bounds__(kRouterThreads)
-router_kernel(RouterLaunch a, int experts_per_cta) {
+router_kernel(RouterLaunch a, int experts_per_cta, int dsplit) {
     extern __shared__ __align__(16) uint4 xs[];  // [8][D] bf16 tokens of this block
     __shared__ int s_last;
+    // per-warp partial sums of a pass when the dot products are split over warps
+    __shared__ float s_part[kRouterThreads / 32][kExpertsPerWarp][kTokensPerCta];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int D = a.D, E = a.E;
     const int t0 = blockIdx.x * kTokensPerCta;
@@ -213,12 +216,17 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
     }
     __syncthreads();
 
-    // ---- logits of this CTA's expert slab: each warp takes kExpertsPerWarp expert rows at
-    //      a time (one unpack of x serves all of them), each lane keeps kUnroll chunks of
-    //      16-byte weight loads per row in flight
+    // ---- logits of this CTA's expert slab: each group of dsplit warps takes kExpertsPerWarp
+    //      expert rows at a time (one unpack of x serves all of them), warp w of the group
+    //      the w-th D / dsplit columns; each lane keeps kUnroll chunks of 16-byte weight loads
+    //      per row in flight; the group's partial sums meet in shared memory
     constexpr int kUnroll = 4;
-    for (int e0 = e_begin + warp * kExpertsPerWarp; e0 < e_end;
-         e0 += (kRouterThreads / 32) * kExpertsPerWarp) {
+    const int groups = (kRouterThreads / 32) / dsplit;
+    const int grp = warp / dsplit, part = warp % dsplit;
+    const int c_lo = part * vec_per_row / dsplit, c_hi = (part + 1) * vec_per_row / dsplit;
+    const int passes = (e_end - e_begin + groups * kExpertsPerWarp - 1) / (groups * kExpertsPerWarp);
+    for (int pass = 0; pass < passes; ++pass) {
+        const int e0 = e_begin + (pass * groups + grp) * kExpertsPerWarp;
         const uint4* wv[kExpertsPerWarp];
         bool has[kExpertsPerWarp];
 #pragma unroll
@@ -233,19 +241,19 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
         for (int u = 0; u < kExpertsPerWarp; ++u)
 #pragma unroll
             for (int t = 0; t < kTokensPerCta; ++t) acc[u][t] = 0.f;
-        for (int c0 = lane; c0 < vec_per_row; c0 += 32 * kUnroll) {
+        for (int c0 = c_lo + lane; c0 < c_hi; c0 += 32 * kUnroll) {
             uint4 w[kUnroll][kExpertsPerWarp];
 #pragma unroll
             for (int v = 0; v < kUnroll; ++v)
 #pragma unroll
                 for (int u = 0; u < kExpertsPerWarp; ++u) {
                     const int c = c0 + 32 * v;
-                    w[v][u] = (c < vec_per_row && has[u]) ? __ldg(wv[u] + c) : make_uint4(0, 0, 0, 0);
+                    w[v][u] = (c < c_hi && has[u]) ? __ldg(wv[u] + c) : make_uint4(0, 0, 0, 0);
                 }
 #pragma unroll
             for (int v = 0; v < kUnroll; ++v) {
                 const int c = c0 + 32 * v;
-                if (c >= vec_per_row) break;
+                if (c >= c_hi) break;
                 float wf[kExpertsPerWarp][8];
 #pragma unroll
                 for (int u = 0; u < kExpertsPerWarp; ++u) {
@@ -283,7 +291,22 @@ router_kernel(RouterLaunch a, int experts_per_cta) {
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1)
                     acc[u][t] += __shfl_xor_sync(0xffffffffu, acc[u][t], off);
-        if (lane == 0) {
+        if (dsplit > 1) {
+            if (lane == 0)
+#pragma unroll
+                for (int u = 0; u < kExpertsPerWarp; ++u)
+#pragma unroll
+                    for (int t = 0; t < kTokensPerCta; ++t) s_part[warp][u][t] = acc[u][t];
+            __syncthreads();
+            if (part == 0 && lane == 0)  // the group's parts in D order
+                for (int q = 1; q < dsplit; ++q)
+#pragma unroll
+                    for (int u = 0; u < kExpertsPerWarp; ++u)
+#pragma unroll
+                        for (int t = 0; t < kTokensPerCta; ++t) acc[u][t] += s_part[warp + q][u][t];
+            __syncthreads();
+        }
+        if (part == 0 && lane == 0) {
 #pragma unroll
             for (int u = 0; u < kExpertsPerWarp; ++u) {
                 const int e = e0 + u;
@@ -373,7 +396,15 @@ cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bo
     if (a.T == 0) return cudaSuccess;
     const int n_tb = ceil_div(a.T, kTokensPerCta);
     const int rows_total = a.E + (a.w_shared_gate ? 1 : 0);
-    const int rows_per_pass = (kRouterThreads / 32) * kExpertsPerWarp;
+    // Few token blocks: the dot products of an expert pair are split over dsplit warps (a
+    // shorter chain per warp, at least 512 columns each) while one-pass CTAs would still
+    // fill at most half the GPU
+    int dsplit = 1;
+    while (dsplit < 8 && a.D / (2 * dsplit) >= 512 &&
+           2ll * n_tb * ceil_div(rows_total, (kRouterThreads / 32 / dsplit) * kExpertsPerWarp) <=
+               num_sms)
+        dsplit *= 2;
+    const int rows_per_pass = (kRouterThreads / 32 / dsplit) * kExpertsPerWarp;
     // split the experts so that the grid covers about one wave of the GPU
     int n_eb = ceil_div(num_sms, n_tb);
     n_eb = max(1, min(n_eb, ceil_div(rows_total, rows_per_pass)));
@@ -383,7 +414,7 @@ cudaError_t launch_router(const RouterLaunch& a, int num_sms, cudaStream_t s, bo
     cudaError_t err = set_smem_limit(reinterpret_cast<const void*>(router_kernel), smem);
     if (err != cudaSuccess) return err;
     err = launch_kernel(router_kernel, dim3(n_tb, n_eb), dim3(kRouterThreads), smem, s, pdl, a,
-                        per_cta);
+                        per_cta, dsplit);
     count_launches(1);
     return err;
 }
