@@ -265,6 +265,7 @@ __device__ __forceinline__ int slice_begin(int nk, int nsplit, int slice) {
 }
 __device__ __forceinline__ int choose_split(int tiles, int ctas, int nk, int smax) {
     int best = 1;
+    if (tiles <= 0) return best;
     long long best_cost = static_cast<long long>((tiles + ctas - 1) / ctas) * (nk + kSplitRampSteps);
     for (int s = 2; s <= smax && s <= kSplitSlicesMax; ++s) {
         if (nk / s < kSplitMinSteps) break;
@@ -278,12 +279,33 @@ __device__ __forceinline__ int choose_split(int tiles, int ctas, int nk, int sma
     return best;
 }
 
-// Slices per tile for this launch (host-fixed ksplit, else chosen on the device).
-__device__ __forceinline__ int tile_split(const Params& p, int tiles, bool gate_up) {
-    if (p.ksplit > 1) return p.ksplit;
-    if (p.ksplit_max <= 1 || tiles == 0) return 1;
-    if (gate_up && (p.part == nullptr || p.tickets == nullptr || tiles > p.ticket_cap)) return 1;
-    return choose_split(tiles, gridDim.x, p.nk, p.ksplit_max);
+// Work units of a launch: tiles [0, full) whole, then each remaining tile cut into s K
+// slices, the slice varying fastest.  A host-fixed ksplit cuts every tile.  Otherwise,
+// with fewer tiles than two waves of the grid, every tile is cut into the slices
+// choose_split picks; with more, the tiles of the full waves stay whole and only the last,
+// partial wave's tiles are cut, so that the tail of the launch is shared by more CTAs
+// (measured: cutting every tile was faster below two waves, cutting the tail above).
+struct Units {
+    int full, s, total;
+};
+struct Unit {
+    int tile, slice, nsl;
+};
+__device__ __forceinline__ Units plan_units(const Params& p, int tiles, bool gate_up) {
+    if (p.ksplit > 1) return {0, p.ksplit, tiles * p.ksplit};
+    Units w{tiles, 1, tiles};
+    if (p.ksplit_max <= 1 || tiles == 0) return w;
+    if (gate_up && (p.part == nullptr || p.tickets == nullptr || tiles > p.ticket_cap)) return w;
+    const int ctas = gridDim.x;
+    const int whole = tiles < 2 * ctas ? 0 : (tiles / ctas) * ctas;
+    const int s = choose_split(tiles - whole, ctas, p.nk, p.ksplit_max);
+    if (s > 1) w = {whole, s, whole + (tiles - whole) * s};
+    return w;
+}
+__device__ __forceinline__ Unit unit_at(const Units& w, int u) {
+    if (u < w.full) return {u, 0, 1};
+    const int v = u - w.full;
+    return {w.full + v / w.s, v % w.s, w.s};
 }
 
 // gate_up split: once every epilogue thread has written its partial sums of the tile, one
@@ -399,8 +421,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
     const uint32_t tmem_base = *tmem_slot;
     // units: (group tile, K slice) with the slice varying fastest, so that CTAs working at
     // the same time read different K ranges of the weights
-    const int nsplit = tile_split(p, *total_slot, GATE_UP);
-    const int total = *total_slot * nsplit;
+    const Units units = plan_units(p, *total_slot, GATE_UP);
+    const int total = units.total;
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
@@ -416,9 +438,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
             uint32_t phase = 0, filled = 0, fill_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const Tile t = decode_tile(tile / nsplit, g_tile, g_off, p.G, BN);
-                const int kb = slice_begin(p.nk, nsplit, tile % nsplit);
-                const int ke = slice_begin(p.nk, nsplit, tile % nsplit + 1);
+                const Unit un = unit_at(units, tile);
+                const Tile t = decode_tile(un.tile, g_tile, g_off, p.G, BN);
+                const int kb = slice_begin(p.nk, un.nsl, un.slice);
+                const int ke = slice_begin(p.nk, un.nsl, un.slice + 1);
                 const int wr0 = t.g * p.w_group_rows + t.i * kBM;
                 RowGather<BN> rg;
                 if (gather) rg.plan(p.gather_tok, t.row0, t.row_end, p.nk * kBK, lane);
@@ -476,8 +499,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + abuf * C::kAccCols;
                 constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
-                const int nks = slice_begin(p.nk, nsplit, tile % nsplit + 1) -
-                                slice_begin(p.nk, nsplit, tile % nsplit);
+                const Unit un = unit_at(units, tile);
+                const int nks = slice_begin(p.nk, un.nsl, un.slice + 1) -
+                                slice_begin(p.nk, un.nsl, un.slice);
                 for (int kk = 0; kk < nks; ++kk) {
                     if (!mbar_wait(&full[stage], phase, kWaitBudgetNs, abort_flag)) {
                         set_status(p.status, MOE_ERR_TIMEOUT);
@@ -519,12 +543,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
         if (GATE_UP) clear_accumulator(p, threadIdx.x - 64, kEpiThreads);
         uint32_t abuf = 0, aphase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const Tile t = decode_tile(tile / nsplit, g_tile, g_off, p.G, BN);
-            float* y_slice = p.y_out ? p.y_out + (tile % nsplit) * p.split_stride : nullptr;
+            const Unit un = unit_at(units, tile);
+            const Tile t = decode_tile(un.tile, g_tile, g_off, p.G, BN);
+            float* y_slice = p.y_out ? p.y_out + un.slice * p.split_stride : nullptr;
             // gate_up cut into slices: this slice's partial sums, [row][gate f | up f]
-            float* part = (GATE_UP && nsplit > 1)
-                              ? p.part + static_cast<size_t>(tile % nsplit) * p.part_rows * 2 * p.out_cols
+            float* part = (GATE_UP && un.nsl > 1)
+                              ? p.part + static_cast<size_t>(un.slice) * p.part_rows * 2 * p.out_cols
                               : nullptr;
+            const int nsplit = un.nsl;
             const bool ready = mbar_wait(&tfull[abuf], aphase, kWaitBudgetNs, abort_flag);
             if (!epilogue_bar_and(ready)) {
                 set_status(p.status, MOE_ERR_TIMEOUT);
@@ -572,7 +598,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
             if (abuf == 0) aphase ^= 1u;
             // the slice that completes the tile: sum the slices' partial sums in slice
             // order, then SwiGLU into h
-            if (GATE_UP && part && split_tile_done<kEpiThreads>(p, tile / nsplit, nsplit, 64)) {
+            if (GATE_UP && part && split_tile_done<kEpiThreads>(p, un.tile, nsplit, 64)) {
                 // 4 rows' partial sums in flight at a time
                 const int row_hi = min(t.row0 + BN, t.row_end);
 #pragma unroll 1
@@ -937,8 +963,8 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     // units: (tile, K slice), the slice varying fastest
-    const int nsplit = tile_split(p, *total_slot, GATE_UP);
-    const int total = *total_slot * nsplit;
+    const Units units = plan_units(p, *total_slot, GATE_UP);
+    const int total = units.total;
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
@@ -951,9 +977,10 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
             uint32_t phase = 0, filled = 0, fill_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const Tile t = decode_tile(tile / nsplit, g_tile, g_off, p.G, kTmRows);
-                const int kb = slice_begin(p.nk, nsplit, tile % nsplit);
-                const int ke = slice_begin(p.nk, nsplit, tile % nsplit + 1);
+                const Unit un = unit_at(units, tile);
+                const Tile t = decode_tile(un.tile, g_tile, g_off, p.G, kTmRows);
+                const int kb = slice_begin(p.nk, un.nsl, un.slice);
+                const int ke = slice_begin(p.nk, un.nsl, un.slice + 1);
                 // gate_up: gate rows g*2f + i*128 and up rows g*2f + f + i*128;
                 // down: rows g*D + i*256 and the next 128
                 const int wr0 = t.g * p.w_group_rows + t.i * (GATE_UP ? kBM : kTmN);
@@ -1011,8 +1038,9 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
                 }
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + abuf * C::kAccCols;
-                const int nks = slice_begin(p.nk, nsplit, tile % nsplit + 1) -
-                                slice_begin(p.nk, nsplit, tile % nsplit);
+                const Unit un = unit_at(units, tile);
+                const int nks = slice_begin(p.nk, un.nsl, un.slice + 1) -
+                                slice_begin(p.nk, un.nsl, un.slice);
                 for (int kk = 0; kk < nks; ++kk) {
                     if (!mbar_wait(&full[stage], phase, kWaitBudgetNs, abort_flag)) {
                         set_status(p.status, MOE_ERR_TIMEOUT);
@@ -1049,7 +1077,8 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
         if (GATE_UP) clear_accumulator(p, threadIdx.x - 64, kTmEpiThreads);
         uint32_t abuf = 0, aphase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const Tile t = decode_tile(tile / nsplit, g_tile, g_off, p.G, kTmRows);
+            const Unit un = unit_at(units, tile);
+            const Tile t = decode_tile(un.tile, g_tile, g_off, p.G, kTmRows);
             const bool ready = mbar_wait(&tfull[abuf], aphase, kWaitBudgetNs, abort_flag);
             if (!epilogue_bar_and<kTmEpiThreads>(ready)) {
                 set_status(p.status, MOE_ERR_TIMEOUT);
@@ -1063,8 +1092,8 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
             const bool valid = row < t.row_end;
             const int half = (warp - 2) >> 2;
             // gate_up cut into slices: this slice's partial sums, [row][gate f | up f]
-            float* part = (GATE_UP && nsplit > 1)
-                              ? p.part + static_cast<size_t>(tile % nsplit) * p.part_rows * 2 * p.out_cols
+            float* part = (GATE_UP && un.nsl > 1)
+                              ? p.part + static_cast<size_t>(un.slice) * p.part_rows * 2 * p.out_cols
                               : nullptr;
             tm_epilogue<GATE_UP>(p, tbase, row, valid, t.i, half,
                                  GATE_UP ? nullptr : epi_stage(g_tile + p.G + 1, warp), kTmN, part);
@@ -1074,9 +1103,9 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
             if (abuf == 0) aphase ^= 1u;
             // the slice that completes the tile sums the slices' partial sums in slice
             // order and applies SwiGLU
-            if (GATE_UP && part && split_tile_done<kTmEpiThreads>(p, tile / nsplit, nsplit, 64))
+            if (GATE_UP && part && split_tile_done<kTmEpiThreads>(p, un.tile, un.nsl, 64))
                 split_fixup_tile<kTmEpiThreads>(p, t.row0, min(t.row0 + kTmRows, t.row_end),
-                                                t.i * (kTmN / 2), kTmN / 2, nsplit,
+                                                t.i * (kTmN / 2), kTmN / 2, un.nsl,
                                                 threadIdx.x - 64);
         }
     }
