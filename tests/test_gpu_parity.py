@@ -251,8 +251,12 @@ def test_layer_matches_oracle(moe, oracle_mod, name):
     print(name, rep)
 
 
+# decode (its last wave's gate_up tiles), deep_gate_up, decode_concentrated (every tile) and
+# single_token (weights on M) cut gate_up tiles into K slices: the slices' partial sums are
+# added in slice order, so the fixed-order mode stays bit-for-bit repeatable
 @pytest.mark.parametrize("name", ["tiny", "decode", "shared_small", "ragged_T", "deep_gate_up",
-                                  "deep_down", "deep_shared", "shared_fused"])
+                                  "deep_down", "deep_shared", "shared_fused",
+                                  "decode_concentrated", "single_token"])
 def test_layer_deterministic_mode(moe, oracle_mod, name):
     inp = make_inputs(SMALL_LAYERS[name]).to("cuda")
     layer, y1, idx, w, _ = _run_layer(moe, inp, deterministic=True)
