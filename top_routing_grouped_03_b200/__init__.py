@@ -332,6 +332,7 @@ class MoELayer:
         self.min_capacity = int(min_capacity)
         self._ws = None
         self._ws_T = -1
+        self._copy_streams = None
 
     @classmethod
     def from_inputs(cls, inp, deterministic=False, **router):
@@ -393,6 +394,48 @@ class MoELayer:
         self(x_dev, out=y_dev, stream=stream)
         y_host.copy_(y_dev, non_blocking=True)
         return y_host
+
+    def forward_host_stream(self, x_hosts, y_hosts, x_devs, y_devs, stream=None):
+        """End to end for a sequence of batches from host memory, each batch's copies
+        overlapping the layer on its neighbours: batch i's x (pinned host) goes in on a copy
+        stream while batch i-1 runs, its y comes back to pinned host memory on another copy
+        stream while batch i+1 runs.  x_devs and y_devs hold two device buffers each (used
+        in turn).  The layer runs on `stream` (default: the current stream), which at the end
+        waits for the last copy out; returns y_hosts."""
+        cur = torch.cuda.current_stream() if stream is None else stream
+        if self._copy_streams is None:
+            self._copy_streams = (torch.cuda.Stream(device=cur.device),
+                                  torch.cuda.Stream(device=cur.device))
+        h2d, d2h = self._copy_streams
+        start = torch.cuda.Event()
+        start.record(cur)
+        h2d.wait_event(start)
+        d2h.wait_event(start)
+        ran, out = [], []
+        for i, (xh, yh) in enumerate(zip(x_hosts, y_hosts)):
+            b = i % 2
+            with torch.cuda.stream(h2d):
+                if i >= 2:
+                    h2d.wait_event(ran[i - 2])  # the layer is done with x buffer b
+                x_devs[b].copy_(xh, non_blocking=True)
+                arrived = torch.cuda.Event()
+                arrived.record(h2d)
+            cur.wait_event(arrived)
+            if i >= 2:
+                cur.wait_event(out[i - 2])  # y buffer b has been copied out
+            self(x_devs[b], out=y_devs[b], stream=cur)
+            done = torch.cuda.Event()
+            done.record(cur)
+            ran.append(done)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(done)
+                yh.copy_(y_devs[b], non_blocking=True)
+                copied = torch.cuda.Event()
+                copied.record(d2h)
+            out.append(copied)
+        if out:
+            cur.wait_event(out[-1])
+        return y_hosts
 
     def device_status(self, stream=None) -> int:
         return read_device_status(self._ws, stream) if self._ws is not None else 0
