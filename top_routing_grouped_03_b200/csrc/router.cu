@@ -52,12 +52,19 @@ __device__ __forceinline__ void select_topk_nv(const float* lg, int planes, size
                                                const float* select_bias, int bf16_weights) {
     float v[NV];  // logits (+ the logit bias)
 #pragma unroll
+    for (int j = 0; j < NV; ++j) v[j] = 0.f;
+    // plane by plane, each plane's NV loads in flight together; planes added in order
+    for (int q = 0; q < planes; ++q) {
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const int e = j * 32 + lane;
+            if (e < E) v[j] += __ldcg(lg + q * plane_stride + e);
+        }
+    }
+#pragma unroll
     for (int j = 0; j < NV; ++j) {
         const int e = j * 32 + lane;
-        float r = 0.f;
-        if (e < E)
-            for (int q = 0; q < planes; ++q) r += __ldcg(lg + q * plane_stride + e);
-        v[j] = (e < E) ? r + (add_bias ? __ldg(add_bias + e) : 0.f) : -FLT_MAX;
+        v[j] = (e < E) ? v[j] + (add_bias ? __ldg(add_bias + e) : 0.f) : -FLT_MAX;
     }
     // scores and selection keys.  Softmax without selection bias: the key is the logit
     // itself (softmax is increasing) and only the K selected terms are exponentiated.
