@@ -659,9 +659,12 @@ constexpr int kTmThreads = 64 + 256;
 constexpr int kTmEpiThreads = 256;
 
 
+// Reductions into the fp32 accumulator keep its lines in L2 (evict-last) while the expert
+// weights stream through (evict-first).
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-                 "f"(c), "f"(d)
+    const uint64_t pol = policy_evict_last();
+    asm volatile("red.global.add.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(addr),
+                 "f"(a), "f"(b), "f"(c), "f"(d), "l"(pol)
                  : "memory");
 }
 
