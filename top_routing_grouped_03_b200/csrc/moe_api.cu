@@ -99,7 +99,8 @@ Layout layout(long long T, long long D, long long E, long long K, long long f, l
     L.counts = take(sizeof(int32_t) * E);
     L.tickets = take(sizeof(unsigned) * gate_up_ticket_cap(T, E, K, f));
     L.zero_end = o;
-    // depends on T, E and K only, so any workspace sized for the same T, E, K has it here
+    // its offset depends on T, E, K and (through the split tickets) f; the single-step entry
+    // points all lay the workspace out with f = 128, so they agree with each other
     L.perm_hist = take(sizeof(int32_t) * E * permute_chunks(T * K));
     // router logits: [T, E+1] (CUDA-core router) or partial-sum planes of [T, E]
     L.logits = take(sizeof(float) * T *
