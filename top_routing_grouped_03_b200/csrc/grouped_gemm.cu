@@ -327,6 +327,29 @@ __device__ __forceinline__ bool split_tile_done(const Params& p, int tile, int n
     return epilogue_bar_and<kThreads>(last);
 }
 
+// The one-CTA tokens-on-M kernel shares the fix-up among the tile's slices instead: each
+// slice posts its ticket, waits (bounded) until all nsplit slices have posted -- the grid
+// is persistent with at most one CTA per SM, so the tile's other slices are resident or
+// will run once earlier work leaves the SMs, and a slice posts before it waits -- and then
+// fixes up its own share of the tile's rows.  False on a wait that ran out of time.
+template <int kThreads>
+__device__ __forceinline__ bool split_tile_all_posted(const Params& p, int tile, int nsplit,
+                                                      int first_epi_tid) {
+    epilogue_bar_and<kThreads>(true);
+    bool ok = true;
+    if (threadIdx.x == first_epi_tid) {
+        atom_add_acq_rel_gpu(p.tickets + tile, 1u);
+        const uint64_t t0 = global_timer_ns();
+        while (ld_acquire_gpu(p.tickets + tile) < static_cast<unsigned>(nsplit)) {
+            if (global_timer_ns() - t0 > kWaitBudgetNs) {
+                ok = false;
+                break;
+            }
+        }
+    }
+    return epilogue_bar_and<kThreads>(ok);
+}
+
 // Per-lane plan for gathering ROWS token rows of x into a 128-byte-swizzled operand tile
 // with cp.async: lane l owns 16-byte chunk c = l % 8 of tile rows l/8 + 4u; that chunk of
 // tile row r lands at r*128 + ((c ^ (r % 8)) * 16).
@@ -714,17 +737,21 @@ __device__ __forceinline__ void reduce16_transposed(const Params& p, const uint3
     __syncwarp();
 }
 
-// gate_up cut into K slices, the CTA whose slice completed the tile: h[row, feat0 + j] for
-// the tile's rows [row0, row_end) and its F features, from the slices' partial sums added
-// in slice order.  The epilogue threads share (row, 8-feature chunk) items, so that a tile
-// of a few rows costs one round trip to L2.
+// gate_up cut into K slices, slice `share` of nsplit once all slices have posted:
+// h[row, feat0 + j] for its share of the (row, 8-feature chunk) items of the tile's rows
+// [row0, row_end) and F features, from the slices' partial sums added in slice order.  The
+// epilogue threads share the items, so that a share of a few rows costs one round trip to
+// L2.
 template <int kThreads>
 __device__ __forceinline__ void split_fixup_tile(const Params& p, int row0, int row_end,
-                                                 int feat0, int F, int nsplit, int epi_tid) {
+                                                 int feat0, int F, int nsplit, int share,
+                                                 int epi_tid) {
     const int chunks = F / 8;
     const int items = (row_end - row0) * chunks;
+    const int it_end = static_cast<int>(static_cast<long long>(items) * (share + 1) / nsplit);
 #pragma unroll 1
-    for (int it = epi_tid; it < items; it += kThreads) {
+    for (int it = static_cast<int>(static_cast<long long>(items) * share / nsplit) + epi_tid;
+         it < it_end; it += kThreads) {
         const int row = row0 + it / chunks;
         const int f = feat0 + (it % chunks) * 8;
         float4 a[kSplitSlicesMax][2], b[kSplitSlicesMax][2];
@@ -1104,12 +1131,16 @@ grouped_gemm_tm_kernel(const __grid_constant__ CUtensorMap map_w,
             mbar_arrive(&tempty[abuf]);
             abuf ^= 1u;
             if (abuf == 0) aphase ^= 1u;
-            // the slice that completes the tile sums the slices' partial sums in slice
-            // order and applies SwiGLU
-            if (GATE_UP && part && split_tile_done<kTmEpiThreads>(p, un.tile, un.nsl, 64))
-                split_fixup_tile<kTmEpiThreads>(p, t.row0, min(t.row0 + kTmRows, t.row_end),
-                                                t.i * (kTmN / 2), kTmN / 2, un.nsl,
-                                                threadIdx.x - 64);
+            // every slice of the tile, once all have posted, sums its share of the rows'
+            // partial sums in slice order and applies SwiGLU
+            if (GATE_UP && part) {
+                if (split_tile_all_posted<kTmEpiThreads>(p, un.tile, un.nsl, 64))
+                    split_fixup_tile<kTmEpiThreads>(p, t.row0, min(t.row0 + kTmRows, t.row_end),
+                                                    t.i * (kTmN / 2), kTmN / 2, un.nsl, un.slice,
+                                                    threadIdx.x - 64);
+                else if (threadIdx.x == 64)
+                    set_status(p.status, MOE_ERR_TIMEOUT);
+            }
         }
     }
 
